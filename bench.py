@@ -1,0 +1,394 @@
+#!/usr/bin/env python
+"""Benchmark of one MLA decode layer-step through libmla's C ABI on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl mla|reference]
+
+A step is one pass of the whole hot path over one batch: append the new token's latent row,
+absorb the query, latent attention over every cached token, output projection (for the
+12-layer running-model workload: all 12 layers). Inputs (weights, caches, new hidden states)
+are seeded synthetic data resident in HBM before timing. With N > 1 (torchrun, one process per
+GPU) every rank runs its own replica of the workload: sequences are independent, so there is no
+data-path collective; ``value`` aggregates the ranks and the time is the max over ranks.
+
+One JSON line on rank 0. ``value`` is µs per layer-step of the whole job (step time divided by
+layers and by N). ``e2e`` is the same metric with host buffers: the step's inputs copied from
+pinned host memory and its output copied back inside the timed region. ``roofline`` reports
+the dominant call, mla_decode_attention, against max(bytes / HBM, flops / tensor peak) with the
+measured peaks. ``cpu_baseline`` times the fp64 oracle on a bounded sample (rank 0, N = 1).
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "MLA absorbed decode µs/layer, TFLOP/s & latent-cache GB/s vs B200 roofline"
+UNIT = "us/layer-step"
+DEFAULT_WORKLOAD = "production_b64_n4096_bf16"
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+
+def load_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            j = json.load(f)
+        return j, "measured"
+    return dict(FALLBACK_PEAKS), "fallback"
+
+
+def dims_desc(d):
+    return (f"d={d.d_model}, n_h={d.n_heads}, d_h={d.d_head}, d_c={d.d_c}, d_c'={d.d_cq}, d_R={d.d_rope}, "
+            f"page={d.page_size}")
+
+
+# ----------------------------------------------------------------------------------- clocks
+class ClockSampler:
+    """nvidia-smi samples of SM clock and throttle reasons while the timed region runs."""
+
+    FIELDS = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,clocks_event_reasons.hw_slowdown,"
+              "clocks_event_reasons.hw_thermal_slowdown,clocks_event_reasons.sw_thermal_slowdown,"
+              "clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_id: str):
+        self.gpu_id = gpu_id
+        self.samples = []
+        self.proc = None
+        self.thread = None
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", self.gpu_id, f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                 "-lms", "50"], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except (OSError, ValueError):
+            self.proc = None
+            return
+        self.thread = threading.Thread(target=self._read, daemon=True)
+        self.thread.start()
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.samples.append((time.time(), line.strip()))
+
+    def stop(self):
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+            self.thread.join(timeout=5)
+
+    def summary(self, t0, t1):
+        rows = []
+        for ts, line in self.samples:
+            parts = [p.strip() for p in line.split(",")]
+            if len(parts) < 8:
+                continue
+            rows.append((ts, parts))
+        inside = [r for r in rows if t0 <= r[0] <= t1] or rows
+        if not inside:
+            return None
+        sm = [float(p[0]) for _, p in inside if p[0].replace(".", "").isdigit()]
+        mx = [float(p[1]) for _, p in inside if p[1].replace(".", "").isdigit()]
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[i] for _, p in inside for i in range(4) if p[4 + i].lower() == "active"})
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": max(mx) if mx else None,
+                "reasons": reasons, "samples": len(inside)}
+
+
+# ----------------------------------------------------------------------------------- CPU oracle
+class OracleSample:
+    """A bounded sample of the workload for the fp64 oracle: the first ``n`` sequences of one layer."""
+
+    def __init__(self, w, n, layer=0):
+        import oracle as O
+        from mla_latent_kv_42_b200 import synth
+        self.O, self.w = O, w
+        self.cached = synth.cached_lengths(w)
+        self.W64 = {k: O.as64(v) for k, v in synth.weights(w, layer).items()}
+        self.picks = list(range(min(n, w.batch)))
+        sub = self.cached[self.picks]
+        rows = synth.prefix_rows(w, sub, layer=layer, device="cpu")
+        offs = np.concatenate([[0], np.cumsum(sub)])
+        self.prefix = [O.as64(rows[offs[i]:offs[i + 1]]) for i in range(len(self.picks))]
+        self.h = O.as64(synth.hidden(w))[self.picks]
+        self.frac = float(np.sum(sub + 1)) / float(np.sum(self.cached + 1))
+
+    def run(self, n=None):
+        """Seconds for the naive oracle's layer-step over the first ``n`` sampled sequences."""
+        k = len(self.picks) if n is None else n
+        t = time.perf_counter()
+        self.O.layer_step_naive(self.W64, self.h[:k], self.prefix[:k], self.w.dims)
+        return time.perf_counter() - t
+
+
+def cpu_baseline(w, target_s=12.0):
+    """Time the naive oracle on a bounded sample of whole sequences; extrapolate to the step."""
+    probe = OracleSample(w, 1)
+    t1 = probe.run()
+    n = max(1, min(w.batch, int(target_s / max(t1, 1e-3))))
+    smp = OracleSample(w, n)
+    t = smp.run()
+    cores = len(os.sched_getaffinity(0))
+    attended = int(np.sum(smp.cached[smp.picks] + 1))
+    return {"value": t / smp.frac * 1e6, "unit": UNIT, "cores": cores, "kind": "oracle",
+            "sample": (f"naive fp64 oracle, one layer, {len(smp.picks)} of {w.batch} sequences (all heads, "
+                       f"{attended} attended tokens), extrapolated by attended tokens x{1 / smp.frac:.1f}; "
+                       f"{t:.1f} s of CPU time")}
+
+
+def run_reference(args):
+    """The reference arm: the fp64 oracle as it stands, on the host cores (rank 0 only)."""
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return 0
+    from mla_latent_kv_42_b200 import synth
+    w = synth.workload(args.workload)
+    smp = OracleSample(w, 1)
+    cached = smp.cached
+    per = []
+    for i in range(args.warmup + args.steps):
+        t = smp.run()
+        if i >= args.warmup:
+            per.append(t / smp.frac)
+    us = float(np.mean(per)) * 1e6
+    cores = len(os.sched_getaffinity(0))
+    sample = (f"naive fp64 oracle on sequence 0 of {w.batch} each step (all heads, {int(cached[0]) + 1} attended "
+              f"tokens), extrapolated by attended tokens to the whole batch")
+    line = {
+        "impl": "reference", "metric": METRIC, "value": us, "unit": UNIT, "n_gpus": args.gpus, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": us * w.layers / 1e3, "higher_is_better": False, "scaling": "weak",
+        "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": w.name, "batch": w.batch, "layers": w.layers, "dims": dims_desc(w.dims)},
+        "cpu_baseline": {"value": us, "unit": UNIT, "cores": cores, "kind": "oracle", "sample": sample},
+        "e2e": {"value": us, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+# ----------------------------------------------------------------------------------- GPU arm
+def run_mla(args):
+    import torch
+    import torch.distributed as dist
+
+    import mla_latent_kv_42_b200 as M
+    from mla_latent_kv_42_b200 import build, harness, synth
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world != args.gpus:
+        raise SystemExit(f"--gpus {args.gpus} but WORLD_SIZE={world}")
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if world > 1:
+        import datetime
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=dev)
+    if rank == 0 or not os.path.exists(M.library_path()):
+        build.build()
+    if world > 1:
+        dist.barrier()
+    M.load_library()
+
+    w = synth.workload(args.workload)
+    d = w.dims
+    cached = synth.cached_lengths(w)
+    ix = harness.step_index(cached, device=dev)
+    layers = [harness.make_layer(w, cached, layer=l, device=dev) for l in range(w.layers)]
+    B = w.batch
+    h0 = synth.hidden(w).to(dev)
+    h = h0.clone()
+    ws = torch.empty(M.step_workspace_bytes(d, B, ix.max_seq_len), dtype=torch.uint8, device=dev)
+    e = synth.storage_dtype(d)
+    outs = [{"q": torch.empty((B, d.n_heads, d.D), dtype=e, device=dev),
+             "o_lat": torch.empty((B, d.n_heads, d.d_c), dtype=e, device=dev),
+             "lse": torch.empty((B, d.n_heads), dtype=torch.float32, device=dev),
+             "u": torch.empty((B, d.d_model), dtype=e, device=dev)} for _ in layers]
+    stream = torch.cuda.current_stream(dev)
+    EV = lambda: torch.cuda.Event(enable_timing=True)
+    call_ms = np.zeros(4)
+    launches = [0]
+
+    def one_step(record=False):
+        x = h
+        for L, o in zip(layers, outs):
+            st, w_ = L.state, L.state.w
+            if record:
+                ev = [EV() for _ in range(5)]
+                ev[0].record(stream)
+            M.append_kv(d, x, w_["w_dkv_kr"], ix.seq_idx, ix.pos, st.block_table, st.pool, ws=ws, stream=stream)
+            n = M.last_launch_count(0)
+            if record:
+                ev[1].record(stream)
+            M.absorb_query(d, x, w_["w_dq"], w_["w_uq_qr"], w_["w_uk"], ix.pos, q_out=o["q"], ws=ws, stream=stream)
+            n += M.last_launch_count(1)
+            if record:
+                ev[2].record(stream)
+            M.decode_attention(d, o["q"], st.pool, st.block_table, ix.seq_lens, ix.max_seq_len, o_lat=o["o_lat"],
+                               lse=o["lse"], ws=ws, stream=stream)
+            n += M.last_launch_count(2)
+            if record:
+                ev[3].record(stream)
+            M.out_proj(d, o["o_lat"], w_["w_uv"], w_["w_o"], u=o["u"], ws=ws, stream=stream)
+            n += M.last_launch_count(3)
+            if record:
+                ev[4].record(stream)
+                pending.append(ev)
+            launches[0] += n
+            if len(layers) > 1:
+                x = x + o["u"]          # residual between layers (harness glue, torch)
+        return o["u"]
+
+    pending = []
+    for _ in range(args.warmup):
+        one_step()
+    torch.cuda.synchronize(dev)
+    assert M.read_device_status(stream) == 0
+
+    gpu_uuid = str(getattr(torch.cuda.get_device_properties(dev), "uuid", local))
+    if gpu_uuid and not gpu_uuid.startswith("GPU-") and len(gpu_uuid) == 36:
+        gpu_uuid = "GPU-" + gpu_uuid
+    sampler = ClockSampler(gpu_uuid if gpu_uuid else str(local))
+    sampler.start()
+    time.sleep(0.3)
+
+    # ---- timed region: K steps, device time, barrier + synchronize on both sides
+    launches[0] = 0
+    pending.clear()
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize(dev)
+    t_wall0 = time.time()
+    start, end = EV(), EV()
+    start.record(stream)
+    for _ in range(args.steps):
+        one_step(record=True)
+    end.record(stream)
+    torch.cuda.synchronize(dev)
+    t_wall1 = time.time()
+    if world > 1:
+        dist.barrier()
+    ms_total = start.elapsed_time(end)
+    for ev in pending:
+        for c in range(4):
+            call_ms[c] += ev[c].elapsed_time(ev[c + 1])
+    gpu_launches = launches[0]
+    n_layer_steps = args.steps * len(layers)
+    call_ms /= n_layer_steps
+
+    # ---- e2e: host buffers through the public API (pinned h in, u out, inside the timed region)
+    h_host = h0.cpu().pin_memory()
+    pos_host = ix.pos.cpu().pin_memory()
+    lens_host = ix.seq_lens.cpu().pin_memory()
+    u_host = torch.empty((B, d.d_model), dtype=e).pin_memory()
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize(dev)
+    s2, e2 = EV(), EV()
+    s2.record(stream)
+    for _ in range(args.steps):
+        h.copy_(h_host, non_blocking=True)
+        ix.pos.copy_(pos_host, non_blocking=True)
+        ix.seq_lens.copy_(lens_host, non_blocking=True)
+        u = one_step()
+        u_host.copy_(u, non_blocking=True)
+    e2.record(stream)
+    torch.cuda.synchronize(dev)
+    if world > 1:
+        dist.barrier()
+    ms_e2e = s2.elapsed_time(e2)
+    sampler.stop()
+    assert M.read_device_status(stream) == 0
+
+    # max over ranks
+    t = torch.tensor([ms_total, ms_e2e, call_ms[2]], dtype=torch.float64, device=dev)
+    if world > 1:
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    ms_total, ms_e2e, decode_ms = t.tolist()
+
+    if rank == 0:
+        peaks, peak_src = load_peaks()
+        ms_step = ms_total / args.steps
+        us_layer_job = ms_step * 1e3 / len(layers) / world
+        us_e2e_job = ms_e2e / args.steps * 1e3 / len(layers) / world
+        seq_lens = cached + 1
+        dbytes, dflops = harness.decode_work(d, seq_lens)
+        sbytes, sflops = harness.step_work(d, seq_lens)
+        dec_s = decode_ms * 1e-3
+        t_mem = dbytes / (peaks["hbm_gbs"] * 1e9)
+        t_flop = dflops / (peaks["bf16_tflops"] * 1e12)
+        if t_mem >= t_flop:
+            roof = {"bound": "hbm", "achieved": dbytes / dec_s / 1e9, "peak": peaks["hbm_gbs"], "unit": "GB/s"}
+        else:
+            roof = {"bound": "tensor", "achieved": dflops / dec_s / 1e12, "peak": peaks["bf16_tflops"],
+                    "unit": "TFLOP/s"}
+        roof["frac"] = roof["achieved"] / roof["peak"]
+        roof["traffic"] = None
+        roof["kernel"] = "mla_decode_attention"
+        roof["peak_source"] = peak_src + " (burst; MEASURED_PEAKS.json)" if peak_src == "measured" else peak_src
+        roof["roofline_us"] = max(t_mem, t_flop) * 1e6
+        roof["algorithmic_bytes"] = dbytes
+        roof["algorithmic_flops"] = dflops
+        step_s = ms_step * 1e-3 / len(layers)
+        line = {
+            "metric": METRIC, "value": us_layer_job, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": False, "scaling": "weak",
+            "vs_baseline": None, "dtype": "bf16" if d.dtype == "bf16" else "fp16", "data": "synthetic",
+            "config": {"workload": w.name, "batch": B, "cached_tokens": (int(cached[0]) if not w.ragged else
+                                                                         f"U[{w.cached[0]},{w.cached[1]}], sum "
+                                                                         f"{int(cached.sum())}"),
+                       "layers": len(layers), "dims": dims_desc(d), "paging": w.paging,
+                       "l2": "inputs larger than L2" if sbytes > 126e6 else "L2 not flushed (inputs below L2)",
+                       "parallelism": f"replicas x{world} (sequence-independent, no collective)"},
+            "tflops": sflops / step_s / 1e12,
+            "cache_gbs": dbytes / dec_s / 1e9,
+            "decode_us": decode_ms * 1e3,
+            "per_call_us": {"append_kv": call_ms[0] * 1e3, "absorb_query": call_ms[1] * 1e3,
+                            "decode_attention": call_ms[2] * 1e3, "out_proj": call_ms[3] * 1e3},
+            "layer_step_roofline_us": max(sbytes / (peaks["hbm_gbs"] * 1e9), sflops / (peaks["bf16_tflops"] * 1e12))
+            * 1e6,
+            "roofline": roof,
+            "e2e": {"value": us_e2e_job, "unit": UNIT, "h2d_bytes_per_step": int(h0.numel() * 2 + 2 * B * 4),
+                    "d2h_bytes_per_step": int(B * d.d_model * 2)},
+            "gpu_launches": int(gpu_launches),
+            "clocks": sampler.summary(t_wall0 - 0.1, t_wall1 + 0.1),
+        }
+        if world == 1 and not args.no_cpu_baseline:
+            line["cpu_baseline"] = cpu_baseline(w)
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+    return 0
+
+
+def main():
+    ap = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawDescriptionHelpFormatter)
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--workload", default=DEFAULT_WORKLOAD)
+    ap.add_argument("--impl", choices=["mla", "reference"], default="mla")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    args.warmup = max(3, args.warmup)     # at least 3 untimed warm-up steps
+    if args.impl == "reference":
+        return run_reference(args)
+    return run_mla(args)
+
+
+if __name__ == "__main__":
+    sys.exit(main())

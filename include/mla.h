@@ -1,0 +1,170 @@
+/*
+ * mla.h — C ABI of libmla: Multi-head Latent Attention (DeepSeek-V2) at decode time, in its
+ * weight-absorbed form, on NVIDIA B200 (sm_100a).
+ *
+ * Method source: "DeepSeek-V2 from Scratch: Multi-head Latent Attention and DeepSeekMoE",
+ * §2 (joint KV compression), §4 (decoupled RoPE), §5 (matrix absorption), §6 (the complete
+ * algorithm). Notation: d = d_model, n_h heads of d_h, KV latent d_c, query latent d_c'
+ * (d_cq), decoupled RoPE width d_h^R (d_rope). One cache row is [c^KV (d_c) ‖ k^R (d_rope)].
+ *
+ * Conventions for every call
+ *   - Matrices follow the pages' y = W x convention: W is [out, in], row-major. Head i of
+ *     W^UQ / W^UK / W^UV is the contiguous row block [i*d_h, (i+1)*d_h); head i of W^QR the
+ *     row block [i*d_rope, (i+1)*d_rope); head i of W^O its column block [i*d_h, (i+1)*d_h).
+ *   - Element type of every activation, weight and cache buffer is dims->dtype (bf16 or
+ *     fp16); accumulation is fp32. Results are rounded to the element type to nearest even.
+ *   - RoPE rotates adjacent pairs (x[2k], x[2k+1]) by the angle pos * rope_base^(-2k/d_rope),
+ *     formed in double precision; positions are 0-based.
+ *   - Ownership: the caller owns every buffer. All pointer arguments are DEVICE pointers,
+ *     16-byte aligned, on the current device. The library allocates no device memory and
+ *     keeps no per-call state besides one device status word per device.
+ *   - Asynchrony: work is queued on `stream` (NULL = the legacy default stream) and the call
+ *     returns without synchronising. Calls on different streams may run concurrently if their
+ *     buffers (including workspaces) do not overlap.
+ *   - Errors: calls return MLA_OK (0) or a negative mla_status. Argument checks run before
+ *     anything is queued, so an error return from a check means no work was queued. A launch
+ *     failure returns MLA_ERR_CUDA. Kernels never trap or assert: a bad page id or sequence
+ *     length found on the device is recorded in the device status word (see
+ *     mla_read_device_status) and the offending row is skipped (written as zeros).
+ */
+#ifndef MLA_H_
+#define MLA_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* A CUDA stream (cudaStream_t / CUstream). */
+typedef struct CUstream_st* mla_stream_t;
+
+enum mla_dtype { MLA_BF16 = 0, MLA_FP16 = 1 };
+
+typedef struct mla_dims {
+  int32_t d_model;   /* d */
+  int32_t n_heads;   /* n_h, 1..128 */
+  int32_t d_head;    /* d_h */
+  int32_t d_c;       /* KV latent width */
+  int32_t d_cq;      /* query latent width d_c' */
+  int32_t d_rope;    /* d_h^R, even */
+  int32_t page_size; /* tokens per cache page */
+  int32_t dtype;     /* enum mla_dtype */
+  double rope_base;  /* RoPE frequency base, e.g. 10000 */
+} mla_dims;
+/* The softmax scale is derived, 1/sqrt(d_head + d_rope) (from-scratch page, §4.4). */
+
+enum mla_status {
+  MLA_OK = 0,
+  MLA_ERR_INVALID_ARG = -1,         /* null pointer, negative size, bad enum */
+  MLA_ERR_UNSUPPORTED_DIMS = -2,    /* dims outside what the kernels support (see mla_check_dims) */
+  MLA_ERR_WORKSPACE_TOO_SMALL = -3, /* ws_bytes < mla_workspace_size(...) */
+  MLA_ERR_ALIGNMENT = -4,           /* a pointer is not 16-byte aligned */
+  MLA_ERR_CUDA = -5,                /* a CUDA runtime call or launch failed */
+  MLA_ERR_TIMEOUT = -6,             /* device status: a bounded wait in a kernel gave up */
+  MLA_ERR_BAD_PAGE = -7,            /* device status: block-table entry outside [0, num_pages) */
+  MLA_ERR_BAD_SEQ_LEN = -8          /* device status: seq_len < 1, > max_seq_len or > max_pages*page_size */
+};
+
+enum mla_call {
+  MLA_CALL_APPEND_KV = 0,
+  MLA_CALL_ABSORB_QUERY = 1,
+  MLA_CALL_DECODE_ATTENTION = 2,
+  MLA_CALL_OUT_PROJ = 3
+};
+
+/* Returns MLA_OK if every call supports `dims`, else MLA_ERR_UNSUPPORTED_DIMS or
+ * MLA_ERR_INVALID_ARG. Supported: all widths positive multiples of 8 (d_rope a multiple of 8),
+ * n_heads <= 128, d_c <= 512, d_c + d_rope <= 576, page_size >= 1, dtype bf16/fp16,
+ * rope_base > 0. */
+int mla_check_dims(const mla_dims* dims);
+
+/* Elements cached per token per layer, d_c + d_rope ("What Gets Cached", from-scratch page
+ * §4.5; 160 for the running model, 576 at DeepSeek-V2 dims). Negative on invalid dims. */
+int32_t mla_cache_elems_per_token(const mla_dims* dims);
+
+/* Bytes of workspace the call `call` needs for batch B (tokens T for append) and longest
+ * attended length max_seq_len, on the current device. 0 on invalid arguments. */
+size_t mla_workspace_size(const mla_dims* dims, int32_t call, int32_t B, int32_t max_seq_len);
+
+/*
+ * mla_append_kv — KV pathway and cache write (from-scratch page §2.1 and §4.2, boxed in §6).
+ * For each of the T new tokens t:
+ *   [c ; k^] = W_dkv_kr h_t            (W^DKV rows then W^KR rows, fp32 accumulate)
+ *   k^R = RoPE(k^, pos[t])
+ *   pool row  bt[seq_idx[t]][pos[t] / page_size] * page_size + pos[t] % page_size
+ *        <- [c ‖ k^R] rounded to the element type.
+ * h         [T, d_model]
+ * w_dkv_kr  [d_c + d_rope, d_model]
+ * seq_idx   int32 [T], each in [0, num_seqs)        pos int32 [T], >= 0
+ * block_table int32 [num_seqs, max_pages]; pool [num_pages, page_size, d_c + d_rope]
+ * ws        at least mla_workspace_size(dims, MLA_CALL_APPEND_KV, T, 0) bytes (may be NULL if 0)
+ * A token whose page entry is outside [0, num_pages) or whose pos/page_size >= max_pages is
+ * not written; the device status records MLA_ERR_BAD_PAGE. T == 0 is a no-op.
+ */
+int mla_append_kv(const mla_dims* dims, const void* h, const void* w_dkv_kr,
+                  const int32_t* seq_idx, const int32_t* pos,
+                  const int32_t* block_table, int32_t num_seqs, int32_t max_pages,
+                  void* pool, int32_t num_pages, int32_t T,
+                  void* ws, size_t ws_bytes, mla_stream_t stream);
+
+/*
+ * mla_absorb_query — query pathway with W^UK absorbed (from-scratch page §4.1 and §5.1,
+ * step 1 of §5.3):
+ *   c^Q = W^DQ h;  [q^C ; q^] = [W^UQ ; W^QR] c^Q;  q^R_i = RoPE(q^_i, pos)
+ *   q~_i = (W^UK_i)^T q^C_i
+ *   q_out[b][i] = [q~_i (d_c) ‖ q^R_i (d_rope)]   — the same layout as a cache row.
+ * h [B, d_model]; w_dq [d_cq, d_model]; w_uq_qr [n_heads*(d_head + d_rope), d_cq] (W^UQ rows
+ * then W^QR rows); w_uk [n_heads*d_head, d_c]; pos int32 [B]; q_out [B, n_heads, d_c + d_rope].
+ * c^Q and q^C are rounded to the element type before their next product.
+ */
+int mla_absorb_query(const mla_dims* dims, const void* h, const void* w_dq, const void* w_uq_qr,
+                     const void* w_uk, const int32_t* pos, void* q_out, int32_t B,
+                     void* ws, size_t ws_bytes, mla_stream_t stream);
+
+/*
+ * mla_decode_attention — latent attention (from-scratch page §4.4 with §5.3 steps 2-3):
+ * for every sequence b and head i, over the attended tokens j = 0 .. seq_lens[b]-1
+ *   s_j = (q~_i . c_j + q^R_i . k^R_j) / sqrt(d_head + d_rope)
+ *   p = softmax_j(s);   o_lat[b][i] = sum_j p_j c_j                      (d_c values)
+ *   lse_out[b][i] = log sum_j exp(s_j)   (natural log; skipped if lse_out is NULL)
+ * q [B, n_heads, d_c + d_rope]; pool, block_table as in mla_append_kv (num_seqs = B);
+ * seq_lens int32 [B], 1 <= seq_lens[b] <= max_seq_len, the new token already appended;
+ * o_lat [B, n_heads, d_c] element type; lse_out float [B, n_heads] or NULL.
+ * Long sequences are split across SMs and the partials merged by log-sum-exp; the result is
+ * bitwise reproducible run to run. A bad seq_len or page id zeroes that sequence's output and
+ * records the error in the device status.
+ */
+int mla_decode_attention(const mla_dims* dims, const void* q, const void* pool, int32_t num_pages,
+                         const int32_t* block_table, int32_t max_pages, const int32_t* seq_lens,
+                         int32_t B, int32_t max_seq_len, void* o_lat, float* lse_out,
+                         void* ws, size_t ws_bytes, mla_stream_t stream);
+
+/*
+ * mla_out_proj — output projection with W^UV absorbed (from-scratch page §5.2, step 4 of
+ * §5.3, and u = W^O [o_1; ...; o_n_h] of §6):
+ *   o_i = W^UV_i o_lat_i   (d_head values, rounded to the element type)
+ *   u   = W^O [o_1 ; ... ; o_n_h]
+ * o_lat [B, n_heads, d_c]; w_uv [n_heads*d_head, d_c]; w_o [d_model, n_heads*d_head];
+ * u [B, d_model].
+ */
+int mla_out_proj(const mla_dims* dims, const void* o_lat, const void* w_uv, const void* w_o,
+                 void* u, int32_t B, void* ws, size_t ws_bytes, mla_stream_t stream);
+
+/* Synchronises `stream`, returns the current device's status word in *status_out (MLA_OK or
+ * the first device-side error recorded since the last read) and clears it. */
+int mla_read_device_status(mla_stream_t stream, int32_t* status_out);
+
+/* Static string for a status code. */
+const char* mla_error_string(int code);
+
+/* Number of kernel launches the last successful call of `call` on this thread queued
+ * (for launch accounting in benchmarks). */
+int32_t mla_last_launch_count(int32_t call);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* MLA_H_ */

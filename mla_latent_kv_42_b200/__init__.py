@@ -1,0 +1,246 @@
+"""Python binding of libmla, the MLA absorbed-decode library for B200 (sm_100a).
+
+Argument marshalling only: every step of the path runs in libmla's CUDA kernels, reached
+through the C ABI of ``include/mla.h``. Torch supplies device memory and streams. If the
+shared library is missing, every call raises; there is no fallback of any kind.
+
+Method: "DeepSeek-V2 from Scratch", §6 (the complete MLA algorithm) in the absorbed form of
+§5.3: append the new token's latent row, absorb W^UK into the query, attend in latent space,
+fold W^UV into the output projection.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+from dataclasses import dataclass
+
+__all__ = [
+    "MLAError", "load_library", "library_path", "c_dims", "workspace_size", "cache_elems_per_token",
+    "append_kv", "absorb_query", "decode_attention", "out_proj", "read_device_status", "last_launch_count",
+    "LayerState", "layer_step", "CALL_APPEND_KV", "CALL_ABSORB_QUERY", "CALL_DECODE_ATTENTION", "CALL_OUT_PROJ",
+]
+
+CALL_APPEND_KV, CALL_ABSORB_QUERY, CALL_DECODE_ATTENTION, CALL_OUT_PROJ = 0, 1, 2, 3
+_PKG = os.path.dirname(os.path.abspath(__file__))
+
+
+def library_path() -> str:
+    return os.path.join(_PKG, "libmla.so")
+
+
+class MLAError(RuntimeError):
+    def __init__(self, code: int, what: str):
+        self.code = code
+        super().__init__(f"{what}: {_lib().mla_error_string(code).decode()} ({code})")
+
+
+class _Dims(ctypes.Structure):
+    _fields_ = [("d_model", ctypes.c_int32), ("n_heads", ctypes.c_int32), ("d_head", ctypes.c_int32),
+                ("d_c", ctypes.c_int32), ("d_cq", ctypes.c_int32), ("d_rope", ctypes.c_int32),
+                ("page_size", ctypes.c_int32), ("dtype", ctypes.c_int32), ("rope_base", ctypes.c_double)]
+
+
+_LIB = None
+_P, _I32, _SZ = ctypes.c_void_p, ctypes.c_int32, ctypes.c_size_t
+_SIGS = {
+    "mla_check_dims": (ctypes.c_int, [_P]),
+    "mla_cache_elems_per_token": (_I32, [_P]),
+    "mla_workspace_size": (_SZ, [_P, _I32, _I32, _I32]),
+    "mla_append_kv": (ctypes.c_int, [_P, _P, _P, _P, _P, _P, _I32, _I32, _P, _I32, _I32, _P, _SZ, _P]),
+    "mla_absorb_query": (ctypes.c_int, [_P, _P, _P, _P, _P, _P, _P, _I32, _P, _SZ, _P]),
+    "mla_decode_attention": (ctypes.c_int, [_P, _P, _P, _I32, _P, _I32, _P, _I32, _I32, _P, _P, _P, _SZ, _P]),
+    "mla_out_proj": (ctypes.c_int, [_P, _P, _P, _P, _P, _I32, _P, _SZ, _P]),
+    "mla_read_device_status": (ctypes.c_int, [_P, ctypes.POINTER(_I32)]),
+    "mla_error_string": (ctypes.c_char_p, [ctypes.c_int]),
+    "mla_last_launch_count": (_I32, [_I32]),
+}
+
+
+def load_library(path: str | None = None):
+    """Load libmla.so (built by ``python -m mla_latent_kv_42_b200.build``); raise if absent."""
+    global _LIB
+    if _LIB is not None and path is None:
+        return _LIB
+    p = path or library_path()
+    if not os.path.exists(p):
+        raise RuntimeError(f"libmla.so is not built ({p}); run `python -m mla_latent_kv_42_b200.build`")
+    lib = ctypes.CDLL(p)
+    for name, (res, args) in _SIGS.items():
+        fn = getattr(lib, name)
+        fn.restype, fn.argtypes = res, args
+    if path is None:
+        _LIB = lib
+    return lib
+
+
+_lib = load_library
+
+
+def c_dims(d) -> _Dims:
+    """mla_dims from a ``synth.Dims`` (or anything with the same attributes)."""
+    return _Dims(d.d_model, d.n_heads, d.d_head, d.d_c, d.d_cq, d.d_rope, d.page_size,
+                 {"bf16": 0, "fp16": 1}[d.dtype], float(d.rope_base))
+
+
+def _ptr(t):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(stream):
+    import torch
+    s = torch.cuda.current_stream() if stream is None else stream
+    return ctypes.c_void_p(s.cuda_stream)
+
+
+def _check(code: int, what: str):
+    if code != 0:
+        raise MLAError(code, what)
+
+
+def _need(t, dtype, name, dims=None):
+    import torch
+    if t.device.type != "cuda":
+        raise ValueError(f"{name} must be a CUDA tensor")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+    if dtype is not None and t.dtype != dtype:
+        raise ValueError(f"{name} must be {dtype}, got {t.dtype}")
+
+
+def _elem(d):
+    import torch
+    return {"bf16": torch.bfloat16, "fp16": torch.float16}[d.dtype]
+
+
+def workspace_size(dims, call: int, B: int, max_seq_len: int = 0) -> int:
+    cd = c_dims(dims)
+    return int(_lib().mla_workspace_size(ctypes.byref(cd), call, B, max_seq_len))
+
+
+def cache_elems_per_token(dims) -> int:
+    cd = c_dims(dims)
+    return int(_lib().mla_cache_elems_per_token(ctypes.byref(cd)))
+
+
+def _ws(dims, call, B, max_seq_len, ws, device):
+    import torch
+    n = workspace_size(dims, call, B, max_seq_len)
+    if ws is None:
+        ws = torch.empty(max(n, 16), dtype=torch.uint8, device=device)
+    return ws, ws.numel() * ws.element_size()
+
+
+def append_kv(dims, h, w_dkv_kr, seq_idx, pos, block_table, pool, ws=None, stream=None):
+    """mla_append_kv: write [c ‖ RoPE(k^)] of each new token into its paged slot of ``pool``."""
+    import torch
+    e = _elem(dims)
+    for t, n, dt in ((h, "h", e), (w_dkv_kr, "w_dkv_kr", e), (seq_idx, "seq_idx", torch.int32),
+                     (pos, "pos", torch.int32), (block_table, "block_table", torch.int32), (pool, "pool", e)):
+        _need(t, dt, n)
+    T = h.shape[0]
+    ws, nbytes = _ws(dims, CALL_APPEND_KV, T, 0, ws, h.device)
+    cd = c_dims(dims)
+    _check(_lib().mla_append_kv(ctypes.byref(cd), _ptr(h), _ptr(w_dkv_kr), _ptr(seq_idx), _ptr(pos),
+                                _ptr(block_table), block_table.shape[0], block_table.shape[1], _ptr(pool),
+                                pool.shape[0], T, _ptr(ws), nbytes, _stream(stream)), "mla_append_kv")
+    return pool
+
+
+def absorb_query(dims, h, w_dq, w_uq_qr, w_uk, pos, q_out=None, ws=None, stream=None):
+    """mla_absorb_query: q_out[b][i] = [(W^UK_i)^T q^C_i ‖ RoPE(q^_i, pos[b])]."""
+    import torch
+    e = _elem(dims)
+    for t, n, dt in ((h, "h", e), (w_dq, "w_dq", e), (w_uq_qr, "w_uq_qr", e), (w_uk, "w_uk", e),
+                     (pos, "pos", torch.int32)):
+        _need(t, dt, n)
+    B = h.shape[0]
+    if q_out is None:
+        q_out = torch.empty((B, dims.n_heads, dims.d_c + dims.d_rope), dtype=e, device=h.device)
+    _need(q_out, e, "q_out")
+    ws, nbytes = _ws(dims, CALL_ABSORB_QUERY, B, 0, ws, h.device)
+    cd = c_dims(dims)
+    _check(_lib().mla_absorb_query(ctypes.byref(cd), _ptr(h), _ptr(w_dq), _ptr(w_uq_qr), _ptr(w_uk), _ptr(pos),
+                                   _ptr(q_out), B, _ptr(ws), nbytes, _stream(stream)), "mla_absorb_query")
+    return q_out
+
+
+def decode_attention(dims, q, pool, block_table, seq_lens, max_seq_len, o_lat=None, lse=None, want_lse=True,
+                     ws=None, stream=None):
+    """mla_decode_attention: latent-space softmax attention of every head over its sequence's cache."""
+    import torch
+    e = _elem(dims)
+    for t, n, dt in ((q, "q", e), (pool, "pool", e), (block_table, "block_table", torch.int32),
+                     (seq_lens, "seq_lens", torch.int32)):
+        _need(t, dt, n)
+    B = q.shape[0]
+    if o_lat is None:
+        o_lat = torch.empty((B, dims.n_heads, dims.d_c), dtype=e, device=q.device)
+    if lse is None and want_lse:
+        lse = torch.empty((B, dims.n_heads), dtype=torch.float32, device=q.device)
+    _need(o_lat, e, "o_lat")
+    if lse is not None:
+        _need(lse, torch.float32, "lse")
+    ws, nbytes = _ws(dims, CALL_DECODE_ATTENTION, B, max_seq_len, ws, q.device)
+    cd = c_dims(dims)
+    _check(_lib().mla_decode_attention(ctypes.byref(cd), _ptr(q), _ptr(pool), pool.shape[0], _ptr(block_table),
+                                       block_table.shape[1], _ptr(seq_lens), B, int(max_seq_len), _ptr(o_lat),
+                                       _ptr(lse), _ptr(ws), nbytes, _stream(stream)), "mla_decode_attention")
+    return o_lat, lse
+
+
+def out_proj(dims, o_lat, w_uv, w_o, u=None, ws=None, stream=None):
+    """mla_out_proj: u = W^O [W^UV_1 o_lat_1; ...; W^UV_n_h o_lat_n_h]."""
+    import torch
+    e = _elem(dims)
+    for t, n in ((o_lat, "o_lat"), (w_uv, "w_uv"), (w_o, "w_o")):
+        _need(t, e, n)
+    B = o_lat.shape[0]
+    if u is None:
+        u = torch.empty((B, dims.d_model), dtype=e, device=o_lat.device)
+    _need(u, e, "u")
+    ws, nbytes = _ws(dims, CALL_OUT_PROJ, B, 0, ws, o_lat.device)
+    cd = c_dims(dims)
+    _check(_lib().mla_out_proj(ctypes.byref(cd), _ptr(o_lat), _ptr(w_uv), _ptr(w_o), _ptr(u), B, _ptr(ws), nbytes,
+                               _stream(stream)), "mla_out_proj")
+    return u
+
+
+def read_device_status(stream=None) -> int:
+    """Synchronise the stream; return and clear the device status word (0 = no device-side error)."""
+    v = ctypes.c_int32(0)
+    _check(_lib().mla_read_device_status(_stream(stream), ctypes.byref(v)), "mla_read_device_status")
+    return int(v.value)
+
+
+def last_launch_count(call: int) -> int:
+    return int(_lib().mla_last_launch_count(call))
+
+
+@dataclass
+class LayerState:
+    """Device-resident state of one layer: weights and its paged latent cache."""
+    dims: object
+    w: dict            # w_dkv_kr, w_dq, w_uq_qr, w_uk, w_uv, w_o (CUDA tensors)
+    pool: object       # [num_pages, page_size, d_c + d_rope]
+    block_table: object  # int32 [B, max_pages]
+
+
+def layer_step(st: LayerState, h, pos, seq_idx, seq_lens, max_seq_len, ws=None, out=None, stream=None):
+    """One decode step of one layer through the four C-ABI calls; returns (u, q, o_lat, lse).
+
+    ``pos`` = cached length of each sequence (the new token's position), ``seq_lens`` = pos + 1.
+    ``ws`` is one byte buffer at least as large as the largest of the four workspaces (the calls
+    run in order on one stream, so they can share it).
+    """
+    d, w = st.dims, st.w
+    out = out or {}
+    append_kv(d, h, w["w_dkv_kr"], seq_idx, pos, st.block_table, st.pool, ws=ws, stream=stream)
+    q = absorb_query(d, h, w["w_dq"], w["w_uq_qr"], w["w_uk"], pos, q_out=out.get("q"), ws=ws, stream=stream)
+    o_lat, lse = decode_attention(d, q, st.pool, st.block_table, seq_lens, max_seq_len, o_lat=out.get("o_lat"),
+                                  lse=out.get("lse"), want_lse=out.get("want_lse", True), ws=ws, stream=stream)
+    u = out_proj(d, o_lat, w["w_uv"], w["w_o"], u=out.get("u"), ws=ws, stream=stream)
+    return u, q, o_lat, lse
+
+
+def step_workspace_bytes(dims, B: int, max_seq_len: int) -> int:
+    return max(workspace_size(dims, c, B, max_seq_len) for c in range(4))

@@ -1,0 +1,85 @@
+// Shared device helpers: element types, packed loads, warp reductions, the device status word,
+// and the RoPE angle. Every kernel of libmla is compiled in one translation unit (libmla.cu).
+#pragma once
+
+#include <cuda_bf16.h>
+#include <cuda_fp16.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "mla.h"
+
+namespace mla {
+
+// First device-side error since the last mla_read_device_status (0 = none). Kernels record
+// errors here instead of trapping; the first writer wins.
+__device__ int g_status;
+
+__device__ __forceinline__ void record_error(int code) { atomicCAS(&g_status, 0, code); }
+
+template <typename T> struct Pack;
+template <> struct Pack<__nv_bfloat16> {
+  using T2 = __nv_bfloat162;
+  static __device__ __forceinline__ float2 f2(T2 v) { return __bfloat1622float2(v); }
+  static __device__ __forceinline__ T2 make(float a, float b) { return __floats2bfloat162_rn(a, b); }
+  static __device__ __forceinline__ float f(__nv_bfloat16 v) { return __bfloat162float(v); }
+  static __device__ __forceinline__ __nv_bfloat16 one(float a) { return __float2bfloat16_rn(a); }
+};
+template <> struct Pack<__half> {
+  using T2 = __half2;
+  static __device__ __forceinline__ float2 f2(T2 v) { return __half22float2(v); }
+  static __device__ __forceinline__ T2 make(float a, float b) { return __floats2half2_rn(a, b); }
+  static __device__ __forceinline__ float f(__half v) { return __half2float(v); }
+  static __device__ __forceinline__ __half one(float a) { return __float2half_rn(a); }
+};
+
+// Store helpers for fp32 or element-type outputs.
+template <typename O> struct Out;
+template <> struct Out<float> {
+  static __device__ __forceinline__ void put(float* p, float v) { *p = v; }
+};
+template <> struct Out<__nv_bfloat16> {
+  static __device__ __forceinline__ void put(__nv_bfloat16* p, float v) { *p = __float2bfloat16_rn(v); }
+};
+template <> struct Out<__half> {
+  static __device__ __forceinline__ void put(__half* p, float v) { *p = __float2half_rn(v); }
+};
+
+// 8 consecutive elements (16 bytes) to fp32.
+template <typename T>
+__device__ __forceinline__ void unpack8(const uint4& v, float (&f)[8]) {
+  using T2 = typename Pack<T>::T2;
+  const T2* p = reinterpret_cast<const T2*>(&v);
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    float2 x = Pack<T>::f2(p[i]);
+    f[2 * i] = x.x;
+    f[2 * i + 1] = x.y;
+  }
+}
+
+__device__ __forceinline__ uint4 ldg16(const void* p) { return __ldg(reinterpret_cast<const uint4*>(p)); }
+
+__device__ __forceinline__ float warp_sum(float v) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+  return v;
+}
+__device__ __forceinline__ float warp_max(float v) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, o));
+  return v;
+}
+
+// cos/sin of the RoPE angle of pair k at position pos: pos * base^(-2k/d_rope). The angle is
+// formed and reduced in double precision (an fp32 angle at position 131072 would be off by
+// up to ~1e-2 rad); only the final cos/sin are rounded to fp32.
+__device__ __forceinline__ void rope_cos_sin(int pos, int k, int d_rope, double base, float& c, float& s) {
+  const double theta = pow(base, -2.0 * (double)k / (double)d_rope);
+  double sd, cd;
+  sincos((double)pos * theta, &sd, &cd);
+  c = (float)cd;
+  s = (float)sd;
+}
+
+}  // namespace mla

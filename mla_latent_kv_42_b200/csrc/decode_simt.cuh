@@ -1,0 +1,124 @@
+// CUDA-core latent attention (any supported dims; the path for small head counts):
+// one warp per head, tokens streamed with an online softmax, split-KV partials merged by
+// log-sum-exp in a fixed order (bitwise reproducible).
+#pragma once
+
+#include "common.cuh"
+
+namespace mla {
+
+constexpr float kLog2e = 1.4426950408889634f;
+constexpr float kLn2 = 0.6931471805599453f;
+
+// grid (n_splits, B, ceil(n_h / 8)), block 256 (warp w -> head blockIdx.z*8 + w).
+// NPAIR = ceil(D / 64): element pairs of one row held per lane.
+template <typename T, int NPAIR>
+__global__ void __launch_bounds__(256) k_decode_simt(
+    const T* __restrict__ q, const T* __restrict__ pool, const int* __restrict__ bt, int max_pages,
+    const int* __restrict__ seq_lens, int max_seq_len, int num_pages, int n_h, int d_c, int D, int page_size,
+    float scale_log2, int split_len, int n_splits, T* __restrict__ o_lat, float* __restrict__ lse_out,
+    float* __restrict__ o_part, float* __restrict__ lse_part) {
+  using P = Pack<T>;
+  using T2 = typename P::T2;
+  const int lane = threadIdx.x & 31;
+  const int h = blockIdx.z * 8 + (threadIdx.x >> 5);
+  const int split = blockIdx.x, b = blockIdx.y;
+  if (h >= n_h) return;
+  int L = seq_lens[b];
+  if (L < 1 || L > max_seq_len || (L + page_size - 1) / page_size > max_pages) {
+    if (split == 0 && h == 0 && lane == 0) record_error(MLA_ERR_BAD_SEQ_LEN);
+    L = 0;  // the sequence's output becomes zeros
+  }
+  const int npairs = D / 2, lpairs = d_c / 2;
+  const T2* qp = reinterpret_cast<const T2*>(q + ((long)b * n_h + h) * D);
+  float2 qf[NPAIR], o[NPAIR];
+#pragma unroll
+  for (int r = 0; r < NPAIR; ++r) {
+    const int p = lane + 32 * r;
+    float2 v = make_float2(0.f, 0.f);
+    if (p < npairs) v = P::f2(qp[p]);
+    qf[r] = make_float2(v.x * scale_log2, v.y * scale_log2);
+    o[r] = make_float2(0.f, 0.f);
+  }
+  float m = -INFINITY, l = 0.f;  // running max (log2 units) and denominator
+  const int t0 = split * split_len;
+  const int t1 = min(L, t0 + split_len);
+  const int* btb = bt + (long)b * max_pages;
+  for (int t = t0; t < t1; ++t) {
+    const int page = btb[t / page_size];
+    if (page < 0 || page >= num_pages) {
+      if (lane == 0) record_error(MLA_ERR_BAD_PAGE);
+      continue;
+    }
+    const T2* row = reinterpret_cast<const T2*>(pool + ((long)page * page_size + t % page_size) * D);
+    float2 c[NPAIR];
+    float s = 0.f;
+#pragma unroll
+    for (int r = 0; r < NPAIR; ++r) {
+      const int p = lane + 32 * r;
+      c[r] = make_float2(0.f, 0.f);
+      if (p < npairs) c[r] = P::f2(row[p]);
+      s = fmaf(qf[r].x, c[r].x, fmaf(qf[r].y, c[r].y, s));
+    }
+    s = warp_sum(s);
+    const float m_new = fmaxf(m, s);
+    const float alpha = exp2f(m - m_new);
+    const float pj = exp2f(s - m_new);
+    l = fmaf(l, alpha, pj);
+#pragma unroll
+    for (int r = 0; r < NPAIR; ++r) {
+      if (lane + 32 * r < lpairs) {
+        o[r].x = fmaf(o[r].x, alpha, pj * c[r].x);
+        o[r].y = fmaf(o[r].y, alpha, pj * c[r].y);
+      }
+    }
+    m = m_new;
+  }
+  const float inv = l > 0.f ? 1.f / l : 0.f;
+  const float lse = l > 0.f ? (m + log2f(l)) * kLn2 : -INFINITY;
+  const long bh = (long)b * n_h + h;
+  if (n_splits == 1) {
+    T2* out = reinterpret_cast<T2*>(o_lat + bh * d_c);
+#pragma unroll
+    for (int r = 0; r < NPAIR; ++r) {
+      const int p = lane + 32 * r;
+      if (p < lpairs) out[p] = P::make(o[r].x * inv, o[r].y * inv);
+    }
+    if (lse_out != nullptr && lane == 0) lse_out[bh] = lse;
+  } else {
+    float2* out = reinterpret_cast<float2*>(o_part + (bh * n_splits + split) * d_c);
+#pragma unroll
+    for (int r = 0; r < NPAIR; ++r) {
+      const int p = lane + 32 * r;
+      if (p < lpairs) out[p] = make_float2(o[r].x * inv, o[r].y * inv);
+    }
+    if (lane == 0) lse_part[bh * n_splits + split] = lse;
+  }
+}
+
+// Merge of split-KV partials: o = sum_s w_s o_s / sum_s w_s with w_s = e^{lse_s - max lse},
+// summed in split order. One block per (b, head); o_part [BH][S][d_c], lse_part [BH][S].
+template <typename T>
+__global__ void k_lse_merge(const float* __restrict__ o_part, const float* __restrict__ lse_part, int n_splits,
+                            int d_c, T* __restrict__ o_lat, float* __restrict__ lse_out) {
+  const long bh = blockIdx.x;
+  const float* lp = lse_part + bh * n_splits;
+  float mx = -INFINITY;
+  for (int s = 0; s < n_splits; ++s) mx = fmaxf(mx, lp[s]);
+  float z = 0.f;
+  if (mx != -INFINITY)
+    for (int s = 0; s < n_splits; ++s) z += exp2f((lp[s] - mx) * kLog2e);
+  const float inv = z > 0.f ? 1.f / z : 0.f;
+  for (int e = threadIdx.x; e < d_c; e += blockDim.x) {
+    float acc = 0.f;
+    if (z > 0.f)
+      for (int s = 0; s < n_splits; ++s) {
+        const float w = exp2f((lp[s] - mx) * kLog2e);
+        acc = fmaf(w, o_part[(bh * n_splits + s) * d_c + e], acc);
+      }
+    Out<T>::put(o_lat + bh * d_c + e, acc * inv);
+  }
+  if (lse_out != nullptr && threadIdx.x == 0) lse_out[bh] = z > 0.f ? mx + logf(z) : -INFINITY;
+}
+
+}  // namespace mla

@@ -1,0 +1,358 @@
+// libmla — C ABI of the MLA absorbed-decode path (declared in include/mla.h).
+// One translation unit: the kernels are included from the .cuh files beside this one.
+// Host code here validates arguments (before anything is queued), carves the caller's
+// workspace, picks kernels and launches them on the caller's stream. It allocates nothing.
+#include <cmath>
+#include <cstring>
+
+#include "common.cuh"
+#include "decode_simt.cuh"
+#include "proj_simt.cuh"
+
+using namespace mla;
+
+namespace {
+
+thread_local int32_t t_launches[4] = {0, 0, 0, 0};
+
+constexpr int kMaxDevices = 64;
+
+int device_sm_count() {
+  static int cache[kMaxDevices] = {0};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return 148;
+  if (cache[dev] == 0) {
+    int n = 0;
+    if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0) n = 148;
+    cache[dev] = n;
+  }
+  return cache[dev];
+}
+
+inline bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+inline size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
+inline size_t esize(const mla_dims* d) { (void)d; return 2; }
+
+// Sequential sub-allocation of the caller's workspace (256-byte aligned pieces).
+struct Carve {
+  char* base;
+  size_t off = 0;
+  template <typename X>
+  X* take(size_t count) {
+    X* p = reinterpret_cast<X*>(base + off);
+    off += align256(count * sizeof(X));
+    return p;
+  }
+};
+
+int check_dims_impl(const mla_dims* d) {
+  if (d == nullptr) return MLA_ERR_INVALID_ARG;
+  if (d->dtype != MLA_BF16 && d->dtype != MLA_FP16) return MLA_ERR_INVALID_ARG;
+  if (!(d->rope_base > 0.0) || !std::isfinite(d->rope_base)) return MLA_ERR_INVALID_ARG;
+  const int32_t w[] = {d->d_model, d->n_heads, d->d_head, d->d_c, d->d_cq, d->d_rope, d->page_size};
+  for (int32_t v : w)
+    if (v <= 0) return MLA_ERR_INVALID_ARG;
+  if (d->d_model % 8 || d->d_head % 8 || d->d_c % 8 || d->d_cq % 8 || d->d_rope % 8) return MLA_ERR_UNSUPPORTED_DIMS;
+  if (d->n_heads > 128 || d->d_c > 512 || d->d_c + d->d_rope > 576) return MLA_ERR_UNSUPPORTED_DIMS;
+  return MLA_OK;
+}
+
+// ---------------------------------------------------------------- decode planning
+struct DecodePlan {
+  int n_splits;
+  int split_len;
+  int head_groups;
+};
+
+DecodePlan plan_decode(const mla_dims* d, int B, int max_seq_len) {
+  DecodePlan p;
+  p.head_groups = (d->n_heads + 7) / 8;
+  const long blocks_wanted = 4L * device_sm_count();
+  const long base = (long)B * p.head_groups;
+  long s = (blocks_wanted + base - 1) / base;
+  const long by_len = (max_seq_len + 255) / 256;  // at least 256 tokens per split
+  if (s > by_len) s = by_len;
+  if (s < 1) s = 1;
+  p.n_splits = (int)s;
+  p.split_len = (int)((max_seq_len + s - 1) / s);
+  return p;
+}
+
+size_t ws_append(const mla_dims* d, int T) { return T > 0 ? align256((size_t)T * (d->d_c + d->d_rope) * 4) : 0; }
+
+size_t ws_absorb(const mla_dims* d, int B) {
+  if (B <= 0) return 0;
+  const size_t nq = (size_t)d->n_heads * (d->d_head + d->d_rope);
+  return align256((size_t)B * d->d_cq * esize(d)) + align256((size_t)B * nq * 4) +
+         align256((size_t)B * d->n_heads * d->d_head * esize(d));
+}
+
+size_t ws_decode(const mla_dims* d, int B, int max_seq_len) {
+  if (B <= 0 || max_seq_len <= 0) return 0;
+  const DecodePlan p = plan_decode(d, B, max_seq_len);
+  if (p.n_splits == 1) return 0;
+  const size_t bh = (size_t)B * d->n_heads;
+  return align256(bh * p.n_splits * d->d_c * 4) + align256(bh * p.n_splits * 4);
+}
+
+size_t ws_out(const mla_dims* d, int B) {
+  return B > 0 ? align256((size_t)B * d->n_heads * d->d_head * esize(d)) : 0;
+}
+
+template <typename T, typename OutT>
+void launch_rowdot(const T* W, const T* X, OutT* Y, int M, int K, int Tn, long ldx, long ldy, int batch, long sW,
+                   long sX, long sY, cudaStream_t st, int32_t& launches) {
+  if (Tn <= 0 || M <= 0 || batch <= 0) return;
+  dim3 grid((M + 7) / 8, 1, batch);
+  if (Tn <= 8)
+    k_rowdot<T, OutT, 8><<<grid, 256, 0, st>>>(W, X, Y, M, K, Tn, ldx, ldy, sW, sX, sY);
+  else
+    k_rowdot<T, OutT, 16><<<grid, 256, 0, st>>>(W, X, Y, M, K, Tn, ldx, ldy, sW, sX, sY);
+  ++launches;
+}
+
+int finish_launches(int call, int32_t launches) {
+  const cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return MLA_ERR_CUDA;
+  t_launches[call] = launches;
+  return MLA_OK;
+}
+
+template <typename T>
+int append_impl(const mla_dims* d, const void* h, const void* w, const int32_t* seq_idx, const int32_t* pos,
+                const int32_t* bt, int32_t num_seqs, int32_t max_pages, void* pool, int32_t num_pages, int32_t T_,
+                void* ws, cudaStream_t st) {
+  const int D = d->d_c + d->d_rope;
+  int32_t n = 0;
+  Carve c{static_cast<char*>(ws)};
+  float* Y = c.take<float>((size_t)T_ * D);
+  launch_rowdot<T, float>(static_cast<const T*>(w), static_cast<const T*>(h), Y, D, d->d_model, T_, d->d_model, D,
+                          1, 0, 0, 0, st, n);
+  k_append_epilogue<T><<<T_, 128, 0, st>>>(Y, seq_idx, pos, bt, num_seqs, max_pages, static_cast<T*>(pool), num_pages,
+                                          d->page_size, d->d_c, d->d_rope, d->rope_base);
+  ++n;
+  return finish_launches(MLA_CALL_APPEND_KV, n);
+}
+
+template <typename T>
+int absorb_impl(const mla_dims* d, const void* h, const void* w_dq, const void* w_uq_qr, const void* w_uk,
+                const int32_t* pos, void* q_out, int32_t B, void* ws, cudaStream_t st) {
+  const int nq = d->n_heads * (d->d_head + d->d_rope);
+  const int D = d->d_c + d->d_rope;
+  int32_t n = 0;
+  Carve c{static_cast<char*>(ws)};
+  T* cq = c.take<T>((size_t)B * d->d_cq);
+  float* Y2 = c.take<float>((size_t)B * nq);
+  T* qc = c.take<T>((size_t)B * d->n_heads * d->d_head);
+  launch_rowdot<T, T>(static_cast<const T*>(w_dq), static_cast<const T*>(h), cq, d->d_cq, d->d_model, B, d->d_model,
+                      d->d_cq, 1, 0, 0, 0, st, n);
+  launch_rowdot<T, float>(static_cast<const T*>(w_uq_qr), cq, Y2, nq, d->d_cq, B, d->d_cq, nq, 1, 0, 0, 0, st, n);
+  k_query_epilogue<T><<<B, 256, 0, st>>>(Y2, pos, qc, static_cast<T*>(q_out), d->n_heads, d->d_head, d->d_rope,
+                                         d->d_c, d->rope_base);
+  ++n;
+  const int threads = 128;
+  dim3 grid((d->d_c / 2 + threads - 1) / threads, d->n_heads);
+  k_absorb_uk<T, 16><<<grid, threads, 16 * d->d_head * sizeof(float), st>>>(
+      static_cast<const T*>(w_uk), qc, static_cast<T*>(q_out), B, d->n_heads, d->d_head, d->d_c, D);
+  ++n;
+  return finish_launches(MLA_CALL_ABSORB_QUERY, n);
+}
+
+template <typename T, int NPAIR>
+void launch_decode_simt(const mla_dims* d, const DecodePlan& p, const void* q, const void* pool, int32_t num_pages,
+                        const int32_t* bt, int32_t max_pages, const int32_t* seq_lens, int32_t B, int32_t max_seq_len,
+                        void* o_lat, float* lse_out, float* o_part, float* lse_part, cudaStream_t st) {
+  const float scale_log2 = (float)(1.0 / std::sqrt((double)(d->d_head + d->d_rope)) * 1.4426950408889634);
+  dim3 grid(p.n_splits, B, p.head_groups);
+  k_decode_simt<T, NPAIR><<<grid, 256, 0, st>>>(
+      static_cast<const T*>(q), static_cast<const T*>(pool), bt, max_pages, seq_lens, max_seq_len, num_pages,
+      d->n_heads, d->d_c, d->d_c + d->d_rope, d->page_size, scale_log2, p.split_len, p.n_splits,
+      static_cast<T*>(o_lat), lse_out, o_part, lse_part);
+}
+
+template <typename T>
+int decode_impl(const mla_dims* d, const void* q, const void* pool, int32_t num_pages, const int32_t* bt,
+                int32_t max_pages, const int32_t* seq_lens, int32_t B, int32_t max_seq_len, void* o_lat,
+                float* lse_out, void* ws, cudaStream_t st) {
+  const DecodePlan p = plan_decode(d, B, max_seq_len);
+  const size_t bh = (size_t)B * d->n_heads;
+  float* o_part = nullptr;
+  float* lse_part = nullptr;
+  if (p.n_splits > 1) {
+    Carve c{static_cast<char*>(ws)};
+    o_part = c.take<float>(bh * p.n_splits * d->d_c);
+    lse_part = c.take<float>(bh * p.n_splits);
+  }
+  const int D = d->d_c + d->d_rope;
+  int32_t n = 0;
+  if (D <= 192)
+    launch_decode_simt<T, 3>(d, p, q, pool, num_pages, bt, max_pages, seq_lens, B, max_seq_len, o_lat, lse_out,
+                             o_part, lse_part, st);
+  else if (D <= 384)
+    launch_decode_simt<T, 6>(d, p, q, pool, num_pages, bt, max_pages, seq_lens, B, max_seq_len, o_lat, lse_out,
+                             o_part, lse_part, st);
+  else
+    launch_decode_simt<T, 9>(d, p, q, pool, num_pages, bt, max_pages, seq_lens, B, max_seq_len, o_lat, lse_out,
+                             o_part, lse_part, st);
+  ++n;
+  if (p.n_splits > 1) {
+    k_lse_merge<T><<<(unsigned)bh, 128, 0, st>>>(o_part, lse_part, p.n_splits, d->d_c, static_cast<T*>(o_lat),
+                                                 lse_out);
+    ++n;
+  }
+  return finish_launches(MLA_CALL_DECODE_ATTENTION, n);
+}
+
+template <typename T>
+int out_impl(const mla_dims* d, const void* o_lat, const void* w_uv, const void* w_o, void* u, int32_t B, void* ws,
+             cudaStream_t st) {
+  const int nhd = d->n_heads * d->d_head;
+  int32_t n = 0;
+  Carve c{static_cast<char*>(ws)};
+  T* o = c.take<T>((size_t)B * nhd);
+  // o_i = W^UV_i o_lat_i, batched over heads (row block i of W^UV, head i of o_lat)
+  launch_rowdot<T, T>(static_cast<const T*>(w_uv), static_cast<const T*>(o_lat), o, d->d_head, d->d_c, B,
+                      (long)d->n_heads * d->d_c, nhd, d->n_heads, (long)d->d_head * d->d_c, d->d_c, d->d_head, st, n);
+  launch_rowdot<T, T>(static_cast<const T*>(w_o), o, static_cast<T*>(u), d->d_model, nhd, B, nhd, d->d_model, 1, 0,
+                      0, 0, st, n);
+  return finish_launches(MLA_CALL_OUT_PROJ, n);
+}
+
+}  // namespace
+
+extern "C" {
+
+int mla_check_dims(const mla_dims* dims) { return check_dims_impl(dims); }
+
+int32_t mla_cache_elems_per_token(const mla_dims* dims) {
+  const int r = check_dims_impl(dims);
+  if (r != MLA_OK) return r;
+  return dims->d_c + dims->d_rope;
+}
+
+size_t mla_workspace_size(const mla_dims* dims, int32_t call, int32_t B, int32_t max_seq_len) {
+  if (check_dims_impl(dims) != MLA_OK || B < 0) return 0;
+  switch (call) {
+    case MLA_CALL_APPEND_KV: return ws_append(dims, B);
+    case MLA_CALL_ABSORB_QUERY: return ws_absorb(dims, B);
+    case MLA_CALL_DECODE_ATTENTION: return ws_decode(dims, B, max_seq_len);
+    case MLA_CALL_OUT_PROJ: return ws_out(dims, B);
+    default: return 0;
+  }
+}
+
+int mla_append_kv(const mla_dims* dims, const void* h, const void* w_dkv_kr, const int32_t* seq_idx,
+                  const int32_t* pos, const int32_t* block_table, int32_t num_seqs, int32_t max_pages, void* pool,
+                  int32_t num_pages, int32_t T, void* ws, size_t ws_bytes, mla_stream_t stream) {
+  int r = check_dims_impl(dims);
+  if (r != MLA_OK) return r;
+  if (T < 0 || num_seqs <= 0 || max_pages <= 0 || num_pages <= 0) return MLA_ERR_INVALID_ARG;
+  if (T == 0) {
+    t_launches[MLA_CALL_APPEND_KV] = 0;
+    return MLA_OK;
+  }
+  if (!h || !w_dkv_kr || !seq_idx || !pos || !block_table || !pool) return MLA_ERR_INVALID_ARG;
+  if (!aligned16(h) || !aligned16(w_dkv_kr) || !aligned16(pool) || !aligned16(ws)) return MLA_ERR_ALIGNMENT;
+  if (ws_bytes < ws_append(dims, T)) return MLA_ERR_WORKSPACE_TOO_SMALL;
+  if (!ws) return MLA_ERR_INVALID_ARG;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  if (dims->dtype == MLA_BF16)
+    return append_impl<__nv_bfloat16>(dims, h, w_dkv_kr, seq_idx, pos, block_table, num_seqs, max_pages, pool,
+                                      num_pages, T, ws, st);
+  return append_impl<__half>(dims, h, w_dkv_kr, seq_idx, pos, block_table, num_seqs, max_pages, pool, num_pages, T,
+                             ws, st);
+}
+
+int mla_absorb_query(const mla_dims* dims, const void* h, const void* w_dq, const void* w_uq_qr, const void* w_uk,
+                     const int32_t* pos, void* q_out, int32_t B, void* ws, size_t ws_bytes, mla_stream_t stream) {
+  int r = check_dims_impl(dims);
+  if (r != MLA_OK) return r;
+  if (B < 0 || B > 65535) return MLA_ERR_INVALID_ARG;
+  if (B == 0) {
+    t_launches[MLA_CALL_ABSORB_QUERY] = 0;
+    return MLA_OK;
+  }
+  if (!h || !w_dq || !w_uq_qr || !w_uk || !pos || !q_out || !ws) return MLA_ERR_INVALID_ARG;
+  if (!aligned16(h) || !aligned16(w_dq) || !aligned16(w_uq_qr) || !aligned16(w_uk) || !aligned16(q_out) ||
+      !aligned16(ws))
+    return MLA_ERR_ALIGNMENT;
+  if (ws_bytes < ws_absorb(dims, B)) return MLA_ERR_WORKSPACE_TOO_SMALL;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  if (dims->dtype == MLA_BF16)
+    return absorb_impl<__nv_bfloat16>(dims, h, w_dq, w_uq_qr, w_uk, pos, q_out, B, ws, st);
+  return absorb_impl<__half>(dims, h, w_dq, w_uq_qr, w_uk, pos, q_out, B, ws, st);
+}
+
+int mla_decode_attention(const mla_dims* dims, const void* q, const void* pool, int32_t num_pages,
+                         const int32_t* block_table, int32_t max_pages, const int32_t* seq_lens, int32_t B,
+                         int32_t max_seq_len, void* o_lat, float* lse_out, void* ws, size_t ws_bytes,
+                         mla_stream_t stream) {
+  int r = check_dims_impl(dims);
+  if (r != MLA_OK) return r;
+  if (B < 0 || B > 65535 || max_seq_len < 1 || max_pages <= 0 || num_pages <= 0) return MLA_ERR_INVALID_ARG;
+  if ((long)max_pages * dims->page_size < (long)max_seq_len) return MLA_ERR_INVALID_ARG;
+  if (B == 0) {
+    t_launches[MLA_CALL_DECODE_ATTENTION] = 0;
+    return MLA_OK;
+  }
+  if (!q || !pool || !block_table || !seq_lens || !o_lat) return MLA_ERR_INVALID_ARG;
+  if (!aligned16(q) || !aligned16(pool) || !aligned16(o_lat) || !aligned16(ws) || !aligned16(lse_out))
+    return MLA_ERR_ALIGNMENT;
+  const size_t need = ws_decode(dims, B, max_seq_len);
+  if (ws_bytes < need) return MLA_ERR_WORKSPACE_TOO_SMALL;
+  if (need > 0 && !ws) return MLA_ERR_INVALID_ARG;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  if (dims->dtype == MLA_BF16)
+    return decode_impl<__nv_bfloat16>(dims, q, pool, num_pages, block_table, max_pages, seq_lens, B, max_seq_len,
+                                      o_lat, lse_out, ws, st);
+  return decode_impl<__half>(dims, q, pool, num_pages, block_table, max_pages, seq_lens, B, max_seq_len, o_lat,
+                             lse_out, ws, st);
+}
+
+int mla_out_proj(const mla_dims* dims, const void* o_lat, const void* w_uv, const void* w_o, void* u, int32_t B,
+                 void* ws, size_t ws_bytes, mla_stream_t stream) {
+  int r = check_dims_impl(dims);
+  if (r != MLA_OK) return r;
+  if (B < 0 || B > 65535) return MLA_ERR_INVALID_ARG;
+  if (B == 0) {
+    t_launches[MLA_CALL_OUT_PROJ] = 0;
+    return MLA_OK;
+  }
+  if (!o_lat || !w_uv || !w_o || !u || !ws) return MLA_ERR_INVALID_ARG;
+  if (!aligned16(o_lat) || !aligned16(w_uv) || !aligned16(w_o) || !aligned16(u) || !aligned16(ws))
+    return MLA_ERR_ALIGNMENT;
+  if (ws_bytes < ws_out(dims, B)) return MLA_ERR_WORKSPACE_TOO_SMALL;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  if (dims->dtype == MLA_BF16) return out_impl<__nv_bfloat16>(dims, o_lat, w_uv, w_o, u, B, ws, st);
+  return out_impl<__half>(dims, o_lat, w_uv, w_o, u, B, ws, st);
+}
+
+int mla_read_device_status(mla_stream_t stream, int32_t* status_out) {
+  if (!status_out) return MLA_ERR_INVALID_ARG;
+  if (cudaStreamSynchronize(reinterpret_cast<cudaStream_t>(stream)) != cudaSuccess) return MLA_ERR_CUDA;
+  int v = 0;
+  const int zero = 0;
+  if (cudaMemcpyFromSymbol(&v, mla::g_status, sizeof(int)) != cudaSuccess) return MLA_ERR_CUDA;
+  if (cudaMemcpyToSymbol(mla::g_status, &zero, sizeof(int)) != cudaSuccess) return MLA_ERR_CUDA;
+  *status_out = v;
+  return MLA_OK;
+}
+
+const char* mla_error_string(int code) {
+  switch (code) {
+    case MLA_OK: return "ok";
+    case MLA_ERR_INVALID_ARG: return "invalid argument";
+    case MLA_ERR_UNSUPPORTED_DIMS: return "unsupported dims";
+    case MLA_ERR_WORKSPACE_TOO_SMALL: return "workspace too small";
+    case MLA_ERR_ALIGNMENT: return "pointer not 16-byte aligned";
+    case MLA_ERR_CUDA: return "CUDA error";
+    case MLA_ERR_TIMEOUT: return "device wait timed out";
+    case MLA_ERR_BAD_PAGE: return "block-table entry out of range";
+    case MLA_ERR_BAD_SEQ_LEN: return "sequence length out of range";
+    default: return "unknown status";
+  }
+}
+
+int32_t mla_last_launch_count(int32_t call) { return (call >= 0 && call < 4) ? t_launches[call] : -1; }
+
+}  // extern "C"

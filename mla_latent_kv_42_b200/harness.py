@@ -1,0 +1,88 @@
+"""Workload state for benchmarks, tests and the smoke entry: device-resident weights, paged
+latent caches and per-step index tensors built from ``synth``. No method arithmetic here; the
+step itself is ``mla_latent_kv_42_b200.layer_step`` (the four C-ABI calls)."""
+from __future__ import annotations
+
+from dataclasses import dataclass
+
+import numpy as np
+import torch
+
+from . import LayerState, synth
+
+
+@dataclass
+class Layer:
+    state: LayerState
+    W_host: dict          # weights as drawn (host, storage dtype) — what the oracle reads
+    rows: torch.Tensor    # logical prefix rows [sum N_b, D] on the device
+    offsets: np.ndarray   # row offsets of each sequence in ``rows``
+
+    def prefix(self, b: int) -> torch.Tensor:
+        return self.rows[int(self.offsets[b]):int(self.offsets[b + 1])]
+
+
+@dataclass
+class StepIndex:
+    cached: np.ndarray    # N_b
+    pos: torch.Tensor     # int32 [B], the new token's position = N_b
+    seq_idx: torch.Tensor  # int32 [B] = arange(B)
+    seq_lens: torch.Tensor  # int32 [B] = N_b + 1
+    max_seq_len: int
+
+
+def step_index(cached: np.ndarray, device="cuda") -> StepIndex:
+    cached = np.asarray(cached, dtype=np.int64)
+    B = len(cached)
+    return StepIndex(
+        cached=cached,
+        pos=torch.from_numpy(cached.astype(np.int32)).to(device),
+        seq_idx=torch.arange(B, dtype=torch.int32, device=device),
+        seq_lens=torch.from_numpy((cached + 1).astype(np.int32)).to(device),
+        max_seq_len=int(cached.max()) + 1,
+    )
+
+
+def make_layer(w: synth.Workload, cached: np.ndarray, layer: int = 0, device="cuda", fill: float = 0.0,
+               block_table: np.ndarray | None = None, num_pages: int | None = None) -> Layer:
+    d = w.dims
+    W = synth.weights(w, layer)
+    if block_table is None:
+        block_table, num_pages = synth.page_table(cached, d.page_size, w.paging, w.seed)
+    rows = synth.prefix_rows(w, cached, layer=layer, device=device)
+    pool = synth.paged_pool(rows, cached, block_table, num_pages, d.page_size, fill=fill)
+    st = LayerState(dims=d, w={k: v.to(device) for k, v in W.items()}, pool=pool,
+                    block_table=torch.from_numpy(block_table).to(device))
+    return Layer(state=st, W_host=W, rows=rows, offsets=np.concatenate([[0], np.cumsum(cached)]))
+
+
+def weight_bytes(d: synth.Dims) -> int:
+    n_h = d.n_heads
+    elems = ((d.d_c + d.d_rope) * d.d_model + d.d_cq * d.d_model + n_h * (d.d_head + d.d_rope) * d.d_cq
+             + 2 * n_h * d.d_head * d.d_c + d.d_model * n_h * d.d_head)
+    return 2 * elems
+
+
+def decode_work(d: synth.Dims, seq_lens: np.ndarray) -> tuple[int, int]:
+    """Algorithmic bytes and flops of latent attention over the attended tokens.
+
+    Per attended token: read one cache row of d_c + d_h^R elements; 2 n_h (d_c + d_h^R) flops for
+    the scores and 2 n_h d_c for the latent weighted sum. Per sequence: read q, write o_lat.
+    """
+    L = int(np.sum(seq_lens))
+    B = len(seq_lens)
+    D = d.d_c + d.d_rope
+    byts = 2 * (L * D + B * d.n_heads * D + B * d.n_heads * d.d_c)
+    flops = 2 * L * d.n_heads * (D + d.d_c)
+    return byts, flops
+
+
+def step_work(d: synth.Dims, seq_lens: np.ndarray) -> tuple[int, int]:
+    """Algorithmic bytes and flops of one whole layer step (weights read once + decode)."""
+    B = len(seq_lens)
+    db, df = decode_work(d, seq_lens)
+    n_h = d.n_heads
+    proj_flops = 2 * B * ((d.d_c + d.d_rope) * d.d_model + d.d_cq * d.d_model + n_h * (d.d_head + d.d_rope) * d.d_cq
+                          + 2 * n_h * d.d_head * d.d_c + d.d_model * n_h * d.d_head)
+    act_bytes = 2 * B * (2 * d.d_model + (d.d_c + d.d_rope))  # h in, u out, the appended row
+    return db + weight_bytes(d) + act_bytes, df + proj_flops

@@ -1,0 +1,140 @@
+"""Host-side checks of the C ABI (no GPU): the library loads, exports every declared symbol,
+returns the pages' cache sizes, and rejects bad arguments before queueing anything."""
+import ctypes
+import os
+import re
+
+import pytest
+
+import mla_latent_kv_42_b200 as M
+from mla_latent_kv_42_b200 import build, synth
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+@pytest.fixture(scope="module")
+def lib():
+    build.build()
+    return M.load_library()
+
+
+def declared_functions():
+    text = open(os.path.join(ROOT, "include", "mla.h")).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(mla_[a-z_0-9]+)\s*\(", text)))
+
+
+def test_header_declares_the_four_calls():
+    names = declared_functions()
+    for n in ("mla_append_kv", "mla_absorb_query", "mla_decode_attention", "mla_out_proj"):
+        assert n in names
+
+
+def test_library_exports_every_declared_symbol(lib):
+    names = declared_functions()
+    assert len(names) >= 10
+    for n in names:
+        assert hasattr(lib, n), n
+    # and the symbols are plain C (unmangled) in the dynamic table
+    out = os.popen(f"nm -D --defined-only {M.library_path()}").read()
+    for n in names:
+        assert re.search(rf"\bT {n}$", out, flags=re.M), n
+
+
+def dims(d):
+    return M.c_dims(d)
+
+
+def test_cache_elems_per_token_matches_pages(lib):
+    """160 (running model, from-scratch page §4.5) and 576 (production, visual explainer)."""
+    assert M.cache_elems_per_token(synth.RUNNING) == 160
+    assert M.cache_elems_per_token(synth.PRODUCTION) == 576
+
+
+@pytest.mark.parametrize("field,value,code", [
+    ("n_heads", 129, -2), ("d_c", 520, -2), ("d_rope", 6, -2), ("d_model", 0, -1), ("dtype", 7, -1),
+    ("page_size", 0, -1), ("rope_base", 0.0, -1), ("d_head", 12, -2),
+])
+def test_check_dims_rejects(lib, field, value, code):
+    cd = dims(synth.PRODUCTION)
+    setattr(cd, field, value)
+    assert lib.mla_check_dims(ctypes.byref(cd)) == code
+    assert lib.mla_cache_elems_per_token(ctypes.byref(cd)) == code
+
+
+def test_check_dims_accepts_both_families(lib):
+    for d in (synth.RUNNING, synth.PRODUCTION, synth.RUNNING.with_(dtype="fp16")):
+        cd = dims(d)
+        assert lib.mla_check_dims(ctypes.byref(cd)) == 0
+
+
+def test_null_dims_is_invalid(lib):
+    assert lib.mla_check_dims(None) == -1
+    assert lib.mla_workspace_size(None, 0, 1, 1) == 0
+
+
+FAKE = ctypes.c_void_p(1 << 20)        # aligned, never dereferenced on the host
+MISALIGNED = ctypes.c_void_p((1 << 20) + 8)
+
+
+def test_decode_argument_errors_queue_nothing(lib):
+    cd = dims(synth.PRODUCTION)
+    f = lib.mla_decode_attention
+    args = [ctypes.byref(cd), FAKE, FAKE, 10, FAKE, 4, FAKE, 2, 256, FAKE, None, FAKE, 1 << 30, None]
+    bad = list(args)
+    bad[1] = None
+    assert f(*bad) == -1                                  # null q
+    bad = list(args)
+    bad[9] = MISALIGNED
+    assert f(*bad) == -4                                  # misaligned o_lat
+    bad = list(args)
+    bad[8] = 0
+    assert f(*bad) == -1                                  # max_seq_len < 1
+    bad = list(args)
+    bad[8] = 257
+    assert f(*bad) == -1                                  # max_pages * page_size < max_seq_len
+    bad = list(args)
+    bad[12] = 0
+    need = lib.mla_workspace_size(ctypes.byref(cd), M.CALL_DECODE_ATTENTION, 2, 256)
+    assert f(*bad) == (-3 if need > 0 else f(*bad))        # too-small workspace
+    bad = list(args)
+    bad[7] = 0
+    assert f(*bad) == 0                                   # B == 0 is a no-op
+
+
+def test_append_absorb_out_argument_errors(lib):
+    cd = dims(synth.RUNNING)
+    assert lib.mla_append_kv(ctypes.byref(cd), FAKE, FAKE, FAKE, FAKE, FAKE, 1, 4, FAKE, 8, -1, FAKE, 1 << 20,
+                             None) == -1
+    assert lib.mla_append_kv(ctypes.byref(cd), FAKE, MISALIGNED, FAKE, FAKE, FAKE, 1, 4, FAKE, 8, 3, FAKE, 1 << 20,
+                             None) == -4
+    assert lib.mla_append_kv(ctypes.byref(cd), FAKE, FAKE, FAKE, FAKE, FAKE, 1, 4, FAKE, 8, 3, FAKE, 4,
+                             None) == -3
+    assert lib.mla_append_kv(ctypes.byref(cd), FAKE, FAKE, FAKE, FAKE, FAKE, 1, 4, FAKE, 8, 0, None, 0,
+                             None) == 0
+    assert lib.mla_absorb_query(ctypes.byref(cd), FAKE, FAKE, None, FAKE, FAKE, FAKE, 2, FAKE, 1 << 20, None) == -1
+    assert lib.mla_absorb_query(ctypes.byref(cd), FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, 2, FAKE, 8, None) == -3
+    assert lib.mla_out_proj(ctypes.byref(cd), FAKE, FAKE, FAKE, MISALIGNED, 2, FAKE, 1 << 20, None) == -4
+    assert lib.mla_out_proj(ctypes.byref(cd), FAKE, FAKE, FAKE, FAKE, -1, FAKE, 1 << 20, None) == -1
+
+
+def test_workspace_sizes_are_consistent(lib):
+    for d in (synth.RUNNING, synth.PRODUCTION):
+        for call in range(4):
+            a = M.workspace_size(d, call, 64, 4097)
+            b = M.workspace_size(d, call, 128, 32769)
+            assert a >= 0 and b >= a
+            assert a % 256 == 0
+    assert M.workspace_size(synth.PRODUCTION, 9, 1, 1) == 0
+
+
+def test_error_strings(lib):
+    for code in range(0, -9, -1):
+        s = lib.mla_error_string(code).decode()
+        assert s and s != "unknown status"
+    assert lib.mla_error_string(-99).decode() == "unknown status"
+
+
+def test_product_path_fails_loudly_without_the_library(tmp_path):
+    with pytest.raises(RuntimeError, match="not built"):
+        M.load_library(str(tmp_path / "missing.so"))

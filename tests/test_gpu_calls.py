@@ -1,0 +1,209 @@
+"""GPU parity of each C-ABI call against the fp64 oracle, with edge cases.
+
+Inputs come from ``synth``; the oracle reads the same host values. Tolerance: max and mean
+absolute error normalised by the reference's largest magnitude, <= 2e-2 and <= 2e-3. Paged
+placement and status codes are checked exactly.
+"""
+import numpy as np
+import pytest
+import torch
+
+import mla_latent_kv_42_b200 as M
+import oracle as O
+from mla_latent_kv_42_b200 import build, harness, synth
+from parity import CacheCase, assert_parity, to64
+
+pytestmark = pytest.mark.gpu
+
+W_RUN16 = synth.workload("running_b1_n256_fp16")
+W_RUN = synth.workload("running_b16_n4096_l12_bf16")
+W_PROD = synth.workload("production_b64_n4096_bf16")
+FAMILIES = {"running_fp16": W_RUN16, "running_bf16": W_RUN, "production_bf16": W_PROD}
+
+
+@pytest.fixture(scope="module", autouse=True)
+def lib():
+    build.build()
+    M.load_library()
+    assert M.read_device_status() == 0
+
+
+@pytest.fixture(autouse=True)
+def clean_status():
+    M.read_device_status()
+    yield
+
+
+def weights64(w):
+    W = synth.weights(w)
+    return W, {k: O.as64(v) for k, v in W.items()}
+
+
+# ---------------------------------------------------------------------------------------- append
+@pytest.mark.parametrize("fam", list(FAMILIES))
+def test_append_kv_rows_and_exact_placement(fam):
+    w = FAMILIES[fam]
+    d = w.dims
+    W, W64 = weights64(w)
+    # several tokens per sequence across page boundaries (pos % 64 in {0, 63}), pages shuffled
+    cached = np.array([0, 63, 64, 130])
+    bt, num_pages = synth.page_table(cached + 70, d.page_size, "shuffled", seed=3)
+    seq_idx = np.repeat(np.arange(4), 3).astype(np.int32)
+    pos = np.concatenate([np.arange(c, c + 3) for c in (0, 62, 64, 127)]).astype(np.int32)
+    T = len(pos)
+    h = synth.hidden(w, step=5, batch=T)
+    pool = torch.full((num_pages, d.page_size, d.D), float("nan"), dtype=synth.storage_dtype(d), device="cuda")
+    before = pool.clone()
+    M.append_kv(d, h.cuda(), W["w_dkv_kr"].cuda(), torch.from_numpy(seq_idx).cuda(), torch.from_numpy(pos).cuda(),
+                torch.from_numpy(bt).cuda(), pool)
+    assert M.read_device_status() == 0
+    flat, flat0 = pool.view(-1, d.D), before.view(-1, d.D)
+    changed = (flat.view(torch.int16) != flat0.view(torch.int16)).any(dim=1).nonzero().flatten().cpu().numpy()
+    expected = np.array([O.page_slot(bt, s, p, d.page_size) for s, p in zip(seq_idx, pos)])
+    assert sorted(changed.tolist()) == sorted(expected.tolist())
+    ref = O.kv_rows(W64["w_dkv_kr"], O.as64(h), pos, d)
+    got = to64(flat[torch.from_numpy(expected).cuda()])
+    assert_parity(got[:, :d.d_c], ref[:, :d.d_c], "c^KV")
+    assert_parity(got[:, d.d_c:], ref[:, d.d_c:], "k^R")
+
+
+def test_append_kv_bad_page_is_reported_and_skipped():
+    w = W_RUN
+    d = w.dims
+    W, _ = weights64(w)
+    bt = np.array([[0, -1], [1, 5]], dtype=np.int32)   # page 5 >= num_pages = 2
+    pool = torch.zeros((2, d.page_size, d.D), dtype=torch.bfloat16, device="cuda")
+    h = synth.hidden(w, batch=3).cuda()
+    M.append_kv(d, h, W["w_dkv_kr"].cuda(), torch.tensor([0, 0, 1], dtype=torch.int32, device="cuda"),
+                torch.tensor([3, 70, 65], dtype=torch.int32, device="cuda"), torch.from_numpy(bt).cuda(), pool)
+    assert M.read_device_status() == -7                     # MLA_ERR_BAD_PAGE
+    assert M.read_device_status() == 0                      # reading clears it
+    nz = (pool.view(-1, d.D) != 0).any(dim=1).nonzero().flatten().tolist()
+    assert nz == [3]                                        # only the valid token was written
+
+
+# ---------------------------------------------------------------------------------------- absorb
+@pytest.mark.parametrize("fam", list(FAMILIES))
+def test_absorb_query(fam):
+    w = FAMILIES[fam]
+    d = w.dims
+    W, W64 = weights64(w)
+    B = 19
+    h = synth.hidden(w, step=1, batch=B)
+    pos = np.array([0, 1, 2, 63, 64, 65, 255, 256, 4095, 4096, 4097, 32767, 32768, 65536, 100000, 131071,
+                    131072, 7, 12345], dtype=np.int32)
+    q = M.absorb_query(d, h.cuda(), W["w_dq"].cuda(), W["w_uq_qr"].cuda(), W["w_uk"].cuda(),
+                       torch.from_numpy(pos).cuda())
+    ref = O.absorb_query(W64["w_dq"], W64["w_uq_qr"], W64["w_uk"], O.as64(h), pos, d)
+    got = to64(q)
+    assert_parity(got[..., :d.d_c], ref[..., :d.d_c], "q~")
+    assert_parity(got[..., d.d_c:], ref[..., d.d_c:], "q^R")
+
+
+# ---------------------------------------------------------------------------------------- decode
+def run_decode(case, q, max_seq_len=None):
+    d = case.w.dims
+    seq_lens = torch.from_numpy(case.cached.astype(np.int32)).cuda()
+    msl = int(case.cached.max()) if max_seq_len is None else max_seq_len
+    return M.decode_attention(d, q.cuda(), case.pool, case.block_table, seq_lens, msl)
+
+
+def check_decode(case, q, o_lat, lse, what=""):
+    d = case.w.dims
+    q64 = O.as64(q)
+    for b in range(len(case.cached)):
+        ref_o, ref_l = O.latent_attention(q64[b], O.as64(case.prefix(b)), d)
+        assert_parity(to64(o_lat[b]), ref_o, f"{what} o_lat[b={b}]")
+        np.testing.assert_allclose(to64(lse[b]), ref_l, rtol=0, atol=2e-2, err_msg=f"{what} lse[b={b}]")
+
+
+@pytest.mark.parametrize("fam", list(FAMILIES))
+@pytest.mark.parametrize("scale", [1.0, 300.0], ids=["pages_law", "peaked"])
+def test_decode_attention_ragged_paged(fam, scale):
+    w = FAMILIES[fam]
+    lens = np.array([1, 2, 63, 64, 65, 129, 1000, 4097])
+    case = CacheCase(w, cached=lens, paging="shuffled", fill=float("nan"), spare_tokens=0)
+    q = synth.synthetic_query(w, len(lens), scale=scale)
+    o_lat, lse = run_decode(case, q)
+    assert M.read_device_status() == 0
+    check_decode(case, q, o_lat, lse, fam)
+
+
+def test_decode_split_plans_agree_and_are_deterministic():
+    w = W_PROD
+    lens = np.array([3000, 17, 4097])
+    case = CacheCase(w, cached=lens, paging="shuffled")
+    q = synth.synthetic_query(w, 3, scale=50.0)
+    a, la = run_decode(case, q)
+    b, lb = run_decode(case, q)
+    assert torch.equal(a, b) and torch.equal(la, lb)         # bitwise run to run
+    c, lc = run_decode(case, q, max_seq_len=int(lens.max()) + 60000)   # different split plan
+    assert_parity(to64(c), to64(a), "split plans")
+
+
+def test_decode_all_equal_rows_and_single_token_are_exact():
+    for w in (W_RUN16, W_PROD):
+        d = w.dims
+        lens = np.array([1, 300])
+        case = CacheCase(w, cached=lens)
+        row = case.rows[0].clone()
+        case.pool.view(-1, d.D)[:] = row               # every slot holds the same row
+        q = synth.synthetic_query(w, 2, scale=500.0)
+        o_lat, _ = run_decode(case, q)
+        expect = row[:d.d_c].expand_as(o_lat)
+        assert torch.equal(o_lat, expect)
+
+
+def test_decode_bad_seq_len_and_bad_page():
+    w = W_RUN
+    d = w.dims
+    lens = np.array([10, 20])
+    case = CacheCase(w, cached=lens)
+    q = synth.synthetic_query(w, 2).cuda()
+    seq_lens = torch.tensor([0, 20], dtype=torch.int32, device="cuda")
+    o_lat, _ = M.decode_attention(d, q, case.pool, case.block_table, seq_lens, 20)
+    assert M.read_device_status() == -8
+    assert torch.count_nonzero(o_lat[0]) == 0
+    ref, _ = O.latent_attention(O.as64(q[1]), O.as64(case.prefix(1)), d)
+    assert_parity(to64(o_lat[1]), ref, "other sequence")
+    bt = case.block_table.clone()
+    bt[1, 0] = case.num_pages + 3
+    M.decode_attention(d, q, case.pool, bt, torch.tensor([10, 20], dtype=torch.int32, device="cuda"), 20)
+    assert M.read_device_status() == -7
+
+
+# ---------------------------------------------------------------------------------------- out proj
+@pytest.mark.parametrize("fam", list(FAMILIES))
+def test_out_proj(fam):
+    w = FAMILIES[fam]
+    d = w.dims
+    W, W64 = weights64(w)
+    B = 13
+    rng = np.random.default_rng(7)
+    o_lat = synth.to_storage(rng.standard_normal((B, d.n_heads, d.d_c), dtype=np.float32) * 0.05, d)
+    u = M.out_proj(d, o_lat.cuda(), W["w_uv"].cuda(), W["w_o"].cuda())
+    ref = O.out_proj_absorbed(W64["w_uv"], W64["w_o"], O.as64(o_lat))
+    assert_parity(to64(u), ref, "u")
+
+
+# ---------------------------------------------------------------------------------------- one layer step
+def test_layer_step_running_model_fp16():
+    """The pages' running model, one layer, B=1, 256 cached tokens, fp16 (positions 0..255, new at 256)."""
+    w = W_RUN16
+    d = w.dims
+    cached = synth.cached_lengths(w)
+    L = harness.make_layer(w, cached)
+    ix = harness.step_index(cached)
+    h = synth.hidden(w)
+    u, q, o_lat, lse = M.layer_step(L.state, h.cuda(), ix.pos, ix.seq_idx, ix.seq_lens, ix.max_seq_len)
+    assert M.read_device_status() == 0
+    W64 = {k: O.as64(v) for k, v in L.W_host.items()}
+    prefix = [O.as64(L.prefix(b)) for b in range(w.batch)]
+    naive = O.layer_step_naive(W64, O.as64(h), prefix, d)
+    absd = O.layer_step_absorbed(W64, O.as64(h), prefix, d)
+    slot = O.page_slot(L.state.block_table.cpu().numpy(), 0, cached[0], d.page_size)
+    assert_parity(to64(L.state.pool.view(-1, d.D)[int(slot)])[None], naive["rows"], "new row")
+    assert_parity(to64(q)[..., :d.d_c], absd["q"][..., :d.d_c], "q~")
+    assert_parity(to64(q)[..., d.d_c:], absd["q"][..., d.d_c:], "q^R")
+    assert_parity(to64(o_lat), absd["o_lat"], "o_lat")
+    assert_parity(to64(u), naive["u"], "u")
