@@ -163,6 +163,32 @@ const char* mla_error_string(int code);
  * (for launch accounting in benchmarks). */
 int32_t mla_last_launch_count(int32_t call);
 
+/*
+ * mla_decode_attention_noalloc — mla_decode_attention without a caller-supplied workspace.
+ * The paper has no counterpart: it is a convenience for callers that cannot allocate device
+ * memory at the moment they run a decode step, such as a serving process whose device memory
+ * is reserved up front by its own allocator, code that must not stall on the device-wide
+ * synchronisation that cudaMalloc/cudaFree can cause, or a plain C caller with no workspace
+ * allocator of its own. The caller still passes q, the cache, the block table, the lengths
+ * and the outputs, with the same meaning, layout and checks as mla_decode_attention.
+ *
+ * The split-KV partials go to one static device array of the library instead:
+ * 64 MiB (67108864 bytes), created with the library's module on every GPU that loads it and
+ * held until the process exits. A call whose workspace need, mla_workspace_size(dims,
+ * MLA_CALL_DECODE_ATTENTION, B, max_seq_len), exceeds 64 MiB is rejected with
+ * MLA_ERR_WORKSPACE_TOO_SMALL before anything is queued. The call allocates nothing.
+ *
+ * The first call on a device looks up the array's device address (cudaGetSymbolAddress) with
+ * that device current; make that first call before any stream capture on the device.
+ * Every call on a device shares the one array and it keeps the last call's contents (no part
+ * of it needs to start at zero: every partial a call reads was written by that call), so calls
+ * whose work overlaps on the GPU race: keep them on one stream or order them yourself.
+ */
+int mla_decode_attention_noalloc(const mla_dims* dims, const void* q, const void* pool, int32_t num_pages,
+                                 const int32_t* block_table, int32_t max_pages, const int32_t* seq_lens,
+                                 int32_t B, int32_t max_seq_len, void* o_lat, float* lse_out,
+                                 mla_stream_t stream);
+
 #ifdef __cplusplus
 }
 #endif

@@ -16,7 +16,7 @@ from dataclasses import dataclass
 
 __all__ = [
     "MLAError", "load_library", "library_path", "c_dims", "workspace_size", "cache_elems_per_token",
-    "append_kv", "absorb_query", "decode_attention", "out_proj", "read_device_status", "last_launch_count",
+    "append_kv", "absorb_query", "decode_attention", "decode_attention_noalloc", "out_proj", "read_device_status", "last_launch_count",
     "LayerState", "layer_step", "CALL_APPEND_KV", "CALL_ABSORB_QUERY", "CALL_DECODE_ATTENTION", "CALL_OUT_PROJ",
 ]
 
@@ -53,6 +53,7 @@ _SIGS = {
     "mla_read_device_status": (ctypes.c_int, [_P, ctypes.POINTER(_I32)]),
     "mla_error_string": (ctypes.c_char_p, [ctypes.c_int]),
     "mla_last_launch_count": (_I32, [_I32]),
+    "mla_decode_attention_noalloc": (ctypes.c_int, [_P, _P, _P, _I32, _P, _I32, _P, _I32, _I32, _P, _P, _P]),
 }
 
 
@@ -185,6 +186,36 @@ def decode_attention(dims, q, pool, block_table, seq_lens, max_seq_len, o_lat=No
     _check(_lib().mla_decode_attention(ctypes.byref(cd), _ptr(q), _ptr(pool), pool.shape[0], _ptr(block_table),
                                        block_table.shape[1], _ptr(seq_lens), B, int(max_seq_len), _ptr(o_lat),
                                        _ptr(lse), _ptr(ws), nbytes, _stream(stream)), "mla_decode_attention")
+    return o_lat, lse
+
+
+def decode_attention_noalloc(dims, q, pool, block_table, seq_lens, max_seq_len, o_lat=None, lse=None,
+                             want_lse=True, stream=None):
+    """mla_decode_attention_noalloc: the same attention with the library's static scratch.
+
+    For callers that cannot allocate device memory when they decode (memory reserved up front
+    by their own allocator, no tolerance for cudaMalloc's synchronisation, no workspace
+    allocator). Problems needing more than 64 MiB of split-KV scratch raise MLAError (-3).
+    The scratch is shared by every call on the device: calls overlapping on the GPU race.
+    """
+    import torch
+    e = _elem(dims)
+    for t, n, dt in ((q, "q", e), (pool, "pool", e), (block_table, "block_table", torch.int32),
+                     (seq_lens, "seq_lens", torch.int32)):
+        _need(t, dt, n)
+    B = q.shape[0]
+    if o_lat is None:
+        o_lat = torch.empty((B, dims.n_heads, dims.d_c), dtype=e, device=q.device)
+    if lse is None and want_lse:
+        lse = torch.empty((B, dims.n_heads), dtype=torch.float32, device=q.device)
+    _need(o_lat, e, "o_lat")
+    if lse is not None:
+        _need(lse, torch.float32, "lse")
+    cd = c_dims(dims)
+    _check(_lib().mla_decode_attention_noalloc(ctypes.byref(cd), _ptr(q), _ptr(pool), pool.shape[0],
+                                               _ptr(block_table), block_table.shape[1], _ptr(seq_lens), B,
+                                               int(max_seq_len), _ptr(o_lat), _ptr(lse), _stream(stream)),
+           "mla_decode_attention_noalloc")
     return o_lat, lse
 
 

@@ -4,6 +4,7 @@
 // workspace, picks kernels and launches them on the caller's stream. It allocates nothing.
 #include <cmath>
 #include <cstring>
+#include <mutex>
 
 #include "common.cuh"
 #include "decode_simt.cuh"
@@ -354,5 +355,48 @@ const char* mla_error_string(int code) {
 }
 
 int32_t mla_last_launch_count(int32_t call) { return (call >= 0 && call < 4) ? t_launches[call] : -1; }
+
+}  // extern "C"
+
+// ---------------------------------------------------------------- allocation-free decode
+// Scratch of mla_decode_attention_noalloc: one file-scope device array per GPU that loads this
+// module. Host code must not pass the symbol itself to a kernel (on the host it names a
+// host-side stand-in); its device address is looked up once per device and cached.
+namespace {
+constexpr size_t kStaticScratchBytes = size_t(64) << 20;
+__device__ __align__(256) unsigned char g_decode_scratch[kStaticScratchBytes];
+
+std::mutex g_scratch_mu;
+void* g_scratch_addr[kMaxDevices] = {};
+
+int static_scratch_address(void** out) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return MLA_ERR_CUDA;
+  std::lock_guard<std::mutex> lock(g_scratch_mu);
+  if (g_scratch_addr[dev] == nullptr) {
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_decode_scratch) != cudaSuccess || p == nullptr) return MLA_ERR_CUDA;
+    g_scratch_addr[dev] = p;
+  }
+  *out = g_scratch_addr[dev];
+  return MLA_OK;
+}
+}  // namespace
+
+extern "C" {
+
+int mla_decode_attention_noalloc(const mla_dims* dims, const void* q, const void* pool, int32_t num_pages,
+                                 const int32_t* block_table, int32_t max_pages, const int32_t* seq_lens, int32_t B,
+                                 int32_t max_seq_len, void* o_lat, float* lse_out, mla_stream_t stream) {
+  const int r = check_dims_impl(dims);
+  if (r != MLA_OK) return r;
+  if (B > 0 && max_seq_len >= 1 && ws_decode(dims, B, max_seq_len) > kStaticScratchBytes)
+    return MLA_ERR_WORKSPACE_TOO_SMALL;
+  void* ws = nullptr;
+  const int s = static_scratch_address(&ws);
+  if (s != MLA_OK) return s;
+  return mla_decode_attention(dims, q, pool, num_pages, block_table, max_pages, seq_lens, B, max_seq_len, o_lat,
+                              lse_out, ws, kStaticScratchBytes, stream);
+}
 
 }  // extern "C"
