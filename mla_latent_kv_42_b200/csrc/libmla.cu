@@ -8,7 +8,7 @@
 
 #include "common.cuh"
 #include "decode_simt.cuh"
-#include "proj_simt.cuh"
+#include "proj_host.cuh"
 
 using namespace mla;
 
@@ -32,7 +32,6 @@ int device_sm_count() {
 
 inline bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 inline size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
-inline size_t esize(const mla_dims* d) { (void)d; return 2; }
 
 // Sequential sub-allocation of the caller's workspace (256-byte aligned pieces).
 struct Carve {
@@ -79,14 +78,9 @@ DecodePlan plan_decode(const mla_dims* d, int B, int max_seq_len) {
   return p;
 }
 
-size_t ws_append(const mla_dims* d, int T) { return T > 0 ? align256((size_t)T * (d->d_c + d->d_rope) * 4) : 0; }
-
-size_t ws_absorb(const mla_dims* d, int B) {
-  if (B <= 0) return 0;
-  const size_t nq = (size_t)d->n_heads * (d->d_head + d->d_rope);
-  return align256((size_t)B * d->d_cq * esize(d)) + align256((size_t)B * nq * 4) +
-         align256((size_t)B * d->n_heads * d->d_head * esize(d));
-}
+size_t ws_append(const mla_dims* d, int T) { return T > 0 ? host::append_layout(d, T, nullptr).bytes : 0; }
+size_t ws_absorb(const mla_dims* d, int B) { return B > 0 ? host::absorb_layout(d, B, nullptr).bytes : 0; }
+size_t ws_out(const mla_dims* d, int B) { return B > 0 ? host::out_layout(d, B, nullptr).bytes : 0; }
 
 size_t ws_decode(const mla_dims* d, int B, int max_seq_len) {
   if (B <= 0 || max_seq_len <= 0) return 0;
@@ -94,22 +88,6 @@ size_t ws_decode(const mla_dims* d, int B, int max_seq_len) {
   if (p.n_splits == 1) return 0;
   const size_t bh = (size_t)B * d->n_heads;
   return align256(bh * p.n_splits * d->d_c * 4) + align256(bh * p.n_splits * 4);
-}
-
-size_t ws_out(const mla_dims* d, int B) {
-  return B > 0 ? align256((size_t)B * d->n_heads * d->d_head * esize(d)) : 0;
-}
-
-template <typename T, typename OutT>
-void launch_rowdot(const T* W, const T* X, OutT* Y, int M, int K, int Tn, long ldx, long ldy, int batch, long sW,
-                   long sX, long sY, cudaStream_t st, int32_t& launches) {
-  if (Tn <= 0 || M <= 0 || batch <= 0) return;
-  dim3 grid((M + 7) / 8, 1, batch);
-  if (Tn <= 8)
-    k_rowdot<T, OutT, 8><<<grid, 256, 0, st>>>(W, X, Y, M, K, Tn, ldx, ldy, sW, sX, sY);
-  else
-    k_rowdot<T, OutT, 16><<<grid, 256, 0, st>>>(W, X, Y, M, K, Tn, ldx, ldy, sW, sX, sY);
-  ++launches;
 }
 
 int finish_launches(int call, int32_t launches) {
@@ -123,39 +101,18 @@ template <typename T>
 int append_impl(const mla_dims* d, const void* h, const void* w, const int32_t* seq_idx, const int32_t* pos,
                 const int32_t* bt, int32_t num_seqs, int32_t max_pages, void* pool, int32_t num_pages, int32_t T_,
                 void* ws, cudaStream_t st) {
-  const int D = d->d_c + d->d_rope;
   int32_t n = 0;
-  Carve c{static_cast<char*>(ws)};
-  float* Y = c.take<float>((size_t)T_ * D);
-  launch_rowdot<T, float>(static_cast<const T*>(w), static_cast<const T*>(h), Y, D, d->d_model, T_, d->d_model, D,
-                          1, 0, 0, 0, st, n);
-  k_append_epilogue<T><<<T_, 128, 0, st>>>(Y, seq_idx, pos, bt, num_seqs, max_pages, static_cast<T*>(pool), num_pages,
-                                          d->page_size, d->d_c, d->d_rope, d->rope_base);
-  ++n;
+  const int r = host::append_run<T>(d, h, w, seq_idx, pos, bt, num_seqs, max_pages, pool, num_pages, T_, ws, st, n);
+  if (r != MLA_OK) return r;
   return finish_launches(MLA_CALL_APPEND_KV, n);
 }
 
 template <typename T>
 int absorb_impl(const mla_dims* d, const void* h, const void* w_dq, const void* w_uq_qr, const void* w_uk,
                 const int32_t* pos, void* q_out, int32_t B, void* ws, cudaStream_t st) {
-  const int nq = d->n_heads * (d->d_head + d->d_rope);
-  const int D = d->d_c + d->d_rope;
   int32_t n = 0;
-  Carve c{static_cast<char*>(ws)};
-  T* cq = c.take<T>((size_t)B * d->d_cq);
-  float* Y2 = c.take<float>((size_t)B * nq);
-  T* qc = c.take<T>((size_t)B * d->n_heads * d->d_head);
-  launch_rowdot<T, T>(static_cast<const T*>(w_dq), static_cast<const T*>(h), cq, d->d_cq, d->d_model, B, d->d_model,
-                      d->d_cq, 1, 0, 0, 0, st, n);
-  launch_rowdot<T, float>(static_cast<const T*>(w_uq_qr), cq, Y2, nq, d->d_cq, B, d->d_cq, nq, 1, 0, 0, 0, st, n);
-  k_query_epilogue<T><<<B, 256, 0, st>>>(Y2, pos, qc, static_cast<T*>(q_out), d->n_heads, d->d_head, d->d_rope,
-                                         d->d_c, d->rope_base);
-  ++n;
-  const int threads = 128;
-  dim3 grid((d->d_c / 2 + threads - 1) / threads, d->n_heads);
-  k_absorb_uk<T, 16><<<grid, threads, 16 * d->d_head * sizeof(float), st>>>(
-      static_cast<const T*>(w_uk), qc, static_cast<T*>(q_out), B, d->n_heads, d->d_head, d->d_c, D);
-  ++n;
+  const int r = host::absorb_run<T>(d, h, w_dq, w_uq_qr, w_uk, pos, q_out, B, ws, st, n);
+  if (r != MLA_OK) return r;
   return finish_launches(MLA_CALL_ABSORB_QUERY, n);
 }
 
@@ -207,15 +164,9 @@ int decode_impl(const mla_dims* d, const void* q, const void* pool, int32_t num_
 template <typename T>
 int out_impl(const mla_dims* d, const void* o_lat, const void* w_uv, const void* w_o, void* u, int32_t B, void* ws,
              cudaStream_t st) {
-  const int nhd = d->n_heads * d->d_head;
   int32_t n = 0;
-  Carve c{static_cast<char*>(ws)};
-  T* o = c.take<T>((size_t)B * nhd);
-  // o_i = W^UV_i o_lat_i, batched over heads (row block i of W^UV, head i of o_lat)
-  launch_rowdot<T, T>(static_cast<const T*>(w_uv), static_cast<const T*>(o_lat), o, d->d_head, d->d_c, B,
-                      (long)d->n_heads * d->d_c, nhd, d->n_heads, (long)d->d_head * d->d_c, d->d_c, d->d_head, st, n);
-  launch_rowdot<T, T>(static_cast<const T*>(w_o), o, static_cast<T*>(u), d->d_model, nhd, B, nhd, d->d_model, 1, 0,
-                      0, 0, st, n);
+  const int r = host::out_run<T>(d, o_lat, w_uv, w_o, u, B, ws, st, n);
+  if (r != MLA_OK) return r;
   return finish_launches(MLA_CALL_OUT_PROJ, n);
 }
 

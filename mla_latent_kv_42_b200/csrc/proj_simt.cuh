@@ -86,12 +86,13 @@ __global__ void __launch_bounds__(256) k_absorb_uk(const T* __restrict__ w_uk, c
 }
 
 // Cache-write epilogue of mla_append_kv: row = [c ‖ RoPE(k^, pos)] rounded, stored at the
-// token's paged slot. Y is the fp32 product [T, D]. One block per token.
+// token's paged slot. Y holds `splits` fp32 partial products [T, D], `split_off` apart, summed
+// in split order. One block per token.
 template <typename T>
-__global__ void k_append_epilogue(const float* __restrict__ Y, const int* __restrict__ seq_idx,
-                                  const int* __restrict__ pos, const int* __restrict__ bt, int num_seqs,
-                                  int max_pages, T* __restrict__ pool, int num_pages, int page_size, int d_c,
-                                  int d_rope, double base) {
+__global__ void k_append_epilogue(const float* __restrict__ Y, int splits, long split_off,
+                                  const int* __restrict__ seq_idx, const int* __restrict__ pos,
+                                  const int* __restrict__ bt, int num_seqs, int max_pages, T* __restrict__ pool,
+                                  int num_pages, int page_size, int d_c, int d_rope, double base) {
   using P = Pack<T>;
   const int t = blockIdx.x;
   const int D = d_c + d_rope;
@@ -106,7 +107,11 @@ __global__ void k_append_epilogue(const float* __restrict__ Y, const int* __rest
   T* row = pool + ((long)page * page_size + p % page_size) * D;
   const float* y = Y + (long)t * D;
   for (int e = threadIdx.x; e < D / 2; e += blockDim.x) {
-    float a = y[2 * e], b = y[2 * e + 1];
+    float a = 0.f, b = 0.f;
+    for (int k = 0; k < splits; ++k) {
+      a += y[k * split_off + 2 * e];
+      b += y[k * split_off + 2 * e + 1];
+    }
     if (2 * e >= d_c) {
       float c, sn;
       rope_cos_sin(p, e - d_c / 2, d_rope, base, c, sn);
@@ -118,11 +123,13 @@ __global__ void k_append_epilogue(const float* __restrict__ Y, const int* __rest
   }
 }
 
-// Query epilogue of mla_absorb_query: Y = [q^C ; q^] fp32 [B, n_h*(d_h + d_r)].
-// q^C -> qc (element type, [B, n_h*d_h]); q^R_i = RoPE(q^_i, pos[b]) -> q_out[b][i][d_c:].
+// Query epilogue of mla_absorb_query: Y = [q^C ; q^] fp32 [B, n_h*(d_h + d_r)] as `splits`
+// partials `split_off` apart (summed in order). q^C -> qc (element type, [B, n_h*d_h]);
+// q^R_i = RoPE(q^_i, pos[b]) -> q_out[b][i][d_c:].
 template <typename T>
-__global__ void k_query_epilogue(const float* __restrict__ Y, const int* __restrict__ pos, T* __restrict__ qc,
-                                 T* __restrict__ q_out, int n_h, int d_h, int d_r, int d_c, double base) {
+__global__ void k_query_epilogue(const float* __restrict__ Y, int splits, long split_off, const int* __restrict__ pos,
+                                 T* __restrict__ qc, T* __restrict__ q_out, int n_h, int d_h, int d_r, int d_c,
+                                 double base) {
   using P = Pack<T>;
   using T2 = typename P::T2;
   const int b = blockIdx.x;
@@ -130,7 +137,11 @@ __global__ void k_query_epilogue(const float* __restrict__ Y, const int* __restr
   const float* y = Y + (long)b * n_h * (d_h + d_r);
   const int p = pos[b];
   for (int e = threadIdx.x; e < n_h * (d_h + d_r) / 2; e += blockDim.x) {
-    const float a = y[2 * e], c2 = y[2 * e + 1];
+    float a = 0.f, c2 = 0.f;
+    for (int k = 0; k < splits; ++k) {
+      a += y[k * split_off + 2 * e];
+      c2 += y[k * split_off + 2 * e + 1];
+    }
     if (2 * e < nc) {
       reinterpret_cast<T2*>(qc + (long)b * nc)[e] = P::make(a, c2);
     } else {
