@@ -30,9 +30,6 @@ struct GemmParams {
   int out_f32;        // 1: fp32 output (partials or fp32 result), 0: element type
 };
 
-template <typename T> struct IsBf16 { static constexpr bool value = false; };
-template <> struct IsBf16<__nv_bfloat16> { static constexpr bool value = true; };
-
 template <int BN>
 struct GemmCfg {
   static constexpr int BM = 128, BK = 64;

@@ -8,6 +8,7 @@
 
 #include "common.cuh"
 #include "decode_simt.cuh"
+#include "decode_tc.cuh"
 #include "proj_host.cuh"
 
 using namespace mla;
@@ -82,14 +83,6 @@ size_t ws_append(const mla_dims* d, int T) { return T > 0 ? host::append_layout(
 size_t ws_absorb(const mla_dims* d, int B) { return B > 0 ? host::absorb_layout(d, B, nullptr).bytes : 0; }
 size_t ws_out(const mla_dims* d, int B) { return B > 0 ? host::out_layout(d, B, nullptr).bytes : 0; }
 
-size_t ws_decode(const mla_dims* d, int B, int max_seq_len) {
-  if (B <= 0 || max_seq_len <= 0) return 0;
-  const DecodePlan p = plan_decode(d, B, max_seq_len);
-  if (p.n_splits == 1) return 0;
-  const size_t bh = (size_t)B * d->n_heads;
-  return align256(bh * p.n_splits * d->d_c * 4) + align256(bh * p.n_splits * 4);
-}
-
 int finish_launches(int call, int32_t launches) {
   const cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return MLA_ERR_CUDA;
@@ -116,6 +109,102 @@ int absorb_impl(const mla_dims* d, const void* h, const void* w_dq, const void* 
   return finish_launches(MLA_CALL_ABSORB_QUERY, n);
 }
 
+// ---------------------------------------------------------------- tensor-core decode
+// The tcgen05 path serves DeepSeek-V2-shaped caches (d_c = 512, d_h^R = 64, 64-token pages,
+// 65..128 heads); MLA_DECODE_IMPL=simt selects the CUDA-core kernel instead.
+bool decode_tc_eligible(const mla_dims* d) {
+  static int forced_simt = -1;
+  if (forced_simt < 0) {
+    const char* e = std::getenv("MLA_DECODE_IMPL");
+    forced_simt = (e != nullptr && std::strcmp(e, "simt") == 0) ? 1 : 0;
+  }
+  return !forced_simt && d->n_heads > 64 && d->n_heads <= 128 && d->d_c == tc::dec::kDc &&
+         d->d_c + d->d_rope == tc::dec::kD && d->page_size == tc::dec::kPage;
+}
+
+template <typename T>
+bool decode_tc_set_smem() {
+  static bool done[kMaxDevices] = {};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return false;
+  if (!done[dev]) {
+    if (cudaFuncSetAttribute(tc::k_decode_tc<T>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)tc::dec::kSmem) !=
+        cudaSuccess)
+      return false;
+    done[dev] = true;
+  }
+  return true;
+}
+
+// Clusters of two CTAs that can be resident at once: the work is split statically over them.
+int decode_clusters() {
+  static int cache[kMaxDevices] = {0};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return device_sm_count() / 2;
+  if (cache[dev] == 0) {
+    int n = 0;
+    if (decode_tc_set_smem<__nv_bfloat16>()) {
+      cudaLaunchConfig_t cfg = {};
+      cfg.gridDim = dim3(2 * (device_sm_count() / 2), 1, 1);
+      cfg.blockDim = dim3(tc::dec::kThreads, 1, 1);
+      cfg.dynamicSmemBytes = tc::dec::kSmem;
+      if (cudaOccupancyMaxActiveClusters(&n, tc::k_decode_tc<__nv_bfloat16>, &cfg) != cudaSuccess) n = 0;
+    }
+    cudaGetLastError();
+    cache[dev] = n > 0 ? n : device_sm_count() / 2;
+  }
+  return cache[dev];
+}
+
+size_t ws_decode_tc(const mla_dims* d, int B) {
+  const size_t slots = (size_t)B + decode_clusters();
+  return align256((size_t)(B + 1) * 4) + align256(slots * d->n_heads * tc::dec::kDc * 4) +
+         align256(slots * d->n_heads * 4);
+}
+
+size_t ws_decode(const mla_dims* d, int B, int max_seq_len) {
+  if (B <= 0 || max_seq_len <= 0) return 0;
+  if (decode_tc_eligible(d)) return ws_decode_tc(d, B);
+  const DecodePlan p = plan_decode(d, B, max_seq_len);
+  if (p.n_splits == 1) return 0;
+  const size_t bh = (size_t)B * d->n_heads;
+  return align256(bh * p.n_splits * d->d_c * 4) + align256(bh * p.n_splits * 4);
+}
+
+template <typename T>
+int decode_tc_impl(const mla_dims* d, const void* q, const void* pool, int32_t num_pages, const int32_t* bt,
+                   int32_t max_pages, const int32_t* seq_lens, int32_t B, int32_t max_seq_len, void* o_lat,
+                   float* lse_out, void* ws, cudaStream_t st) {
+  const int C = decode_clusters();
+  if (!decode_tc_set_smem<T>()) return MLA_ERR_CUDA;
+  Carve c{static_cast<char*>(ws)};
+  int* prefix = c.take<int>((size_t)B + 1);
+  float* o_part = c.take<float>(((size_t)B + C) * d->n_heads * tc::dec::kDc);
+  float* lse_part = c.take<float>(((size_t)B + C) * d->n_heads);
+  CUtensorMap map;
+  if (!host::encode_2d(&map, pool, tc::IsBf16<T>::value, tc::dec::kD, (uint64_t)num_pages * tc::dec::kPage,
+                       tc::dec::kD * 2, 64, 64))
+    return MLA_ERR_CUDA;
+  tc::k_decode_plan<<<1, 1024, 0, st>>>(seq_lens, bt, B, max_pages, num_pages, max_seq_len, prefix);
+  tc::DecodeTcParams p;
+  p.q = q;
+  p.bt = bt;
+  p.max_pages = max_pages;
+  p.seq_lens = seq_lens;
+  p.tile_prefix = prefix;
+  p.B = B;
+  p.n_h = d->n_heads;
+  p.scale_log2 = (float)(1.4426950408889634 / std::sqrt((double)(d->d_head + d->d_rope)));
+  p.o_lat = o_lat;
+  p.lse_out = lse_out;
+  p.o_part = o_part;
+  p.lse_part = lse_part;
+  tc::k_decode_tc<T><<<2 * C, tc::dec::kThreads, tc::dec::kSmem, st>>>(map, p);
+  tc::k_decode_tc_merge<T><<<dim3(B, d->n_heads), 128, 0, st>>>(o_part, lse_part, prefix, B, C, d->n_heads,
+                                                               static_cast<T*>(o_lat), lse_out);
+  return finish_launches(MLA_CALL_DECODE_ATTENTION, 3);
+}
+
 template <typename T, int NPAIR>
 void launch_decode_simt(const mla_dims* d, const DecodePlan& p, const void* q, const void* pool, int32_t num_pages,
                         const int32_t* bt, int32_t max_pages, const int32_t* seq_lens, int32_t B, int32_t max_seq_len,
@@ -132,6 +221,8 @@ template <typename T>
 int decode_impl(const mla_dims* d, const void* q, const void* pool, int32_t num_pages, const int32_t* bt,
                 int32_t max_pages, const int32_t* seq_lens, int32_t B, int32_t max_seq_len, void* o_lat,
                 float* lse_out, void* ws, cudaStream_t st) {
+  if (decode_tc_eligible(d))
+    return decode_tc_impl<T>(d, q, pool, num_pages, bt, max_pages, seq_lens, B, max_seq_len, o_lat, lse_out, ws, st);
   const DecodePlan p = plan_decode(d, B, max_seq_len);
   const size_t bh = (size_t)B * d->n_heads;
   float* o_part = nullptr;

@@ -225,7 +225,7 @@ int append_run(const mla_dims* d, const void* h, const void* w, const int32_t* s
     ++n;
     splits = L.g.splits;
   }
-  k_append_epilogue<T><<<T_, 128, 0, st>>>(L.Y, splits, (long)T_ * D, seq_idx, pos, bt, num_seqs, max_pages,
+  k_append_epilogue<T><<<T_, 128, (d->d_rope / 2) * sizeof(float2), st>>>(L.Y, splits, (long)T_ * D, seq_idx, pos, bt, num_seqs, max_pages,
                                           static_cast<T*>(pool), num_pages, d->page_size, d->d_c, d->d_rope,
                                           d->rope_base);
   ++n;
@@ -295,7 +295,7 @@ int absorb_run(const mla_dims* d, const void* h, const void* w_dq, const void* w
     ++n;
     splits2 = L.g2.splits;
   }
-  k_query_epilogue<T><<<B, 256, 0, st>>>(L.Y2, splits2, (long)B * nq, pos, qc, static_cast<T*>(q_out), d->n_heads,
+  k_query_epilogue<T><<<B, 256, (d->d_rope / 2) * sizeof(float2), st>>>(L.Y2, splits2, (long)B * nq, pos, qc, static_cast<T*>(q_out), d->n_heads,
                                          d->d_head, d->d_rope, d->d_c, d->rope_base);
   ++n;
   // q~_i = (W^UK_i)^T q^C_i

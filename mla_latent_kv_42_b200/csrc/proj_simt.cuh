@@ -106,6 +106,9 @@ __global__ void k_append_epilogue(const float* __restrict__ Y, int splits, long 
   }
   T* row = pool + ((long)page * page_size + p % page_size) * D;
   const float* y = Y + (long)t * D;
+  extern __shared__ float2 cs[];  // cos/sin of each RoPE pair at this position
+  for (int k = threadIdx.x; k < d_rope / 2; k += blockDim.x) rope_cos_sin(p, k, d_rope, base, cs[k].x, cs[k].y);
+  __syncthreads();
   for (int e = threadIdx.x; e < D / 2; e += blockDim.x) {
     float a = 0.f, b = 0.f;
     for (int k = 0; k < splits; ++k) {
@@ -113,9 +116,8 @@ __global__ void k_append_epilogue(const float* __restrict__ Y, int splits, long 
       b += y[k * split_off + 2 * e + 1];
     }
     if (2 * e >= d_c) {
-      float c, sn;
-      rope_cos_sin(p, e - d_c / 2, d_rope, base, c, sn);
-      const float ra = a * c - b * sn, rb = a * sn + b * c;
+      const float2 r = cs[e - d_c / 2];
+      const float ra = a * r.x - b * r.y, rb = a * r.y + b * r.x;
       a = ra;
       b = rb;
     }
@@ -136,6 +138,9 @@ __global__ void k_query_epilogue(const float* __restrict__ Y, int splits, long s
   const int nc = n_h * d_h, D = d_c + d_r;
   const float* y = Y + (long)b * n_h * (d_h + d_r);
   const int p = pos[b];
+  extern __shared__ float2 cs[];  // cos/sin of each RoPE pair at this position (shared by all heads)
+  for (int k = threadIdx.x; k < d_r / 2; k += blockDim.x) rope_cos_sin(p, k, d_r, base, cs[k].x, cs[k].y);
+  __syncthreads();
   for (int e = threadIdx.x; e < n_h * (d_h + d_r) / 2; e += blockDim.x) {
     float a = 0.f, c2 = 0.f;
     for (int k = 0; k < splits; ++k) {
@@ -147,9 +152,9 @@ __global__ void k_query_epilogue(const float* __restrict__ Y, int splits, long s
     } else {
       const int r = 2 * e - nc;  // index inside the W^QR block
       const int i = r / d_r, k = (r % d_r) / 2;
-      float c, s;
-      rope_cos_sin(p, k, d_r, base, c, s);
-      reinterpret_cast<T2*>(q_out + ((long)b * n_h + i) * D + d_c)[k] = P::make(a * c - c2 * s, a * s + c2 * c);
+      const float2 q = cs[k];
+      reinterpret_cast<T2*>(q_out + ((long)b * n_h + i) * D + d_c)[k] =
+          P::make(a * q.x - c2 * q.y, a * q.y + c2 * q.x);
     }
   }
 }

@@ -129,6 +129,17 @@ def test_decode_attention_ragged_paged(fam, scale):
     check_decode(case, q, o_lat, lse, fam)
 
 
+def test_decode_fewer_pages_than_sm_pairs():
+    """A handful of pages spread over many SM pairs: most pairs own no page at all."""
+    w = W_PROD
+    lens = np.array([1, 130, 200, 64])
+    case = CacheCase(w, cached=lens, paging="shuffled", fill=float("nan"), spare_tokens=0)
+    q = synth.synthetic_query(w, len(lens), scale=40.0)
+    o_lat, lse = run_decode(case, q)
+    assert M.read_device_status() == 0
+    check_decode(case, q, o_lat, lse, "few pages")
+
+
 def test_decode_split_plans_agree_and_are_deterministic():
     w = W_PROD
     lens = np.array([3000, 17, 4097])
