@@ -179,6 +179,28 @@ def run_reference(args):
     return 0
 
 
+# ----------------------------------------------------------------------------------- multi-rank helpers
+def rank_workload(w, rank: int):
+    """Each rank owns its own sequences: the same workload shape with a rank-specific seed."""
+    import dataclasses
+    return dataclasses.replace(w, seed=w.seed + 1000 * rank) if rank else w
+
+
+def max_over_ranks(values, device, world: int):
+    """Element-wise MAX over ranks of per-rank device times (a plain list when world == 1)."""
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor(list(values), dtype=torch.float64, device=device)
+    if world > 1:
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return t.tolist()
+
+
+def job_us_per_layer_step(ms_total: float, steps: int, layers: int, world: int) -> float:
+    """µs per layer-step of the whole job: every rank advances its own batch one layer per layer-step."""
+    return ms_total / steps * 1e3 / layers / world
+
+
 # ----------------------------------------------------------------------------------- GPU arm
 def run_mla(args):
     import torch
@@ -203,7 +225,7 @@ def run_mla(args):
         dist.barrier()
     M.load_library()
 
-    w = synth.workload(args.workload)
+    w = rank_workload(synth.workload(args.workload), rank)
     d = w.dims
     cached = synth.cached_lengths(w)
     ix = harness.step_index(cached, device=dev)
@@ -314,16 +336,13 @@ def run_mla(args):
     assert M.read_device_status(stream) == 0
 
     # max over ranks
-    t = torch.tensor([ms_total, ms_e2e, call_ms[2]], dtype=torch.float64, device=dev)
-    if world > 1:
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-    ms_total, ms_e2e, decode_ms = t.tolist()
+    ms_total, ms_e2e, decode_ms = max_over_ranks([ms_total, ms_e2e, call_ms[2]], dev, world)
 
     if rank == 0:
         peaks, peak_src = load_peaks()
         ms_step = ms_total / args.steps
-        us_layer_job = ms_step * 1e3 / len(layers) / world
-        us_e2e_job = ms_e2e / args.steps * 1e3 / len(layers) / world
+        us_layer_job = job_us_per_layer_step(ms_total, args.steps, len(layers), world)
+        us_e2e_job = job_us_per_layer_step(ms_e2e, args.steps, len(layers), world)
         seq_lens = cached + 1
         dbytes, dflops = harness.decode_work(d, seq_lens)
         sbytes, sflops = harness.step_work(d, seq_lens)
