@@ -55,7 +55,11 @@ struct Ctrl {
   uint64_t stats_empty;      // score CTA; arrived remotely by the value CTA
   uint64_t p_full[kPBufs];   // value CTA; armed and completed by the score CTA's bulk copy
   uint64_t p_ready[kPBufs];  // value CTA
-  uint64_t o_done, stats_full, o_free, drain;
+  // value CTA: O complete through the last tile that used P buffer pb. One barrier per P buffer
+  // keeps every parity wait on it at most one phase behind: the P ring only guarantees that the
+  // MMAs of tile t-2 are done when tile t's P arrives, so one shared barrier could lag by two.
+  uint64_t o_done[kPBufs];
+  uint64_t stats_full, o_free, drain;
   float stats[128][2];       // value CTA: reference max (log2 units) and denominator
   uint32_t tmem_slot;
   int abort_flag;
@@ -145,9 +149,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(dec::kThreads, 1)
       mbar_init(bar(ctl->p_empty[i]), 1);
       mbar_init(bar(ctl->p_full[i]), 1);
       mbar_init(bar(ctl->p_ready[i]), 128);
+      mbar_init(bar(ctl->o_done[i]), 1);
     }
     mbar_init(bar(ctl->stats_empty), 128);
-    mbar_init(bar(ctl->o_done), 1);
     mbar_init(bar(ctl->stats_full), 128);
     mbar_init(bar(ctl->o_free), 128);
     mbar_init(bar(ctl->drain), 1);
@@ -487,7 +491,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(dec::kThreads, 1)
               }
             if (ok && lane == 0) {
               mma_commit_mc(bar(ctl->p_empty[pb]), (uint16_t)1u);  // P buffer free: tell the score CTA
-              mma_commit(bar(ctl->o_done));
+              mma_commit(bar(ctl->o_done[pb]));
             }
             __syncwarp();
           }
@@ -510,7 +514,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(dec::kThreads, 1)
             }
             const float alpha = reinterpret_cast<const float*>(data + kPOff + pb * kPStride + kPTile)[h];
             if (t != item.t0 && __any_sync(0xffffffffu, alpha != 1.f)) {
-              if (!wwait(ctl->o_done, (tile - 1) & 1)) {
+              if (!wwait(ctl->o_done[(tile - 1) % kPBufs], ((tile - 1) / kPBufs) & 1)) {
                 ok = false;
                 break;
               }
@@ -533,7 +537,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(dec::kThreads, 1)
           if (!wwait_cl(ctl->stats_full, item_i & 1)) break;
           const float m_ref = ctl->stats[h][0], l = ctl->stats[h][1];
           mbar_arrive_remote(stats_empty_remote);
-          if (!wwait(ctl->o_done, (tile - 1) & 1)) break;
+          // O holds every tile of the item once the last one is done; the other buffer's last
+          // arrival is waited for as well so that none is still in flight when the CTA exits
+          if (!wwait(ctl->o_done[(tile - 1) % kPBufs], ((tile - 1) / kPBufs) & 1)) break;
+          if (tile >= 2 && !wwait(ctl->o_done[(tile - 2) % kPBufs], ((tile - 2) / kPBufs) & 1)) break;
           tc_fence_after();
           const float inv = l > 0.f ? 1.f / l : 0.f;
           const float lse = l > 0.f ? (m_ref + log2f(l)) * 0.6931471805599453f : -INFINITY;
@@ -647,43 +654,65 @@ __global__ void __launch_bounds__(1024) k_decode_plan(const int* __restrict__ se
   if (tid == 1023) tile_prefix[B] = part[1023];
 }
 
-// Merge of the partials of sequences that span clusters (fixed cluster order); zero output for
-// rejected sequences. grid (B, n_h), 128 threads.
+// Merge of the partials of sequences that span clusters, in cluster order; zero output for
+// rejected sequences. grid (B, ceil(n_h / 8)), 256 threads: one warp per head, each lane 16 of
+// the 512 latent values (four 16-byte loads per contributing cluster, all in flight together).
 template <typename T>
-__global__ void k_decode_tc_merge(const float* __restrict__ o_part, const float* __restrict__ lse_part,
-                                  const int* __restrict__ tile_prefix, int B, int C, int n_h, T* __restrict__ o_lat,
-                                  float* __restrict__ lse_out) {
-  const int b = blockIdx.x, h = blockIdx.y;
+__global__ void __launch_bounds__(256) k_decode_tc_merge(const float* __restrict__ o_part,
+                                                          const float* __restrict__ lse_part,
+                                                          const int* __restrict__ tile_prefix, int B, int C, int n_h,
+                                                          T* __restrict__ o_lat, float* __restrict__ lse_out) {
+  const int b = blockIdx.x, warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int h = blockIdx.y * 8 + warp;
+  if (h >= n_h) return;
   const long T_ = tile_prefix[B];
   const int g0 = tile_prefix[b], g1 = tile_prefix[b + 1];
   T* out = o_lat + ((long)b * n_h + h) * dec::kDc;
   if (g1 == g0) {
-    for (int e = threadIdx.x; e < dec::kDc; e += blockDim.x) Out<T>::put(out + e, 0.f);
-    if (lse_out != nullptr && threadIdx.x == 0) lse_out[(long)b * n_h + h] = -INFINITY;
+    for (int e = lane; e < dec::kDc; e += 32) Out<T>::put(out + e, 0.f);
+    if (lse_out != nullptr && lane == 0) lse_out[(long)b * n_h + h] = -INFINITY;
     return;
   }
   const int c0 = cluster_of(g0, T_, C), c1 = cluster_of(g1 - 1, T_, C);
   if (c0 == c1) return;  // written whole by its cluster
-  // Clusters between c0 and c1 own consecutive pages of this sequence, except those whose
-  // range is empty (fewer pages than clusters): they wrote nothing and are skipped.
+  // clusters between c0 and c1 own consecutive pages of this sequence, except those whose range
+  // is empty (fewer pages than clusters): they wrote nothing and are skipped
   auto owns = [&](int c) { return T_ * (c + 1) / C > T_ * c / C; };
+  const float* lp = lse_part + (long)b * n_h + h;  // slot b + c is at lp[c * n_h]
   float mx = -INFINITY;
   for (int c = c0; c <= c1; ++c)
-    if (owns(c)) mx = fmaxf(mx, lse_part[((long)b + c) * n_h + h]);
+    if (owns(c)) mx = fmaxf(mx, lp[(long)c * n_h]);
   float z = 0.f;
   for (int c = c0; c <= c1; ++c)
-    if (owns(c)) z += exp2f((lse_part[((long)b + c) * n_h + h] - mx) * 1.4426950408889634f);
+    if (owns(c)) z += exp2f((lp[(long)c * n_h] - mx) * 1.4426950408889634f);
   const float inv = 1.f / z;
-  for (int e = threadIdx.x; e < dec::kDc; e += blockDim.x) {
-    float acc = 0.f;
-    for (int c = c0; c <= c1; ++c) {
-      if (!owns(c)) continue;
-      const float w = exp2f((lse_part[((long)b + c) * n_h + h] - mx) * 1.4426950408889634f);
-      acc = fmaf(w, o_part[(((long)b + c) * n_h + h) * dec::kDc + e], acc);
+  float4 acc[4];
+#pragma unroll
+  for (int j = 0; j < 4; ++j) acc[j] = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll 2
+  for (int c = c0; c <= c1; ++c) {
+    if (!owns(c)) continue;
+    const float w = exp2f((lp[(long)c * n_h] - mx) * 1.4426950408889634f);
+    const float4* src = reinterpret_cast<const float4*>(o_part + (((long)b + c) * n_h + h) * dec::kDc);
+    float4 v[4];
+#pragma unroll
+    for (int j = 0; j < 4; ++j) v[j] = src[lane + 32 * j];
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      acc[j].x = fmaf(w, v[j].x, acc[j].x);
+      acc[j].y = fmaf(w, v[j].y, acc[j].y);
+      acc[j].z = fmaf(w, v[j].z, acc[j].z);
+      acc[j].w = fmaf(w, v[j].w, acc[j].w);
     }
-    Out<T>::put(out + e, acc * inv);
   }
-  if (lse_out != nullptr && threadIdx.x == 0) lse_out[(long)b * n_h + h] = mx + logf(z);
+  typename Pack<T>::T2* dst = reinterpret_cast<typename Pack<T>::T2*>(out);
+#pragma unroll
+  for (int j = 0; j < 4; ++j) {
+    const int e = 4 * (lane + 32 * j);
+    dst[e / 2] = Pack<T>::make(acc[j].x * inv, acc[j].y * inv);
+    dst[e / 2 + 1] = Pack<T>::make(acc[j].z * inv, acc[j].w * inv);
+  }
+  if (lse_out != nullptr && lane == 0) lse_out[(long)b * n_h + h] = mx + logf(z);
 }
 
 }  // namespace tc

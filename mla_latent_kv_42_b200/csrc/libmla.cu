@@ -200,8 +200,8 @@ int decode_tc_impl(const mla_dims* d, const void* q, const void* pool, int32_t n
   p.o_part = o_part;
   p.lse_part = lse_part;
   tc::k_decode_tc<T><<<2 * C, tc::dec::kThreads, tc::dec::kSmem, st>>>(map, p);
-  tc::k_decode_tc_merge<T><<<dim3(B, d->n_heads), 128, 0, st>>>(o_part, lse_part, prefix, B, C, d->n_heads,
-                                                               static_cast<T*>(o_lat), lse_out);
+  tc::k_decode_tc_merge<T><<<dim3(B, (d->n_heads + 7) / 8), 256, 0, st>>>(o_part, lse_part, prefix, B, C, d->n_heads,
+                                                                          static_cast<T*>(o_lat), lse_out);
   return finish_launches(MLA_CALL_DECODE_ATTENTION, 3);
 }
 
