@@ -7,6 +7,8 @@
 #include <cuda_runtime.h>
 #include <stdint.h>
 
+#include <utility>
+
 #include "mla.h"
 
 namespace mla {
@@ -16,6 +18,15 @@ namespace mla {
 __device__ int g_status;
 
 __device__ __forceinline__ void record_error(int code) { atomicCAS(&g_status, 0, code); }
+
+// Programmatic dependent launch. The library's kernels are launched so that the next one may
+// start while this one finishes: each kernel lets its dependents launch once it is resident
+// (griddep_launch), and every thread waits for the kernels before it to complete, with their
+// memory visible, before it touches any memory they may write (griddep_wait). Each CTA passes
+// a griddep_wait before it exits, so completion stays ordered from kernel to kernel. Without
+// the launch attribute both are no-ops.
+__device__ __forceinline__ void griddep_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void griddep_launch() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
 
 template <typename T> struct Pack;
 template <> struct Pack<__nv_bfloat16> {
@@ -74,12 +85,35 @@ __device__ __forceinline__ float warp_max(float v) {
 // cos/sin of the RoPE angle of pair k at position pos: pos * base^(-2k/d_rope). The angle is
 // formed and reduced in double precision (an fp32 angle at position 131072 would be off by
 // up to ~1e-2 rad); only the final cos/sin are rounded to fp32.
-__device__ __forceinline__ void rope_cos_sin(int pos, int k, int d_rope, double base, float& c, float& s) {
-  const double theta = pow(base, -2.0 * (double)k / (double)d_rope);
+__device__ __forceinline__ double rope_inv_freq(int k, int d_rope, double base) {
+  return pow(base, -2.0 * (double)k / (double)d_rope);
+}
+__device__ __forceinline__ void rope_cos_sin_at(int pos, double inv_freq, float& c, float& s) {
   double sd, cd;
-  sincos((double)pos * theta, &sd, &cd);
+  sincos((double)pos * inv_freq, &sd, &cd);
   c = (float)cd;
   s = (float)sd;
+}
+__device__ __forceinline__ void rope_cos_sin(int pos, int k, int d_rope, double base, float& c, float& s) {
+  rope_cos_sin_at(pos, rope_inv_freq(k, d_rope, base), c, s);
+}
+
+// Launch `kern` on `st` with programmatic stream serialization: it may begin while the
+// previous kernel in the stream finishes (see griddep_wait / griddep_launch).
+template <typename... KArgs, typename... Args>
+inline cudaError_t launch_pdl(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t st,
+                              Args&&... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kern, std::forward<Args>(args)...);
 }
 
 }  // namespace mla

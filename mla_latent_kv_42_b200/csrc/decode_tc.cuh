@@ -33,11 +33,12 @@ constexpr int kPBufs = 2;         // P buffers in the value CTA
 constexpr int kPTile = 2 * 16384;  // P tile: 128 heads x 128 tokens bf16, two 64-token swizzled halves
 constexpr int kPBytes = kPTile + 512;  // + 128 rescale factors
 constexpr int kPStride = 33792;   // 1024-aligned stride of P buffers / staging buffers
-constexpr int kStageOff = kScoreSlots * kPair;   // score CTA: 2 staging buffers
+constexpr int kStg = 2;           // score CTA: P staging buffers
+constexpr int kStageOff = kScoreSlots * kPair;   // score CTA: kStg staging buffers
 constexpr int kPOff = kValSlots * 4 * kChunk;    // value CTA: kPBufs P buffers
 constexpr float kLazy = 8.f;      // rescale threshold in log2 units
 constexpr int kDataBytes = 204800;
-static_assert(kStageOff + 2 * kPStride <= kDataBytes, "score layout");
+static_assert(kStageOff + kStg * kPStride <= kDataBytes, "score layout");
 static_assert(kPOff + kPBufs * kPStride <= kDataBytes, "value layout");
 constexpr int kThreads = 224;     // 7 warps
 // TMEM columns
@@ -50,7 +51,7 @@ struct Ctrl {
   uint64_t full[kScoreSlots];
   uint64_t empty[kScoreSlots];
   uint64_t s_full, s_empty, q_ready;
-  uint64_t stg_ready[2], stg_free[2];  // score CTA: staging buffers (softmax warps <-> sender warp)
+  uint64_t stg_ready[kStg], stg_free[kStg];  // score CTA: staging buffers (softmax warps <-> sender warp)
   uint64_t p_empty[kPBufs];  // score CTA; arrived by the value CTA's multicast commit
   uint64_t stats_empty;      // score CTA; arrived remotely by the value CTA
   uint64_t p_full[kPBufs];   // value CTA; armed and completed by the score CTA's bulk copy
@@ -140,7 +141,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(dec::kThreads, 1)
     }
     mbar_init(bar(ctl->s_full), 1);
     mbar_init(bar(ctl->s_empty), 128);
-    for (int i = 0; i < 2; ++i) {
+    for (int i = 0; i < kStg; ++i) {
       mbar_init(bar(ctl->stg_ready[i]), 128);
       mbar_init(bar(ctl->stg_free[i]), 1);
     }
@@ -158,11 +159,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(dec::kThreads, 1)
     ctl->abort_flag = 0;
     fence_mbar_init();
   }
-  const bool has_work = [&] {
-    const long T_ = p.tile_prefix[p.B];
-    return T_ * (cluster + 1) / nclusters > T_ * cluster / nclusters;
-  }();
-  if (has_work && warp == 5) {
+  if (warp == 5) {
     tmem_alloc(smem_u32(&ctl->tmem_slot), kTmemCols);
     tmem_relinquish();
   }
@@ -172,6 +169,12 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(dec::kThreads, 1)
   cluster_wait();
   tc_fence_after();
   const uint32_t tmem = ctl->tmem_slot;
+  if (threadIdx.x == 0) griddep_launch();
+  griddep_wait();  // the plan, the query and the cache come from earlier kernels
+  const bool has_work = [&] {
+    const long T_ = p.tile_prefix[p.B];
+    return T_ * (cluster + 1) / nclusters > T_ * cluster / nclusters;
+  }();
   const uint32_t peer_abort = mapa(smem_u32(&ctl->abort_flag), peer);
   // A wait that gives up also releases the peer CTA's waiters.
   auto wait = [&](uint64_t& b, uint32_t parity) {
@@ -279,8 +282,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(dec::kThreads, 1)
           Item item;
           while (ok && next_item(it, p.tile_prefix, item)) {
             for (int t = item.t0; t < item.t1; t += 2, ++tile) {
-              const int sb = tile & 1, pb = tile % kPBufs;
-              if (!wait(ctl->stg_ready[sb], (tile >> 1) & 1) ||
+              const int sb = tile % kStg, pb = tile % kPBufs;
+              if (!wait(ctl->stg_ready[sb], (tile / kStg) & 1) ||
                   !wait_cl(ctl->p_empty[pb], ((tile / kPBufs) & 1) ^ 1)) {
                 ok = false;
                 break;
@@ -291,7 +294,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(dec::kThreads, 1)
                                 kPBytes, full_remote);
               bulk_commit_group();
               bulk_wait_read<1>();  // the previous tile's staging buffer has been read: hand it back
-              if (tile > 0) mbar_arrive(bar(ctl->stg_free[(tile - 1) & 1]));
+              if (tile > 0) mbar_arrive(bar(ctl->stg_free[(tile - 1) % kStg]));
             }
           }
           bulk_wait<0>();
@@ -370,8 +373,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(dec::kThreads, 1)
               l *= alpha;
               m_ref = mx;
             }
-            const int sb = tile & 1;
-            if (!wwait(ctl->stg_free[sb], ((tile >> 1) & 1) ^ 1)) {
+            const int sb = tile % kStg;
+            if (!wwait(ctl->stg_free[sb], ((tile / kStg) & 1) ^ 1)) {
               ok = false;
               break;
             }
@@ -598,7 +601,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(dec::kThreads, 1)
   }
   tc_fence_before();
   __syncthreads();
-  if (has_work && warp == 5) {
+  if (warp == 5) {
     tc_fence_after();
     tmem_dealloc(tmem, kTmemCols);
   }
@@ -612,6 +615,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(dec::kThreads, 1)
 __global__ void __launch_bounds__(1024) k_decode_plan(const int* __restrict__ seq_lens, const int* __restrict__ bt,
                                                       int B, int max_pages, int num_pages, int max_seq_len,
                                                       int* __restrict__ tile_prefix) {
+  griddep_wait();
+  if (threadIdx.x == 0) griddep_launch();
   __shared__ int part[1024];
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   for (int b = warp; b < B; b += 32) {
@@ -662,6 +667,8 @@ __global__ void __launch_bounds__(256) k_decode_tc_merge(const float* __restrict
                                                           const float* __restrict__ lse_part,
                                                           const int* __restrict__ tile_prefix, int B, int C, int n_h,
                                                           T* __restrict__ o_lat, float* __restrict__ lse_out) {
+  griddep_wait();
+  if (threadIdx.x == 0) griddep_launch();
   const int b = blockIdx.x, warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int h = blockIdx.y * 8 + warp;
   if (h >= n_h) return;

@@ -1,0 +1,460 @@
+// Persistent stream-K GEMM on tcgen05 for the projections, with the projection epilogues fused:
+//   D[z][m][n] = sum_k A[z][m][k] * B[z][n][k]
+// The weights are the M = 128 side of the MMA and the few tokens of a decode step the N side
+// ("swap-AB"), so every launch is a stream of weight bytes: what matters is that all SMs pull
+// from HBM without a tail. The iteration space (tile, 64-wide k block), tiles ordered
+// (z, m tile, n tile), is cut into G contiguous ranges, one per CTA: either evenly by
+// iteration (stream-K, for long tiles) or at tile boundaries (for short ones). A CTA walks its
+// range as segments, one per tile it touches; the MMA warp accumulates a segment in one of two
+// TMEM buffers while the four epilogue warps drain the other.
+//
+// A segment that covers a whole tile is finished in the CTA: the epilogue applies the
+// projection's output step and stores. A partial segment is written as fp32 to slot
+// (tile + cta) of the partial buffer — unique, because both the tile and the CTA index only
+// grow along the iteration space — and k_sk_reduce sums a tile's slots in CTA order (a fixed
+// order, so results repeat bit for bit) before applying the same output step.
+//
+// Output steps (EpiParams::mode):
+//   plain   out[z * batch_off + n * ld + m]
+//   append  the DeepSeek-V2 KV row [c^KV ; k^R] of token n: rows at and past rope_lo get RoPE
+//           (adjacent pairs, angle at pos[n]) and the row goes to its paged-cache slot
+//           (block_table[seq_idx[n]][pos[n] / page_size], row pos[n] % page_size)
+//   query   [q^C ; q^R-before-RoPE] of token n: rows below rope_lo are q^C -> qc[n][m];
+//           rope rows (head i, element j) get RoPE and go to q_out[n][i][d_c + j]
+// ("DeepSeek-V2 from Scratch" §4.2 for the compressed KV and decoupled RoPE key, §5.3 for the
+// absorbed query.)
+//
+// Warp roles (192 threads): 0-3 epilogue (thread = TMEM lane = row m), 4 TMA producer,
+// 5 TMEM allocation + MMA issue (one elected lane).
+#pragma once
+
+#include "tc_common.cuh"
+
+namespace mla {
+namespace tc {
+
+enum EpiMode : int { kEpiPlain = 0, kEpiAppend = 1, kEpiQuery = 2 };
+
+struct EpiParams {
+  int mode;
+  void* out;            // plain: element type; append: the cache pool; query: q_out
+  long out_ld, out_batch_off;
+  // RoPE (append, query): rows m >= rope_lo rotate in pairs (m, m ^ 1)
+  int rope_lo, d_rope;
+  double rope_base;
+  const int* pos;       // [N]
+  float2* cs_glob;      // [N][d_rope/2] cos/sin, written by CTA 0 for the reduction (or null)
+  // append
+  const int* seq_idx;   // [N]
+  const int* bt;
+  int num_seqs, max_pages, num_pages, page_size;
+  // query
+  void* qc;             // [N][rope_lo] element type
+  int n_h, d_c;
+};
+
+struct SkParams {
+  int M, N, K;
+  int m_tiles, n_tiles;
+  int kb;               // 64-wide k blocks per tile
+  long iters;           // tiles * kb
+  int aligned;          // 1: CTA ranges start at tile boundaries
+  int tiles;
+  int stages;
+  int a_batch_off;      // per z: row offset (K-major A) or K-row offset (MN-major A)
+  int b_batch_off;      // per z: K (column) offset into B's rows
+  float* part;          // [tiles + G][BN][128] fp32 partial slots
+  EpiParams epi;
+};
+
+// First iteration of CTA c out of G.
+__device__ __forceinline__ long sk_start(const SkParams& p, int c, int G) {
+  if (p.aligned) return ((long)p.tiles * c / G) * p.kb;
+  return p.iters * c / G;
+}
+// CTA whose range holds iteration i (inverse of sk_start).
+__device__ __forceinline__ int sk_owner(const SkParams& p, long i, int G) {
+  if (p.aligned) {
+    const long t = i / p.kb;
+    return (int)(((t + 1) * G - 1) / p.tiles);
+  }
+  return (int)(((i + 1) * G - 1) / p.iters);
+}
+
+template <int BN>
+struct SkCfg {
+  static constexpr int BM = 128, BK = 64;
+  static constexpr uint32_t A_BYTES = BM * BK * 2;
+  static constexpr uint32_t B_BYTES = BN * BK * 2;
+  static constexpr uint32_t STAGE_BYTES = A_BYTES + B_BYTES;
+  static constexpr uint32_t TMEM_COLS = 2 * BN;  // two accumulator buffers
+  static constexpr int MAX_STAGES = 12;
+};
+
+// Host and device: bytes of the RoPE table kept in shared memory (float2 per token and pair).
+__host__ __device__ inline size_t sk_table_bytes(int BN, const EpiParams& e) {
+  return e.mode == kEpiPlain ? 0 : (size_t)BN * (e.d_rope / 2) * 8 + (size_t)BN * 8;
+}
+
+// Where row m of the output goes, for one tile: element (m, n) is stored at
+// base + n * stride (plain, query) or at the token's cache row + m (append, see row_off).
+// The per-row part is computed once per tile so that the store loop stays short: the
+// epilogue runs once per tile, and its instructions are fetched cold each time.
+template <typename T, int MODE>
+struct RowDest {
+  T* base;
+  long stride;
+  __device__ __forceinline__ RowDest(const EpiParams& e, int z, int m) {
+    if (MODE == kEpiPlain) {
+      base = static_cast<T*>(e.out) + (long)z * e.out_batch_off + m;
+      stride = e.out_ld;
+    } else if (MODE == kEpiAppend) {
+      base = static_cast<T*>(e.out) + m;
+      stride = 0;
+    } else if (m < e.rope_lo) {
+      base = static_cast<T*>(e.qc) + m;
+      stride = e.rope_lo;
+    } else {
+      const int r = m - e.rope_lo;
+      base = static_cast<T*>(e.out) + (long)(r / e.d_rope) * (e.d_c + e.d_rope) + e.d_c + r % e.d_rope;
+      stride = (long)e.n_h * (e.d_c + e.d_rope);
+    }
+  }
+  // row_off: the token's cache row offset (append; negative = no valid slot, nothing stored)
+  __device__ __forceinline__ void put(int n, float v, long row_off) const {
+    if (MODE == kEpiAppend) {
+      if (row_off >= 0) Out<T>::put(base + row_off, v);
+    } else {
+      Out<T>::put(base + (long)n * stride, v);
+    }
+  }
+};
+
+// Cache row offset (elements) of token n for the append step, or -1 (error recorded).
+__device__ __forceinline__ long append_row_base(const EpiParams& e, int n) {
+  const int s = e.seq_idx[n], p = e.pos[n];
+  const int lp = p >= 0 ? p / e.page_size : -1;
+  int page = -1;
+  if (s >= 0 && s < e.num_seqs && p >= 0 && lp < e.max_pages) page = e.bt[(long)s * e.max_pages + lp];
+  if (page < 0 || page >= e.num_pages) return -1;
+  return ((long)page * e.page_size + p % e.page_size) * (e.rope_lo + e.d_rope);
+}
+
+template <typename T, int BN, bool A_MN, int MODE>
+__global__ void __launch_bounds__(192, 1)
+    k_gemm_sk(const __grid_constant__ CUtensorMap tma_a, const __grid_constant__ CUtensorMap tma_b,
+              const SkParams p) {
+  using C = SkCfg<BN>;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  const int S = p.stages;
+  const int half_rope = p.epi.d_rope / 2;
+  float2* cs_tab = reinterpret_cast<float2*>(smem + (size_t)S * C::STAGE_BYTES);        // [BN][d_rope/2]
+  long* row_tab = reinterpret_cast<long*>(cs_tab + (p.epi.mode == kEpiPlain ? 0 : BN * half_rope));  // [BN]
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + (size_t)S * C::STAGE_BYTES + sk_table_bytes(BN, p.epi));
+  uint64_t* full = bars;
+  uint64_t* empty = bars + S;
+  uint64_t* acc_full = bars + 2 * S;
+  uint64_t* acc_empty = bars + 2 * S + 2;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 2 * S + 4);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int cta = blockIdx.x, G = gridDim.x;
+  const long i0 = sk_start(p, cta, G), i1 = sk_start(p, cta + 1, G);
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < S; ++s) {
+      mbar_init(smem_u32(full + s), 1);
+      mbar_init(smem_u32(empty + s), 1);
+    }
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(smem_u32(acc_full + b), 1);
+      mbar_init(smem_u32(acc_empty + b), 128);
+    }
+    *abort_flag = 0;
+    fence_mbar_init();
+  }
+  if (warp == 5) {
+    tmem_alloc(smem_u32(tmem_slot), C::TMEM_COLS);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+  if (threadIdx.x == 0) griddep_launch();
+
+  auto tile_coords = [&](int tile, int& z, int& mt, int& nt) {
+    nt = tile % p.n_tiles;
+    mt = (tile / p.n_tiles) % p.m_tiles;
+    z = tile / (p.n_tiles * p.m_tiles);
+  };
+
+  if (warp == 4) {  // ------------------------------------------------ TMA producer
+    if (lane == 0) {
+      tma_prefetch_map(&tma_a);
+      tma_prefetch_map(&tma_b);
+      // Counters advance incrementally: this single thread paces the whole CTA, so the loop
+      // carries no divisions. The weights are written by no kernel, so the first ring stages
+      // start streaming them before the wait for the previous kernel; the activations (B)
+      // are loaded after it.
+      const int n_it = (int)(i1 - i0);
+      auto load_a = [&](int s, int z, int mt, int kbi) {
+        uint8_t* sa = smem + (size_t)s * C::STAGE_BYTES;
+        const uint32_t fb = smem_u32(full + s);
+        const int k = kbi * C::BK;
+        if (A_MN) {
+          tma_load_2d(smem_u32(sa), &tma_a, fb, mt * C::BM, k + z * p.a_batch_off);
+          tma_load_2d(smem_u32(sa + 8192), &tma_a, fb, mt * C::BM + 64, k + z * p.a_batch_off);
+        } else {
+          tma_load_2d(smem_u32(sa), &tma_a, fb, k, mt * C::BM + z * p.a_batch_off);
+        }
+      };
+      auto load_b = [&](int s, int z, int nt, int kbi) {
+        tma_load_2d(smem_u32(smem + (size_t)s * C::STAGE_BYTES + C::A_BYTES), &tma_b, smem_u32(full + s),
+                    kbi * C::BK + z * p.b_batch_off, nt * BN);
+      };
+      const int pre = min(S, n_it);
+      for (int j = 0; j < pre; ++j) {  // ring slots start empty: no wait
+        const long i = i0 + j;
+        int z, mt, nt;
+        tile_coords((int)(i / p.kb), z, mt, nt);
+        mbar_arrive_expect_tx(smem_u32(full + j), C::STAGE_BYTES);
+        load_a(j, z, mt, (int)(i % p.kb));
+      }
+      griddep_wait();
+      for (int j = 0; j < pre; ++j) {
+        const long i = i0 + j;
+        int z, mt, nt;
+        tile_coords((int)(i / p.kb), z, mt, nt);
+        load_b(j, z, nt, (int)(i % p.kb));
+      }
+      int z, mt, nt, kbi = (int)((i0 + pre) % p.kb);
+      tile_coords((int)((i0 + pre) / p.kb), z, mt, nt);
+      int s = pre % S, it = pre;
+      uint32_t ph = pre == S ? 1u : 0u;
+      for (; it < n_it; ++it) {
+        if (!mbar_wait(smem_u32(empty + s), ph ^ 1, abort_flag)) break;
+        mbar_arrive_expect_tx(smem_u32(full + s), C::STAGE_BYTES);
+        load_a(s, z, mt, kbi);
+        load_b(s, z, nt, kbi);
+        if (++s == S) {
+          s = 0;
+          ph ^= 1;
+        }
+        if (++kbi == p.kb) {
+          kbi = 0;
+          if (++nt == p.n_tiles) {
+            nt = 0;
+            if (++mt == p.m_tiles) {
+              mt = 0;
+              ++z;
+            }
+          }
+        }
+      }
+      if (*abort_flag) {  // copies still in flight land before the CTA exits
+        for (int j = max(0, it - S); j < it; ++j) mbar_wait_slow<false>(smem_u32(full + j % S), (j / S) & 1, nullptr);
+      }
+    }
+    __syncwarp();
+  } else if (warp == 5) {  // ----------------------------------------- MMA issue
+    if (lane == 0) {
+      const uint32_t idesc = idesc_f16(C::BM, BN, IsBf16<T>::value, A_MN, false);
+      const int n_it = (int)(i1 - i0);
+      int kbi = (int)(i0 % p.kb), seg = 0, s = 0;
+      uint32_t ph = 0, acc_col = 0;
+      bool first = true;
+      for (int it = 0; it < n_it; ++it) {
+        if (it == 0 || kbi == 0) {  // a new segment: wait until its accumulator buffer is drained
+          const int b = seg & 1;
+          if (!mbar_wait(smem_u32(acc_empty + b), ((seg >> 1) & 1) ^ 1, abort_flag)) break;
+          tc_fence_after();
+          acc_col = (uint32_t)(b * BN);
+          first = true;
+        }
+        if (!mbar_wait(smem_u32(full + s), ph, abort_flag)) break;
+        tc_fence_after();
+        const uint32_t sa = smem_u32(smem + (size_t)s * C::STAGE_BYTES), sb = sa + C::A_BYTES;
+#pragma unroll
+        for (int ks = 0; ks < 4; ++ks) {
+          const uint64_t ad = A_MN ? desc_sw128(sa + ks * 2048, 8192, 1024) : desc_sw128(sa + ks * 32, 16, 1024);
+          const uint64_t bd = desc_sw128(sb + ks * 32, 16, 1024);
+          mma_ss(tmem + acc_col, ad, bd, idesc, !(first && ks == 0));
+        }
+        mma_commit(smem_u32(empty + s));
+        first = false;
+        if (it == n_it - 1 || kbi == p.kb - 1) {
+          mma_commit(smem_u32(acc_full + (seg & 1)));
+          ++seg;
+        }
+        if (++s == S) {
+          s = 0;
+          ph ^= 1;
+        }
+        if (++kbi == p.kb) kbi = 0;
+      }
+    }
+    __syncwarp();
+  } else {  // ---------------------------------------------------------- epilogue warps 0-3
+    const int ml = warp * 32 + lane;  // row within the tile = TMEM lane
+    const uint32_t lane_base = (uint32_t)(warp * 32) << 16;
+    // Tables of the fused output step for the one n tile (RoPE cos/sin per token and pair,
+    // cache row offset per token), built once while the first tiles stream in. With several
+    // n tiles the step computes them per element instead.
+    const bool use_tab = MODE != kEpiPlain && p.n_tiles == 1;
+    griddep_wait();  // token positions, cache slots and outputs belong to earlier kernels
+    if (use_tab) {
+      double theta = 0.0;
+      int theta_k = -1;
+      for (int e = ml; e < BN * half_rope; e += 128) {
+        const int n = e / half_rope, k = e % half_rope;
+        if (k != theta_k) {  // with half_rope dividing 128 this runs once per thread
+          theta = rope_inv_freq(k, p.epi.d_rope, p.epi.rope_base);
+          theta_k = k;
+        }
+        float c = 1.f, sn = 0.f;
+        if (n < p.N) rope_cos_sin_at(p.epi.pos[n], theta, c, sn);
+        cs_tab[e] = make_float2(c, sn);
+        if (cta == 0 && p.epi.cs_glob != nullptr && n < p.N) p.epi.cs_glob[e] = make_float2(c, sn);
+      }
+      if (MODE == kEpiAppend)
+        for (int e = ml; e < BN; e += 128) {
+          long rb = -1;
+          if (e < p.N) {
+            rb = append_row_base(p.epi, e);
+            if (rb < 0 && cta == 0) record_error(MLA_ERR_BAD_PAGE);
+          }
+          row_tab[e] = rb;
+        }
+      named_bar_sync(1, 128);
+    }
+    int seg = 0;
+    long i = i0;
+    while (i < i1) {
+      const int tile = (int)(i / p.kb), kbi0 = (int)(i % p.kb);
+      const long seg_end = min(i1, (long)(tile + 1) * p.kb);
+      const bool whole = kbi0 == 0 && seg_end == (long)(tile + 1) * p.kb;
+      int z, mt, nt;
+      tile_coords(tile, z, mt, nt);
+      const int m = mt * C::BM + ml;
+      const int n0 = nt * BN;
+      const bool rot = MODE != kEpiPlain && m >= p.epi.rope_lo;
+      const bool rope_warp = __any_sync(0xffffffffu, rot);
+      const int k = rot ? ((m - p.epi.rope_lo) % p.epi.d_rope) >> 1 : 0;
+      const RowDest<T, MODE> dst(p.epi, z, m);
+      const bool row_ok = m < p.M;
+      const int nv = min(BN, p.N - n0);  // valid columns of this tile
+      const int b = seg & 1;
+      if (!__all_sync(0xffffffffu, mbar_wait(smem_u32(acc_full + b), (seg >> 1) & 1, abort_flag))) break;
+      tc_fence_after();
+      const uint32_t acc = tmem + lane_base + (uint32_t)(b * BN);
+      float* slot = p.part + ((long)tile + cta) * (128L * BN) + ml;
+#pragma unroll 1
+      for (int c0 = 0; c0 < BN; c0 += 8) {
+        uint32_t r[8];
+        tmem_ld8(acc + c0, r);
+        tmem_wait_ld();
+        if (!whole) {
+#pragma unroll
+          for (int j = 0; j < 8; ++j)
+            if (c0 + j < nv) slot[(long)(c0 + j) * 128] = u2f(r[j]);
+          continue;
+        }
+#pragma unroll
+        for (int j = 0; j < 8; ++j) {
+          float v = u2f(r[j]);
+          const int nl = c0 + j;
+          if (MODE != kEpiPlain && rope_warp) {  // warp-uniform: every lane takes part in the exchange
+            const float w = __shfl_xor_sync(0xffffffffu, v, 1);  // the pair partner's value
+            if (rot && nl < nv) {
+              float2 q;
+              if (use_tab) q = cs_tab[nl * half_rope + k];
+              else rope_cos_sin(p.epi.pos[n0 + nl], k, p.epi.d_rope, p.epi.rope_base, q.x, q.y);
+              v = (m & 1) ? fmaf(w, q.y, v * q.x) : fmaf(v, q.x, -w * q.y);
+            }
+          }
+          if (nl < nv && row_ok)
+            dst.put(n0 + nl, v, MODE != kEpiAppend ? 0 : use_tab ? row_tab[nl] : append_row_base(p.epi, n0 + nl));
+        }
+      }
+      tc_fence_before();
+      mbar_arrive(smem_u32(acc_empty + b));
+      ++seg;
+      i = seg_end;
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 5) {
+    tc_fence_after();
+    tmem_dealloc(tmem, C::TMEM_COLS);
+  }
+}
+
+// Tiles split over several CTAs: sum the fp32 partial slots in CTA order and apply the output
+// step. Block (tile, 8-column group); thread = row pair (2q, 2q+1) of one column.
+template <typename T, int BN, int MODE>
+__global__ void __launch_bounds__(256) k_sk_reduce(const SkParams p, int G) {
+  griddep_wait();
+  if (threadIdx.x == 0) griddep_launch();
+  const int tile = blockIdx.x;
+  const long t0 = (long)tile * p.kb;
+  const int c_lo = sk_owner(p, t0, G), c_hi = sk_owner(p, t0 + p.kb - 1, G);
+  if (c_lo == c_hi) return;  // finished whole by its CTA
+  const int nt = tile % p.n_tiles, mt = (tile / p.n_tiles) % p.m_tiles, z = tile / (p.n_tiles * p.m_tiles);
+  const int q = threadIdx.x & 63;
+  const int m = mt * 128 + 2 * q;
+#pragma unroll
+  for (int j = 0; j < 2; ++j) {
+    const int nl = blockIdx.y * 8 + (threadIdx.x >> 6) + 4 * j;
+    const int n = nt * BN + nl;
+    if (nl >= BN || n >= p.N || m >= p.M) continue;
+    const float* src = p.part + ((long)tile + c_lo) * (128L * BN) + (long)nl * 128 + 2 * q;
+    float a = 0.f, b = 0.f;
+    int c = c_lo;
+    for (; c + 3 <= c_hi; c += 4, src += 4 * 128L * BN) {  // loads in flight together, sums in CTA order
+      float2 v[4];
+#pragma unroll
+      for (int u = 0; u < 4; ++u) v[u] = *reinterpret_cast<const float2*>(src + u * 128L * BN);
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        a += v[u].x;
+        b += v[u].y;
+      }
+    }
+    for (; c <= c_hi; ++c, src += 128L * BN) {
+      const float2 v = *reinterpret_cast<const float2*>(src);
+      a += v.x;
+      b += v.y;
+    }
+    long rb = 0;
+    if (MODE == kEpiAppend) {
+      rb = append_row_base(p.epi, n);
+      if (rb < 0) {
+        record_error(MLA_ERR_BAD_PAGE);
+        continue;
+      }
+    }
+    if (MODE != kEpiPlain && m >= p.epi.rope_lo) {
+      const int k = ((m - p.epi.rope_lo) % p.epi.d_rope) >> 1;
+      float cs, sn;
+      if (p.epi.cs_glob != nullptr) {
+        const float2 t = p.epi.cs_glob[(long)n * (p.epi.d_rope / 2) + k];
+        cs = t.x;
+        sn = t.y;
+      } else {
+        rope_cos_sin(p.epi.pos[n], k, p.epi.d_rope, p.epi.rope_base, cs, sn);
+      }
+      const float ra = fmaf(a, cs, -b * sn), rb2 = fmaf(b, cs, a * sn);
+      a = ra;
+      b = rb2;
+    }
+    RowDest<T, MODE>(p.epi, z, m).put(n, a, rb);
+    if (m + 1 < p.M) RowDest<T, MODE>(p.epi, z, m + 1).put(n, b, rb);
+  }
+}
+
+}  // namespace tc
+}  // namespace mla

@@ -185,7 +185,9 @@ int decode_tc_impl(const mla_dims* d, const void* q, const void* pool, int32_t n
   if (!host::encode_2d(&map, pool, tc::IsBf16<T>::value, tc::dec::kD, (uint64_t)num_pages * tc::dec::kPage,
                        tc::dec::kD * 2, 64, 64))
     return MLA_ERR_CUDA;
-  tc::k_decode_plan<<<1, 1024, 0, st>>>(seq_lens, bt, B, max_pages, num_pages, max_seq_len, prefix);
+  if (launch_pdl(tc::k_decode_plan, dim3(1), dim3(1024), 0, st, seq_lens, bt, (int)B, (int)max_pages, (int)num_pages,
+                 (int)max_seq_len, prefix) != cudaSuccess)
+    return MLA_ERR_CUDA;
   tc::DecodeTcParams p;
   p.q = q;
   p.bt = bt;
@@ -199,9 +201,13 @@ int decode_tc_impl(const mla_dims* d, const void* q, const void* pool, int32_t n
   p.lse_out = lse_out;
   p.o_part = o_part;
   p.lse_part = lse_part;
-  tc::k_decode_tc<T><<<2 * C, tc::dec::kThreads, tc::dec::kSmem, st>>>(map, p);
-  tc::k_decode_tc_merge<T><<<dim3(B, (d->n_heads + 7) / 8), 256, 0, st>>>(o_part, lse_part, prefix, B, C, d->n_heads,
-                                                                          static_cast<T*>(o_lat), lse_out);
+  if (launch_pdl(tc::k_decode_tc<T>, dim3(2 * C), dim3(tc::dec::kThreads), tc::dec::kSmem, st, map, p) != cudaSuccess)
+    return MLA_ERR_CUDA;
+  if (launch_pdl(tc::k_decode_tc_merge<T>, dim3(B, (d->n_heads + 7) / 8), dim3(256), 0, st,
+                 static_cast<const float*>(o_part), static_cast<const float*>(lse_part),
+                 static_cast<const int*>(prefix), (int)B, C, (int)d->n_heads, static_cast<T*>(o_lat),
+                 lse_out) != cudaSuccess)
+    return MLA_ERR_CUDA;
   return finish_launches(MLA_CALL_DECODE_ATTENTION, 3);
 }
 

@@ -12,7 +12,7 @@
 #include <cstring>
 #include <mutex>
 
-#include "gemm_tc.cuh"
+#include "gemm_sk.cuh"
 #include "proj_simt.cuh"
 
 namespace mla {
@@ -84,21 +84,46 @@ inline bool encode_2d(CUtensorMap* map, const void* base, bool bf16, uint64_t in
 }
 
 // ------------------------------------------------------------------ GEMM planning
-struct GemmPlan {
-  int bn, n_tiles, m_tiles, splits, kbps;
+// One stream-K GEMM launch (see gemm_sk.cuh): tile sizes, CTA count, ring depth, and whether
+// any tile is shared by several CTAs (then fp32 partials and a reduction launch are needed).
+struct SkPlan {
+  int bn, m_tiles, n_tiles, batch, kb, tiles, G, stages;
+  long iters;
+  bool aligned, split;
+  size_t smem, part_bytes;
 };
 
-inline GemmPlan plan_gemm(int M, int N, int K, int batch, bool allow_split) {
-  GemmPlan g;
-  g.bn = N <= 16 ? 16 : N <= 32 ? 32 : N <= 64 ? 64 : N <= 128 ? 128 : 256;
+constexpr int kSkMinIters = 8;       // k blocks per CTA at least, when tiles are split
+constexpr int kSkLongTile = 16;      // tiles of at least this many k blocks are split (stream-K)
+constexpr size_t kSkSmemMax = 232448;
+
+inline SkPlan plan_sk(int M, int N, int K, int batch, bool fused_epi, int d_rope) {
+  SkPlan g;
+  g.bn = N <= 32 ? 32 : N <= 64 ? 64 : N <= 128 ? 128 : 256;
   g.n_tiles = (N + g.bn - 1) / g.bn;
   g.m_tiles = (M + 127) / 128;
-  const int kb = (K + 63) / 64;
-  const long base = (long)g.m_tiles * g.n_tiles * batch;
-  long s = 1;
-  if (allow_split && base < sm_count()) s = std::max(1L, std::min((long)sm_count() / base, (long)kb / 4));
-  g.kbps = (int)((kb + s - 1) / s);
-  g.splits = (kb + g.kbps - 1) / g.kbps;
+  g.batch = batch;
+  g.kb = (K + 63) / 64;
+  g.tiles = g.m_tiles * g.n_tiles * batch;
+  g.iters = (long)g.tiles * g.kb;
+  const int sms = sm_count();
+  if (g.kb >= kSkLongTile) {
+    g.aligned = false;
+    g.G = (int)std::max(1L, std::min((long)sms, g.iters / kSkMinIters));
+  } else {
+    g.aligned = true;
+    const int per = (g.tiles + sms - 1) / sms;
+    g.G = (g.tiles + per - 1) / per;
+  }
+  g.split = false;
+  if (!g.aligned)
+    for (int c = 1; c < g.G && !g.split; ++c) g.split = (g.iters * c / g.G) % g.kb != 0;
+  const size_t stage = (size_t)(128 + g.bn) * 64 * 2;
+  const size_t table = fused_epi ? (size_t)g.bn * (d_rope / 2) * 8 + (size_t)g.bn * 8 : 0;
+  const size_t fixed = 1024 + table + 256;
+  g.stages = (int)std::min<size_t>(12, (kSkSmemMax - fixed) / stage);
+  g.smem = fixed + (size_t)g.stages * stage;
+  g.part_bytes = g.split ? (size_t)(g.tiles + g.G) * 128 * g.bn * sizeof(float) : 0;
   return g;
 }
 
@@ -112,71 +137,91 @@ struct Operand {
   int batch_off;
 };
 
-template <typename T, int BN, bool MN>
-cudaError_t run_gemm(const CUtensorMap& ma, const CUtensorMap& mb, const tc::GemmParams& p, dim3 grid,
-                     cudaStream_t st) {
-  using C = tc::GemmCfg<BN>;
+template <typename T, int BN, bool MN, int MODE>
+cudaError_t run_sk(const CUtensorMap& ma, const CUtensorMap& mb, const tc::SkParams& p, const SkPlan& g,
+                   cudaStream_t st, int32_t& n) {
   static bool attr_done[kMaxDev] = {};
   int dev = 0;
   cudaGetDevice(&dev);
   if (dev >= 0 && dev < kMaxDev && !attr_done[dev]) {
-    cudaError_t e =
-        cudaFuncSetAttribute(tc::k_gemm_tc<T, BN, MN>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)C::SMEM);
+    cudaError_t e = cudaFuncSetAttribute(tc::k_gemm_sk<T, BN, MN, MODE>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         (int)kSkSmemMax);
     if (e != cudaSuccess) return e;
     attr_done[dev] = true;
   }
-  tc::k_gemm_tc<T, BN, MN><<<grid, 192, C::SMEM, st>>>(ma, mb, p);
+  cudaError_t e = launch_pdl(tc::k_gemm_sk<T, BN, MN, MODE>, dim3(g.G), dim3(192), g.smem, st, ma, mb, p);
+  if (e != cudaSuccess) return e;
+  ++n;
+  if (g.split) {
+    e = launch_pdl(tc::k_sk_reduce<T, BN, MODE>, dim3(g.tiles, BN / 8), dim3(256), 0, st, p, g.G);
+    if (e != cudaSuccess) return e;
+    ++n;
+  }
   return cudaGetLastError();
 }
 
-// out[z][n][m] (or fp32 partial [split][z][n][m]) = sum_k A[z][m][k] B[z][n][k].
+template <typename T, int BN>
+cudaError_t run_sk_mode(const CUtensorMap& ma, const CUtensorMap& mb, bool a_mn, const tc::SkParams& p,
+                        const SkPlan& g, cudaStream_t st, int32_t& n) {
+  switch (p.epi.mode) {
+    case tc::kEpiPlain:
+      return a_mn ? run_sk<T, BN, true, tc::kEpiPlain>(ma, mb, p, g, st, n)
+                  : run_sk<T, BN, false, tc::kEpiPlain>(ma, mb, p, g, st, n);
+    case tc::kEpiAppend:  // the fused steps read K-major weights
+      return a_mn ? cudaErrorInvalidValue : run_sk<T, BN, false, tc::kEpiAppend>(ma, mb, p, g, st, n);
+    case tc::kEpiQuery:
+      return a_mn ? cudaErrorInvalidValue : run_sk<T, BN, false, tc::kEpiQuery>(ma, mb, p, g, st, n);
+    default:
+      return cudaErrorInvalidValue;
+  }
+}
+
+// D[z][m][n] = sum_k A[z][m][k] B[z][n][k], finished by the output step `epi`; `part` holds
+// g.part_bytes of scratch when g.split.
 template <typename T>
-int gemm_tc(const Operand& A, bool a_mn, const Operand& B, int M, int N, int K, int batch, const GemmPlan& g,
-            void* out, bool out_f32, long out_ld, long out_batch_off, long out_split_off, cudaStream_t st) {
+int gemm_sk(const Operand& A, bool a_mn, const Operand& B, int M, int N, int K, const SkPlan& g,
+            const tc::EpiParams& epi, float* part, cudaStream_t st, int32_t& n) {
+  if (N <= 0 || M <= 0) return MLA_OK;
   constexpr bool bf16 = tc::IsBf16<T>::value;
   CUtensorMap ma, mb;
   const bool ok_a = a_mn ? encode_2d(&ma, A.base, bf16, A.cols, A.rows, A.cols * 2, 64, 64)
                          : encode_2d(&ma, A.base, bf16, A.cols, A.rows, A.cols * 2, 64, 128);
   const bool ok_b = encode_2d(&mb, B.base, bf16, B.cols, B.rows, B.cols * 2, 64, g.bn);
   if (!ok_a || !ok_b) return MLA_ERR_CUDA;
-  tc::GemmParams p;
+  tc::SkParams p;
   p.M = M;
   p.N = N;
   p.K = K;
-  p.kb_per_split = g.kbps;
+  p.m_tiles = g.m_tiles;
   p.n_tiles = g.n_tiles;
+  p.kb = g.kb;
+  p.iters = g.iters;
+  p.aligned = g.aligned ? 1 : 0;
+  p.tiles = g.tiles;
+  p.stages = g.stages;
   p.a_batch_off = A.batch_off;
   p.b_batch_off = B.batch_off;
-  p.out = out;
-  p.out_ld = out_ld;
-  p.out_batch_off = out_batch_off;
-  p.out_split_off = out_split_off;
-  p.out_f32 = out_f32 ? 1 : 0;
-  const dim3 grid(g.m_tiles, g.splits * g.n_tiles, batch);
+  p.part = part;
+  p.epi = epi;
   cudaError_t e;
-#define MLA_GEMM_CASE(BNV)                                                              \
-  case BNV:                                                                             \
-    e = a_mn ? run_gemm<T, BNV, true>(ma, mb, p, grid, st) : run_gemm<T, BNV, false>(ma, mb, p, grid, st); \
-    break;
   switch (g.bn) {
-    MLA_GEMM_CASE(16)
-    MLA_GEMM_CASE(32)
-    MLA_GEMM_CASE(64)
-    MLA_GEMM_CASE(128)
-    MLA_GEMM_CASE(256)
+    case 32: e = run_sk_mode<T, 32>(ma, mb, a_mn, p, g, st, n); break;
+    case 64: e = run_sk_mode<T, 64>(ma, mb, a_mn, p, g, st, n); break;
+    case 128: e = run_sk_mode<T, 128>(ma, mb, a_mn, p, g, st, n); break;
+    case 256: e = run_sk_mode<T, 256>(ma, mb, a_mn, p, g, st, n); break;
     default: return MLA_ERR_CUDA;
   }
-#undef MLA_GEMM_CASE
   return e == cudaSuccess ? MLA_OK : MLA_ERR_CUDA;
 }
 
-template <typename T>
-void launch_reduce(const float* part, int splits, long split_off, long rows, long row_len, long out_ld, T* out,
-                   cudaStream_t st) {
-  const long n = rows * row_len;
-  const int threads = 256;
-  const long blocks = std::min((n + threads - 1) / threads, 4L * sm_count());
-  tc::k_splitk_reduce<T><<<(unsigned)blocks, threads, 0, st>>>(part, splits, split_off, n, rows, row_len, out_ld, out);
+inline tc::EpiParams epi_plain(void* out, long ld, long batch_off) {
+  tc::EpiParams e{};
+  e.mode = tc::kEpiPlain;
+  e.out = out;
+  e.out_ld = ld;
+  e.out_batch_off = batch_off;
+  e.d_rope = 2;
+  return e;
 }
 
 template <typename T, typename OutT>
@@ -193,17 +238,20 @@ void launch_rowdot(const T* W, const T* X, OutT* Y, int M, int K, int Tn, long l
 
 // ------------------------------------------------------------------ mla_append_kv
 struct AppendLayout {
-  GemmPlan g;
-  float* Y;
+  SkPlan g;
+  float* Y;     // CUDA-core route: fp32 [T, D]
+  float* part;  // tensor-core route: stream-K partials
+  float2* cs;   // RoPE cos/sin per token for the reduction of split tiles
   size_t bytes;
 };
 inline AppendLayout append_layout(const mla_dims* d, int T_, void* ws) {
   AppendLayout L;
   const int D = d->d_c + d->d_rope;
-  L.g = plan_gemm(D, T_, d->d_model, 1, true);
-  const int splits = proj_uses_simt() ? 1 : L.g.splits;
+  L.g = plan_sk(D, T_, d->d_model, 1, true, d->d_rope);
   Carver c{static_cast<char*>(ws)};
-  L.Y = c.take<float>((size_t)splits * T_ * D);
+  L.Y = proj_uses_simt() ? c.take<float>((size_t)T_ * D) : nullptr;
+  L.part = (!proj_uses_simt() && L.g.split) ? c.take<float>(L.g.part_bytes / sizeof(float)) : nullptr;
+  L.cs = (!proj_uses_simt() && L.g.split && L.g.n_tiles == 1) ? c.take<float2>((size_t)T_ * (d->d_rope / 2)) : nullptr;
   L.bytes = c.off;
   return L;
 }
@@ -214,47 +262,61 @@ int append_run(const mla_dims* d, const void* h, const void* w, const int32_t* s
                void* ws, cudaStream_t st, int32_t& n) {
   const int D = d->d_c + d->d_rope;
   const AppendLayout L = append_layout(d, T_, ws);
-  int splits = 1;
   if (proj_uses_simt()) {
     launch_rowdot<T, float>(static_cast<const T*>(w), static_cast<const T*>(h), L.Y, D, d->d_model, T_, d->d_model,
                             D, 1, 0, 0, 0, st, n);
-  } else {
-    const int r = gemm_tc<T>({w, D, d->d_model, 0}, false, {h, T_, d->d_model, 0}, D, T_, d->d_model, 1, L.g, L.Y,
-                             true, D, 0, (long)T_ * D, st);
-    if (r != MLA_OK) return r;
+    k_append_epilogue<T><<<T_, 128, (d->d_rope / 2) * sizeof(float2), st>>>(
+        L.Y, 1, (long)T_ * D, seq_idx, pos, bt, num_seqs, max_pages, static_cast<T*>(pool), num_pages,
+        d->page_size, d->d_c, d->d_rope, d->rope_base);
     ++n;
-    splits = L.g.splits;
+    return MLA_OK;
   }
-  k_append_epilogue<T><<<T_, 128, (d->d_rope / 2) * sizeof(float2), st>>>(L.Y, splits, (long)T_ * D, seq_idx, pos, bt, num_seqs, max_pages,
-                                          static_cast<T*>(pool), num_pages, d->page_size, d->d_c, d->d_rope,
-                                          d->rope_base);
-  ++n;
-  return MLA_OK;
+  // [c^KV ; k^R] = W^{DKV,KR} h, RoPE on k^R, written to each token's cache slot
+  tc::EpiParams e{};
+  e.mode = tc::kEpiAppend;
+  e.out = pool;
+  e.rope_lo = d->d_c;
+  e.d_rope = d->d_rope;
+  e.rope_base = d->rope_base;
+  e.pos = pos;
+  e.seq_idx = seq_idx;
+  e.bt = bt;
+  e.num_seqs = num_seqs;
+  e.max_pages = max_pages;
+  e.num_pages = num_pages;
+  e.page_size = d->page_size;
+  e.d_c = d->d_c;
+  e.cs_glob = L.cs;
+  return gemm_sk<T>({w, D, d->d_model, 0}, false, {h, T_, d->d_model, 0}, D, T_, d->d_model, L.g, e, L.part, st, n);
 }
 
 // ------------------------------------------------------------------ mla_absorb_query
 struct AbsorbLayout {
-  GemmPlan g1, g2, g3;
-  float* P1;   // split partials of c^Q (fp32), when g1.splits > 1
-  void* cq;    // c^Q, element type [B, d_cq]
-  float* Y2;   // [q^C ; q^] partials, fp32 [g2.splits][B][nq]
-  void* qc;    // q^C, element type [B, n_h*d_h]
+  SkPlan g1, g2, g3;
+  void* cq;     // c^Q, element type [B, d_cq]
+  void* qc;     // q^C, element type [B, n_h*d_h]
+  float* Y2;    // CUDA-core route: [q^C ; q^R before RoPE] fp32 [B, nq]
+  float* part;  // stream-K partials, shared by the three products (they run one after another)
+  float2* cs;   // RoPE cos/sin per token for the reduction of split query tiles
   size_t bytes;
-  bool tc_uk;  // the per-head (W^UK_i)^T product runs on the tensor-core GEMM
+  bool tc_uk;   // the per-head (W^UK_i)^T product runs on the tensor-core GEMM
 };
 inline AbsorbLayout absorb_layout(const mla_dims* d, int B, void* ws) {
   AbsorbLayout L;
   const int nq = d->n_heads * (d->d_head + d->d_rope);
   const bool simt = proj_uses_simt();
-  L.g1 = plan_gemm(d->d_cq, B, d->d_model, 1, true);
-  L.g2 = plan_gemm(nq, B, d->d_cq, 1, true);
-  L.g3 = plan_gemm(d->d_c, B, d->d_head, d->n_heads, false);
+  L.g1 = plan_sk(d->d_cq, B, d->d_model, 1, false, d->d_rope);
+  L.g2 = plan_sk(nq, B, d->d_cq, 1, true, d->d_rope);
+  L.g3 = plan_sk(d->d_c, B, d->d_head, d->n_heads, false, d->d_rope);
   L.tc_uk = !simt && d->d_head % 64 == 0;
   Carver c{static_cast<char*>(ws)};
-  L.P1 = (!simt && L.g1.splits > 1) ? c.take<float>((size_t)L.g1.splits * B * d->d_cq) : nullptr;
   L.cq = c.take<uint16_t>((size_t)B * d->d_cq);
-  L.Y2 = c.take<float>((size_t)(simt ? 1 : L.g2.splits) * B * nq);
   L.qc = c.take<uint16_t>((size_t)B * d->n_heads * d->d_head);
+  L.Y2 = simt ? c.take<float>((size_t)B * nq) : nullptr;
+  size_t part = 0;
+  if (!simt) part = std::max(L.g1.part_bytes, std::max(L.g2.part_bytes, L.tc_uk ? L.g3.part_bytes : 0));
+  L.part = part ? c.take<float>(part / sizeof(float)) : nullptr;
+  L.cs = (!simt && L.g2.split && L.g2.n_tiles == 1) ? c.take<float2>((size_t)B * (d->d_rope / 2)) : nullptr;
   L.bytes = c.off;
   return L;
 }
@@ -268,56 +330,54 @@ int absorb_run(const mla_dims* d, const void* h, const void* w_dq, const void* w
   const AbsorbLayout L = absorb_layout(d, B, ws);
   T* cq = static_cast<T*>(L.cq);
   T* qc = static_cast<T*>(L.qc);
-  int splits2 = 1;
   if (proj_uses_simt()) {
     launch_rowdot<T, T>(static_cast<const T*>(w_dq), static_cast<const T*>(h), cq, d->d_cq, d->d_model, B,
                         d->d_model, d->d_cq, 1, 0, 0, 0, st, n);
     launch_rowdot<T, float>(static_cast<const T*>(w_uq_qr), cq, L.Y2, nq, d->d_cq, B, d->d_cq, nq, 1, 0, 0, 0, st, n);
+    k_query_epilogue<T><<<B, 256, (d->d_rope / 2) * sizeof(float2), st>>>(
+        L.Y2, 1, (long)B * nq, pos, qc, static_cast<T*>(q_out), d->n_heads, d->d_head, d->d_rope, d->d_c,
+        d->rope_base);
+    ++n;
   } else {
     // c^Q = W^DQ h
-    int r;
-    if (L.g1.splits > 1) {
-      r = gemm_tc<T>({w_dq, d->d_cq, d->d_model, 0}, false, {h, B, d->d_model, 0}, d->d_cq, B, d->d_model, 1, L.g1,
-                     L.P1, true, d->d_cq, 0, (long)B * d->d_cq, st);
-      if (r != MLA_OK) return r;
-      launch_reduce<T>(L.P1, L.g1.splits, (long)B * d->d_cq, B, d->d_cq, d->d_cq, cq, st);
-      n += 2;
-    } else {
-      r = gemm_tc<T>({w_dq, d->d_cq, d->d_model, 0}, false, {h, B, d->d_model, 0}, d->d_cq, B, d->d_model, 1, L.g1,
-                     cq, false, d->d_cq, 0, 0, st);
-      if (r != MLA_OK) return r;
-      ++n;
-    }
-    // [q^C ; q^] = [W^UQ ; W^QR] c^Q
-    r = gemm_tc<T>({w_uq_qr, nq, d->d_cq, 0}, false, {cq, B, d->d_cq, 0}, nq, B, d->d_cq, 1, L.g2, L.Y2, true, nq, 0,
-                   (long)B * nq, st);
+    int r = gemm_sk<T>({w_dq, d->d_cq, d->d_model, 0}, false, {h, B, d->d_model, 0}, d->d_cq, B, d->d_model, L.g1,
+                       epi_plain(cq, d->d_cq, 0), L.part, st, n);
     if (r != MLA_OK) return r;
-    ++n;
-    splits2 = L.g2.splits;
+    // [q^C ; q^] = [W^UQ ; W^QR] c^Q; q^C -> qc, q^R_i = RoPE(q^_i) -> q_out[b][i][d_c:]
+    tc::EpiParams e{};
+    e.mode = tc::kEpiQuery;
+    e.out = q_out;
+    e.rope_lo = nhd;
+    e.d_rope = d->d_rope;
+    e.rope_base = d->rope_base;
+    e.pos = pos;
+    e.qc = qc;
+    e.n_h = d->n_heads;
+    e.d_c = d->d_c;
+    e.cs_glob = L.cs;
+    r = gemm_sk<T>({w_uq_qr, nq, d->d_cq, 0}, false, {cq, B, d->d_cq, 0}, nq, B, d->d_cq, L.g2, e, L.part, st, n);
+    if (r != MLA_OK) return r;
   }
-  k_query_epilogue<T><<<B, 256, (d->d_rope / 2) * sizeof(float2), st>>>(L.Y2, splits2, (long)B * nq, pos, qc, static_cast<T*>(q_out), d->n_heads,
-                                         d->d_head, d->d_rope, d->d_c, d->rope_base);
-  ++n;
-  // q~_i = (W^UK_i)^T q^C_i
+  // q~_i = (W^UK_i)^T q^C_i -> q_out[b][i][:d_c]
   if (L.tc_uk) {
-    const int r = gemm_tc<T>({w_uk, nhd, d->d_c, d->d_head}, true, {qc, B, nhd, d->d_head}, d->d_c, B, d->d_head,
-                             d->n_heads, L.g3, q_out, false, (long)d->n_heads * D, D, 0, st);
+    const int r = gemm_sk<T>({w_uk, nhd, d->d_c, d->d_head}, true, {qc, B, nhd, d->d_head}, d->d_c, B, d->d_head,
+                             L.g3, epi_plain(q_out, (long)d->n_heads * D, D), L.part, st, n);
     if (r != MLA_OK) return r;
   } else {
     const int threads = 128;
     dim3 grid((d->d_c / 2 + threads - 1) / threads, d->n_heads);
     k_absorb_uk<T, 16><<<grid, threads, 16 * d->d_head * sizeof(float), st>>>(
         static_cast<const T*>(w_uk), qc, static_cast<T*>(q_out), B, d->n_heads, d->d_head, d->d_c, D);
+    ++n;
   }
-  ++n;
   return MLA_OK;
 }
 
 // ------------------------------------------------------------------ mla_out_proj
 struct OutLayout {
-  GemmPlan g_o, g_u;
-  void* o;    // element type [B, n_h*d_h]
-  float* P;   // split partials of u (fp32), when g_u.splits > 1
+  SkPlan g_o, g_u;
+  void* o;      // element type [B, n_h*d_h]
+  float* part;  // stream-K partials, shared by the two products
   size_t bytes;
   bool tc_o;
 };
@@ -325,12 +385,14 @@ inline OutLayout out_layout(const mla_dims* d, int B, void* ws) {
   OutLayout L;
   const int nhd = d->n_heads * d->d_head;
   const bool simt = proj_uses_simt();
-  L.g_o = plan_gemm(d->d_head, B, d->d_c, d->n_heads, false);
-  L.g_u = plan_gemm(d->d_model, B, nhd, 1, true);
+  L.g_o = plan_sk(d->d_head, B, d->d_c, d->n_heads, false, d->d_rope);
+  L.g_u = plan_sk(d->d_model, B, nhd, 1, false, d->d_rope);
   L.tc_o = !simt && d->d_c % 64 == 0;
   Carver c{static_cast<char*>(ws)};
   L.o = c.take<uint16_t>((size_t)B * nhd);
-  L.P = (!simt && L.g_u.splits > 1) ? c.take<float>((size_t)L.g_u.splits * B * d->d_model) : nullptr;
+  size_t part = 0;
+  if (!simt) part = std::max(L.tc_o ? L.g_o.part_bytes : 0, L.g_u.part_bytes);
+  L.part = part ? c.take<float>(part / sizeof(float)) : nullptr;
   L.bytes = c.off;
   return L;
 }
@@ -343,10 +405,9 @@ int out_run(const mla_dims* d, const void* o_lat, const void* w_uv, const void* 
   T* o = static_cast<T*>(L.o);
   // o_i = W^UV_i o_lat_i (row block i of W^UV, head i of o_lat)
   if (L.tc_o) {
-    const int r = gemm_tc<T>({w_uv, nhd, d->d_c, d->d_head}, false, {o_lat, B, (long)d->n_heads * d->d_c, d->d_c},
-                             d->d_head, B, d->d_c, d->n_heads, L.g_o, o, false, nhd, d->d_head, 0, st);
+    const int r = gemm_sk<T>({w_uv, nhd, d->d_c, d->d_head}, false, {o_lat, B, (long)d->n_heads * d->d_c, d->d_c},
+                             d->d_head, B, d->d_c, L.g_o, epi_plain(o, nhd, d->d_head), L.part, st, n);
     if (r != MLA_OK) return r;
-    ++n;
   } else {
     launch_rowdot<T, T>(static_cast<const T*>(w_uv), static_cast<const T*>(o_lat), o, d->d_head, d->d_c, B,
                         (long)d->n_heads * d->d_c, nhd, d->n_heads, (long)d->d_head * d->d_c, d->d_c, d->d_head, st, n);
@@ -355,19 +416,10 @@ int out_run(const mla_dims* d, const void* o_lat, const void* w_uv, const void* 
   if (proj_uses_simt()) {
     launch_rowdot<T, T>(static_cast<const T*>(w_o), o, static_cast<T*>(u), d->d_model, nhd, B, nhd, d->d_model, 1, 0,
                         0, 0, st, n);
-  } else if (L.g_u.splits > 1) {
-    const int r = gemm_tc<T>({w_o, d->d_model, nhd, 0}, false, {o, B, nhd, 0}, d->d_model, B, nhd, 1, L.g_u, L.P,
-                             true, d->d_model, 0, (long)B * d->d_model, st);
-    if (r != MLA_OK) return r;
-    launch_reduce<T>(L.P, L.g_u.splits, (long)B * d->d_model, B, d->d_model, d->d_model, static_cast<T*>(u), st);
-    n += 2;
-  } else {
-    const int r = gemm_tc<T>({w_o, d->d_model, nhd, 0}, false, {o, B, nhd, 0}, d->d_model, B, nhd, 1, L.g_u, u, false,
-                             d->d_model, 0, 0, st);
-    if (r != MLA_OK) return r;
-    ++n;
+    return MLA_OK;
   }
-  return MLA_OK;
+  return gemm_sk<T>({w_o, d->d_model, nhd, 0}, false, {o, B, nhd, 0}, d->d_model, B, nhd, L.g_u,
+                    epi_plain(u, d->d_model, 0), L.part, st, n);
 }
 
 }  // namespace host

@@ -108,7 +108,9 @@ def test_append_absorb_out_argument_errors(lib):
                              None) == -1
     assert lib.mla_append_kv(ctypes.byref(cd), FAKE, MISALIGNED, FAKE, FAKE, FAKE, 1, 4, FAKE, 8, 3, FAKE, 1 << 20,
                              None) == -4
-    assert lib.mla_append_kv(ctypes.byref(cd), FAKE, FAKE, FAKE, FAKE, FAKE, 1, 4, FAKE, 8, 3, FAKE, 4,
+    cp = dims(synth.PRODUCTION)  # its append splits the reduction over CTAs and needs scratch
+    assert M.workspace_size(synth.PRODUCTION, M.CALL_APPEND_KV, 3, 1) > 4
+    assert lib.mla_append_kv(ctypes.byref(cp), FAKE, FAKE, FAKE, FAKE, FAKE, 1, 4, FAKE, 8, 3, FAKE, 4,
                              None) == -3
     assert lib.mla_append_kv(ctypes.byref(cd), FAKE, FAKE, FAKE, FAKE, FAKE, 1, 4, FAKE, 8, 0, None, 0,
                              None) == 0
