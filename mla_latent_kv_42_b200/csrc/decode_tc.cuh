@@ -347,29 +347,34 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(dec::kThreads, 1)
               break;
             }
             tc_fence_after();
-            float sv[kTile];
+            // S row h: four TMEM loads in flight, one wait
+            uint32_t sr[4][32];
 #pragma unroll
-            for (int c4 = 0; c4 < 4; ++c4) {
-              uint32_t r[32];
-              tmem_ld32(tmem + lane_base + kSCol + c4 * 32, r);
-              tmem_wait_ld();
-#pragma unroll
-              for (int j = 0; j < 32; ++j) sv[c4 * 32 + j] = u2f(r[j]);
-            }
+            for (int c4 = 0; c4 < 4; ++c4) tmem_ld32(tmem + lane_base + kSCol + c4 * 32, sr[c4]);
+            tmem_wait_ld();
             tc_fence_before();
             mbar_arrive(bar(ctl->s_empty));
 
-            // tokens of this tile: page t (0..63) and, if it belongs to this item, page t+1 (64..127)
+            // tokens of this tile: page t (0..63) and, if it belongs to this item, page t+1 (64..127);
+            // masked tokens become -inf and get weight exactly 0
             const int nv = min(t + 1 < item.t1 ? kTile : kPage, L - t * kPage);
-            float mx = -INFINITY;
+            if (nv < kTile) {
 #pragma unroll
-            for (int k = 0; k < kTile; ++k) {
-              sv[k] = k < nv ? sv[k] * p.scale_log2 : -INFINITY;
-              mx = fmaxf(mx, sv[k]);
+              for (int k = 0; k < kTile; ++k)
+                if (k >= nv) sr[k >> 5][k & 31] = __float_as_uint(-INFINITY);
             }
+            // running maximum on the raw scores (the scale is positive, so the order is the same),
+            // eight independent chains
+            float mxs[8];
+#pragma unroll
+            for (int j = 0; j < 8; ++j) mxs[j] = u2f(sr[0][j]);
+#pragma unroll
+            for (int k = 8; k < kTile; ++k) mxs[k & 7] = fmaxf(mxs[k & 7], u2f(sr[k >> 5][k & 31]));
+            const float mx = fmaxf(fmaxf(fmaxf(mxs[0], mxs[1]), fmaxf(mxs[2], mxs[3])),
+                                   fmaxf(fmaxf(mxs[4], mxs[5]), fmaxf(mxs[6], mxs[7]))) * p.scale_log2;
             float alpha = 1.f;
             if (mx > m_ref + kLazy) {
-              alpha = exp2f(m_ref - mx);
+              alpha = ex2_approx(m_ref - mx);
               l *= alpha;
               m_ref = mx;
             }
@@ -378,24 +383,28 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(dec::kThreads, 1)
               ok = false;
               break;
             }
-            // P row h in the 128-byte-swizzled K-major layout (two 64-token halves); the sum
-            // of the rounded weights is the denominator (it matches what the MMA accumulates)
+            // P row h in the 128-byte-swizzled K-major layout (two 64-token halves):
+            // p = 2^(s * scale - m_ref), one FFMA and one ex2 per token. The sum of the rounded
+            // weights is the denominator (it matches what the MMA accumulates); four chains.
             uint8_t* stage = data + kStageOff + sb * kPStride;
-            float sum = 0.f;
+            float sums[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
             for (int c = 0; c < 16; ++c) {
               uint32_t w[4];
 #pragma unroll
               for (int j = 0; j < 4; ++j) {
+                const int k = 8 * c + 2 * j;
                 const typename Pack<T>::T2 pr =
-                    Pack<T>::make(exp2f(sv[8 * c + 2 * j] - m_ref), exp2f(sv[8 * c + 2 * j + 1] - m_ref));
+                    Pack<T>::make(ex2_approx(fmaf(u2f(sr[k >> 5][k & 31]), p.scale_log2, -m_ref)),
+                                  ex2_approx(fmaf(u2f(sr[(k + 1) >> 5][(k + 1) & 31]), p.scale_log2, -m_ref)));
                 const float2 back = Pack<T>::f2(pr);
-                sum += back.x + back.y;
+                sums[j] += back.x + back.y;
                 w[j] = *reinterpret_cast<const uint32_t*>(&pr);
               }
               *reinterpret_cast<uint4*>(stage + (c >> 3) * 16384 + row_off + (((c & 7) ^ (h & 7)) << 4)) =
                   make_uint4(w[0], w[1], w[2], w[3]);
             }
+            const float sum = (sums[0] + sums[1]) + (sums[2] + sums[3]);
             l += sum;
             reinterpret_cast<float*>(stage + kPTile)[h] = alpha;
             fence_proxy_async_cta();
