@@ -532,13 +532,17 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(dec::kThreads, 1)
               }
               tc_fence_after();
 #pragma unroll 1
-              for (int c0 = 0; c0 < kDc; c0 += 32) {
-                uint32_t r[32];
-                tmem_ld32(tmem + lane_base + kOCol + c0, r);
+              for (int c0 = 0; c0 < kDc; c0 += 128) {  // four TMEM loads in flight per wait
+                uint32_t r[4][32];
+#pragma unroll
+                for (int q4 = 0; q4 < 4; ++q4) tmem_ld32(tmem + lane_base + kOCol + c0 + 32 * q4, r[q4]);
                 tmem_wait_ld();
 #pragma unroll
-                for (int j = 0; j < 32; ++j) r[j] = __float_as_uint(u2f(r[j]) * alpha);
-                tmem_st32(tmem + lane_base + kOCol + c0, r);
+                for (int q4 = 0; q4 < 4; ++q4) {
+#pragma unroll
+                  for (int j = 0; j < 32; ++j) r[q4][j] = __float_as_uint(u2f(r[q4][j]) * alpha);
+                  tmem_st32(tmem + lane_base + kOCol + c0 + 32 * q4, r[q4]);
+                }
               }
               tmem_wait_st();
             }
@@ -559,29 +563,34 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(dec::kThreads, 1)
           const bool whole = item.t0 == 0 && item.t1 == item.n_b;
           const long slot = (long)item.b + cluster;
 #pragma unroll 1
-          for (int c0 = 0; c0 < kDc; c0 += 32) {
-            uint32_t r[32];
-            tmem_ld32(tmem + lane_base + kOCol + c0, r);
+          for (int c0 = 0; c0 < kDc; c0 += 128) {  // four TMEM loads in flight per wait
+            uint32_t r[4][32];
+#pragma unroll
+            for (int q4 = 0; q4 < 4; ++q4) tmem_ld32(tmem + lane_base + kOCol + c0 + 32 * q4, r[q4]);
             tmem_wait_ld();
             if (h < p.n_h) {
               if (whole) {
-                typename Pack<T>::T2* dst = reinterpret_cast<typename Pack<T>::T2*>(
-                    static_cast<T*>(p.o_lat) + ((long)item.b * p.n_h + h) * kDc + c0);
-                uint4 w4[4];
-                uint32_t* w = reinterpret_cast<uint32_t*>(w4);
+                uint4* dst = reinterpret_cast<uint4*>(static_cast<T*>(p.o_lat) + ((long)item.b * p.n_h + h) * kDc + c0);
 #pragma unroll
                 for (int j = 0; j < 16; ++j) {
-                  const typename Pack<T>::T2 v = Pack<T>::make(u2f(r[2 * j]) * inv, u2f(r[2 * j + 1]) * inv);
-                  w[j] = *reinterpret_cast<const uint32_t*>(&v);
-                }
+                  uint32_t w[4];
 #pragma unroll
-                for (int j = 0; j < 4; ++j) reinterpret_cast<uint4*>(dst)[j] = w4[j];
+                  for (int e = 0; e < 4; ++e) {
+                    const int k = 8 * j + 2 * e;
+                    const typename Pack<T>::T2 v =
+                        Pack<T>::make(u2f(r[k >> 5][k & 31]) * inv, u2f(r[(k + 1) >> 5][(k + 1) & 31]) * inv);
+                    w[e] = *reinterpret_cast<const uint32_t*>(&v);
+                  }
+                  dst[j] = make_uint4(w[0], w[1], w[2], w[3]);
+                }
               } else {
                 float4* dst = reinterpret_cast<float4*>(p.o_part + (slot * p.n_h + h) * kDc + c0);
 #pragma unroll
-                for (int j = 0; j < 8; ++j)
-                  dst[j] = make_float4(u2f(r[4 * j]) * inv, u2f(r[4 * j + 1]) * inv, u2f(r[4 * j + 2]) * inv,
-                                       u2f(r[4 * j + 3]) * inv);
+                for (int j = 0; j < 32; ++j) {
+                  const int k = 4 * j;
+                  dst[j] = make_float4(u2f(r[k >> 5][k & 31]) * inv, u2f(r[k >> 5][(k & 31) + 1]) * inv,
+                                       u2f(r[k >> 5][(k & 31) + 2]) * inv, u2f(r[k >> 5][(k & 31) + 3]) * inv);
+                }
               }
             }
           }
