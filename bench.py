@@ -21,6 +21,7 @@ from __future__ import annotations
 import argparse
 import json
 import os
+import re
 import statistics
 import subprocess
 import sys
@@ -184,6 +185,24 @@ def rank_workload(w, rank: int):
     """Each rank owns its own sequences: the same workload shape with a rank-specific seed."""
     import dataclasses
     return dataclasses.replace(w, seed=w.seed + 1000 * rank) if rank else w
+
+
+def measured_decode_traffic(workload: str):
+    """DRAM bytes (read + write) of one decode-kernel launch from the committed ncu summary, if it was
+    taken on this workload and the kernel source is unchanged since; otherwise None."""
+    import hashlib
+    prof = os.path.join(ROOT, "profiles", f"ncu_decode_tc_{workload.replace('_bf16', '').replace('_fp16', '')}.md")
+    src = os.path.join(ROOT, "mla_latent_kv_42_b200", "csrc", "decode_tc.cuh")
+    if not os.path.exists(prof):
+        return None
+    text = open(prof).read()
+    m_hash = re.search(r"decode_tc.cuh sha256 prefix at capture: ([0-9a-f]+)", text)
+    m_bytes = re.search(r"^traffic_bytes: (\d+)", text, re.M)
+    if not m_hash or not m_bytes:
+        return None
+    if hashlib.sha256(open(src, "rb").read()).hexdigest()[:len(m_hash.group(1))] != m_hash.group(1):
+        return None
+    return int(m_bytes.group(1))
 
 
 def max_over_ranks(values, device, world: int):
@@ -355,7 +374,7 @@ def run_mla(args):
             roof = {"bound": "tensor", "achieved": dflops / dec_s / 1e12, "peak": peaks["bf16_tflops"],
                     "unit": "TFLOP/s"}
         roof["frac"] = roof["achieved"] / roof["peak"]
-        roof["traffic"] = None
+        roof["traffic"] = measured_decode_traffic(w.name)
         roof["kernel"] = "mla_decode_attention"
         roof["peak_source"] = peak_src + " (burst; MEASURED_PEAKS.json)" if peak_src == "measured" else peak_src
         roof["roofline_us"] = max(t_mem, t_flop) * 1e6
