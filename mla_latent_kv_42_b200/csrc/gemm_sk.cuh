@@ -303,9 +303,29 @@ __global__ void __launch_bounds__(192, 1)
     // Tables of the fused output step for the one n tile (RoPE cos/sin per token and pair,
     // cache row offset per token), built once while the first tiles stream in. With several
     // n tiles the step computes them per element instead.
-    const bool use_tab = MODE != kEpiPlain && p.n_tiles == 1;
+    // Shared-memory tables are built only by CTAs that finish a whole tile themselves: the cache
+    // row offsets for any whole append tile, the RoPE cos/sin for a whole tile with rope rows.
+    bool tab_row = false, tab_cs = false;
+    if (MODE != kEpiPlain && p.n_tiles == 1) {
+      for (long i = i0; i < i1;) {
+        const int tile = (int)(i / p.kb);
+        const long tile_end = (long)(tile + 1) * p.kb, seg_end = min(i1, tile_end);
+        if (i % p.kb == 0 && seg_end == tile_end) {
+          tab_row |= MODE == kEpiAppend;
+          tab_cs |= ((tile / p.n_tiles) % p.m_tiles) * C::BM + C::BM > p.epi.rope_lo;
+        }
+        i = seg_end;
+      }
+    }
     griddep_wait();  // token positions, cache slots and outputs belong to earlier kernels
-    if (use_tab) {
+    if (MODE != kEpiPlain && p.epi.cs_glob != nullptr) {  // the reduction's table: a slice per CTA
+      for (int e = cta * 128 + ml; e < p.N * half_rope; e += G * 128) {
+        float c, sn;
+        rope_cos_sin(p.epi.pos[e / half_rope], e % half_rope, p.epi.d_rope, p.epi.rope_base, c, sn);
+        p.epi.cs_glob[e] = make_float2(c, sn);
+      }
+    }
+    if (tab_cs) {
       double theta = 0.0;
       int theta_k = -1;
       for (int e = ml; e < BN * half_rope; e += 128) {
@@ -317,19 +337,18 @@ __global__ void __launch_bounds__(192, 1)
         float c = 1.f, sn = 0.f;
         if (n < p.N) rope_cos_sin_at(p.epi.pos[n], theta, c, sn);
         cs_tab[e] = make_float2(c, sn);
-        if (cta == 0 && p.epi.cs_glob != nullptr && n < p.N) p.epi.cs_glob[e] = make_float2(c, sn);
       }
-      if (MODE == kEpiAppend)
-        for (int e = ml; e < BN; e += 128) {
-          long rb = -1;
-          if (e < p.N) {
-            rb = append_row_base(p.epi, e);
-            if (rb < 0 && cta == 0) record_error(MLA_ERR_BAD_PAGE);
-          }
-          row_tab[e] = rb;
-        }
-      named_bar_sync(1, 128);
     }
+    if (tab_row)
+      for (int e = ml; e < BN; e += 128) {
+        long rb = -1;
+        if (e < p.N) {
+          rb = append_row_base(p.epi, e);
+          if (rb < 0) record_error(MLA_ERR_BAD_PAGE);
+        }
+        row_tab[e] = rb;
+      }
+    if (tab_cs || tab_row) named_bar_sync(1, 128);
     int seg = 0;
     long i = i0;
     while (i < i1) {
@@ -370,13 +389,13 @@ __global__ void __launch_bounds__(192, 1)
             const float w = __shfl_xor_sync(0xffffffffu, v, 1);  // the pair partner's value
             if (rot && nl < nv) {
               float2 q;
-              if (use_tab) q = cs_tab[nl * half_rope + k];
+              if (tab_cs) q = cs_tab[nl * half_rope + k];
               else rope_cos_sin(p.epi.pos[n0 + nl], k, p.epi.d_rope, p.epi.rope_base, q.x, q.y);
               v = (m & 1) ? fmaf(w, q.y, v * q.x) : fmaf(v, q.x, -w * q.y);
             }
           }
           if (nl < nv && row_ok)
-            dst.put(n0 + nl, v, MODE != kEpiAppend ? 0 : use_tab ? row_tab[nl] : append_row_base(p.epi, n0 + nl));
+            dst.put(n0 + nl, v, MODE != kEpiAppend ? 0 : tab_row ? row_tab[nl] : append_row_base(p.epi, n0 + nl));
         }
       }
       tc_fence_before();
@@ -394,7 +413,7 @@ __global__ void __launch_bounds__(192, 1)
 }
 
 // Tiles split over several CTAs: sum the fp32 partial slots in CTA order and apply the output
-// step. Block (tile, 8-column group); thread = row pair (2q, 2q+1) of one column.
+// step. Block (tile, 4-column group); thread = row pair (2q, 2q+1) of one column.
 template <typename T, int BN, int MODE>
 __global__ void __launch_bounds__(256) k_sk_reduce(const SkParams p, int G) {
   griddep_wait();
@@ -406,54 +425,49 @@ __global__ void __launch_bounds__(256) k_sk_reduce(const SkParams p, int G) {
   const int nt = tile % p.n_tiles, mt = (tile / p.n_tiles) % p.m_tiles, z = tile / (p.n_tiles * p.m_tiles);
   const int q = threadIdx.x & 63;
   const int m = mt * 128 + 2 * q;
+  const int nl = blockIdx.y * 4 + (threadIdx.x >> 6);
+  const int n = nt * BN + nl;
+  if (nl >= BN || n >= p.N || m >= p.M) return;
+  // slot (tile + c) of each contributing CTA c; eight loads in flight, summed in CTA order
+  const float* src = p.part + ((long)tile + c_lo) * (128L * BN) + (long)nl * 128 + 2 * q;
+  float a = 0.f, b = 0.f;
+  for (int c = c_lo; c <= c_hi; c += 8) {
+    float2 v[8];
 #pragma unroll
-  for (int j = 0; j < 2; ++j) {
-    const int nl = blockIdx.y * 8 + (threadIdx.x >> 6) + 4 * j;
-    const int n = nt * BN + nl;
-    if (nl >= BN || n >= p.N || m >= p.M) continue;
-    const float* src = p.part + ((long)tile + c_lo) * (128L * BN) + (long)nl * 128 + 2 * q;
-    float a = 0.f, b = 0.f;
-    int c = c_lo;
-    for (; c + 3 <= c_hi; c += 4, src += 4 * 128L * BN) {  // loads in flight together, sums in CTA order
-      float2 v[4];
+    for (int u = 0; u < 8; ++u)
+      v[u] = c + u <= c_hi ? *reinterpret_cast<const float2*>(src + (long)(c - c_lo + u) * (128L * BN))
+                           : make_float2(0.f, 0.f);
 #pragma unroll
-      for (int u = 0; u < 4; ++u) v[u] = *reinterpret_cast<const float2*>(src + u * 128L * BN);
-#pragma unroll
-      for (int u = 0; u < 4; ++u) {
+    for (int u = 0; u < 8; ++u)
+      if (c + u <= c_hi) {
         a += v[u].x;
         b += v[u].y;
       }
-    }
-    for (; c <= c_hi; ++c, src += 128L * BN) {
-      const float2 v = *reinterpret_cast<const float2*>(src);
-      a += v.x;
-      b += v.y;
-    }
-    long rb = 0;
-    if (MODE == kEpiAppend) {
-      rb = append_row_base(p.epi, n);
-      if (rb < 0) {
-        record_error(MLA_ERR_BAD_PAGE);
-        continue;
-      }
-    }
-    if (MODE != kEpiPlain && m >= p.epi.rope_lo) {
-      const int k = ((m - p.epi.rope_lo) % p.epi.d_rope) >> 1;
-      float cs, sn;
-      if (p.epi.cs_glob != nullptr) {
-        const float2 t = p.epi.cs_glob[(long)n * (p.epi.d_rope / 2) + k];
-        cs = t.x;
-        sn = t.y;
-      } else {
-        rope_cos_sin(p.epi.pos[n], k, p.epi.d_rope, p.epi.rope_base, cs, sn);
-      }
-      const float ra = fmaf(a, cs, -b * sn), rb2 = fmaf(b, cs, a * sn);
-      a = ra;
-      b = rb2;
-    }
-    RowDest<T, MODE>(p.epi, z, m).put(n, a, rb);
-    if (m + 1 < p.M) RowDest<T, MODE>(p.epi, z, m + 1).put(n, b, rb);
   }
+  long rb = 0;
+  if (MODE == kEpiAppend) {
+    rb = append_row_base(p.epi, n);
+    if (rb < 0) {
+      record_error(MLA_ERR_BAD_PAGE);
+      return;
+    }
+  }
+  if (MODE != kEpiPlain && m >= p.epi.rope_lo) {
+    const int k = ((m - p.epi.rope_lo) % p.epi.d_rope) >> 1;
+    float cs, sn;
+    if (p.epi.cs_glob != nullptr) {
+      const float2 t = p.epi.cs_glob[(long)n * (p.epi.d_rope / 2) + k];
+      cs = t.x;
+      sn = t.y;
+    } else {
+      rope_cos_sin(p.epi.pos[n], k, p.epi.d_rope, p.epi.rope_base, cs, sn);
+    }
+    const float ra = fmaf(a, cs, -b * sn), rb2 = fmaf(b, cs, a * sn);
+    a = ra;
+    b = rb2;
+  }
+  RowDest<T, MODE>(p.epi, z, m).put(n, a, rb);
+  if (m + 1 < p.M) RowDest<T, MODE>(p.epi, z, m + 1).put(n, b, rb);
 }
 
 }  // namespace tc

@@ -153,7 +153,7 @@ cudaError_t run_sk(const CUtensorMap& ma, const CUtensorMap& mb, const tc::SkPar
   if (e != cudaSuccess) return e;
   ++n;
   if (g.split) {
-    e = launch_pdl(tc::k_sk_reduce<T, BN, MODE>, dim3(g.tiles, BN / 8), dim3(256), 0, st, p, g.G);
+    e = launch_pdl(tc::k_sk_reduce<T, BN, MODE>, dim3(g.tiles, BN / 4), dim3(256), 0, st, p, g.G);
     if (e != cudaSuccess) return e;
     ++n;
   }
