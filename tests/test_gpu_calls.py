@@ -170,6 +170,30 @@ def test_decode_bitwise_repeatable_at_full_load(scale):
         assert torch.equal(o, first) and torch.equal(l, first_l)
 
 
+@pytest.mark.parametrize("fam", ["running_bf16", "production_bf16"])
+def test_decode_needle_tokens(fam):
+    """One planted token per sequence scores ~20 above every other token, for every head. The
+    needles sit on page, tile and split boundaries and at the first and last token; the output
+    must be the needle's latent, and the split-KV merge must pick the partial that holds it."""
+    w = FAMILIES[fam]
+    d = w.dims
+    lens = np.array([1, 64, 65, 129, 777, 4097, 20000])
+    needles = np.array([0, 63, 64, 128, 776, 4096, 11111])
+    case = CacheCase(w, cached=lens, paging="shuffled", spare_tokens=0)
+    q64 = synth.synthetic_query(w, len(lens)).double()
+    target = 20.0 * np.sqrt(d.d_head + d.d_rope)  # raw dot product whose scaled score is 20
+    for b, j in enumerate(needles):
+        r = case.prefix(b)[int(j)].double().cpu()
+        q64[b] += (target / float(r @ r)) * r  # every head gains q.r = target on the needle
+    q = q64.to(synth.storage_dtype(d))
+    o_lat, lse = run_decode(case, q)
+    assert M.read_device_status() == 0
+    check_decode(case, q, o_lat, lse, f"{fam} needles")
+    for b, j in enumerate(needles):
+        want = to64(case.prefix(b)[int(j)][:d.d_c]).reshape(1, -1).repeat(d.n_heads, 0)
+        assert_parity(to64(o_lat[b]), want, f"{fam} needle row b={b} j={j}")
+
+
 def test_decode_all_equal_rows_and_single_token_are_exact():
     for w in (W_RUN16, W_PROD):
         d = w.dims
