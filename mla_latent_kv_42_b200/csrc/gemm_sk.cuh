@@ -43,7 +43,10 @@ struct EpiParams {
   int rope_lo, d_rope;
   double rope_base;
   const int* pos;       // [N]
-  float2* cs_glob;      // [N][d_rope/2] cos/sin, written by CTA 0 for the reduction (or null)
+  float2* cs_glob;      // [N][d_rope/2] cos/sin for split tiles' reduction (or null)
+  int cs_ready;         // 1: cs_glob was filled by an earlier kernel (read it, do not compute it)
+  int rope_in_reduce;   // 1: tiles with rope rows always go through k_sk_reduce (even whole ones)
+  float2* cs_prefill;   // plain mode: fill this [N][d_rope/2] table for the next kernel (or null)
   // append
   const int* seq_idx;   // [N]
   const int* bt;
@@ -130,6 +133,15 @@ struct RowDest {
   }
 };
 
+// cos/sin of one RoPE angle, kept out of line: the epilogue loop that may call it is unrolled and
+// runs with cold instruction fetch, so an inlined double-precision pow and sincos in its (rarely
+// taken) branch would slow every pass through it.
+__device__ __noinline__ float2 rope_cs_out_of_line(int pos, int k, int d_rope, double base) {
+  float2 q;
+  rope_cos_sin(pos, k, d_rope, base, q.x, q.y);
+  return q;
+}
+
 // Cache row offset (elements) of token n for the append step, or -1 (error recorded).
 __device__ __forceinline__ long append_row_base(const EpiParams& e, int n) {
   const int s = e.seq_idx[n], p = e.pos[n];
@@ -183,7 +195,6 @@ __global__ void __launch_bounds__(192, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
-  if (threadIdx.x == 0) griddep_launch();
 
   auto tile_coords = [&](int tile, int& z, int& mt, int& nt) {
     nt = tile % p.n_tiles;
@@ -310,22 +321,28 @@ __global__ void __launch_bounds__(192, 1)
       for (long i = i0; i < i1;) {
         const int tile = (int)(i / p.kb);
         const long tile_end = (long)(tile + 1) * p.kb, seg_end = min(i1, tile_end);
-        if (i % p.kb == 0 && seg_end == tile_end) {
+        const bool rope_tile = ((tile / p.n_tiles) % p.m_tiles) * C::BM + C::BM > p.epi.rope_lo;
+        if (i % p.kb == 0 && seg_end == tile_end && !(p.epi.rope_in_reduce && rope_tile)) {
           tab_row |= MODE == kEpiAppend;
-          tab_cs |= ((tile / p.n_tiles) % p.m_tiles) * C::BM + C::BM > p.epi.rope_lo;
+          tab_cs |= rope_tile;
         }
         i = seg_end;
       }
     }
     griddep_wait();  // token positions, cache slots and outputs belong to earlier kernels
-    if (MODE != kEpiPlain && p.epi.cs_glob != nullptr) {  // the reduction's table: a slice per CTA
+    // RoPE cos/sin tables in global memory, a slice per CTA: for this kernel's reduction, or
+    // (cs_prefill) for the next kernel, whose epilogues then copy it instead of computing it
+    float2* const fill = MODE == kEpiPlain ? p.epi.cs_prefill : (p.epi.cs_ready ? nullptr : p.epi.cs_glob);
+    if (fill != nullptr)
       for (int e = cta * 128 + ml; e < p.N * half_rope; e += G * 128) {
         float c, sn;
         rope_cos_sin(p.epi.pos[e / half_rope], e % half_rope, p.epi.d_rope, p.epi.rope_base, c, sn);
-        p.epi.cs_glob[e] = make_float2(c, sn);
+        fill[e] = make_float2(c, sn);
       }
-    }
-    if (tab_cs) {
+    if (tab_cs && p.epi.cs_ready) {
+      for (int e = ml; e < BN * half_rope; e += 128)
+        cs_tab[e] = e / half_rope < p.N ? p.epi.cs_glob[e] : make_float2(1.f, 0.f);
+    } else if (tab_cs) {
       double theta = 0.0;
       int theta_k = -1;
       for (int e = ml; e < BN * half_rope; e += 128) {
@@ -354,9 +371,12 @@ __global__ void __launch_bounds__(192, 1)
     while (i < i1) {
       const int tile = (int)(i / p.kb), kbi0 = (int)(i % p.kb);
       const long seg_end = min(i1, (long)(tile + 1) * p.kb);
-      const bool whole = kbi0 == 0 && seg_end == (long)(tile + 1) * p.kb;
       int z, mt, nt;
       tile_coords(tile, z, mt, nt);
+      // A tile with rope rows may be left to the reduction kernel: rotating it here reads the
+      // cos/sin table from shared memory while the next tile streams through it, which is slow.
+      const bool whole = kbi0 == 0 && seg_end == (long)(tile + 1) * p.kb &&
+                         !(p.epi.rope_in_reduce && mt * C::BM + C::BM > p.epi.rope_lo);
       const int m = mt * C::BM + ml;
       const int n0 = nt * BN;
       const bool rot = MODE != kEpiPlain && m >= p.epi.rope_lo;
@@ -370,32 +390,41 @@ __global__ void __launch_bounds__(192, 1)
       tc_fence_after();
       const uint32_t acc = tmem + lane_base + (uint32_t)(b * BN);
       float* slot = p.part + ((long)tile + cta) * (128L * BN) + ml;
+      // 32 columns per TMEM load, the next chunk's load in flight while this one is stored: the
+      // load latency is paid about once per tile instead of once per few columns
+      uint32_t ra[32], rb[32];
+      tmem_ld32(acc, ra);
+      tmem_wait_ld();
 #pragma unroll 1
-      for (int c0 = 0; c0 < BN; c0 += 8) {
-        uint32_t r[8];
-        tmem_ld8(acc + c0, r);
-        tmem_wait_ld();
+      for (int c0 = 0; c0 < BN; c0 += 32) {
+        const bool more = c0 + 32 < BN;
+        if (more) tmem_ld32(acc + c0 + 32, rb);
         if (!whole) {
 #pragma unroll
-          for (int j = 0; j < 8; ++j)
-            if (c0 + j < nv) slot[(long)(c0 + j) * 128] = u2f(r[j]);
-          continue;
-        }
+          for (int j = 0; j < 32; ++j)
+            if (c0 + j < nv) slot[(long)(c0 + j) * 128] = u2f(ra[j]);
+        } else {
 #pragma unroll
-        for (int j = 0; j < 8; ++j) {
-          float v = u2f(r[j]);
-          const int nl = c0 + j;
-          if (MODE != kEpiPlain && rope_warp) {  // warp-uniform: every lane takes part in the exchange
-            const float w = __shfl_xor_sync(0xffffffffu, v, 1);  // the pair partner's value
-            if (rot && nl < nv) {
-              float2 q;
-              if (tab_cs) q = cs_tab[nl * half_rope + k];
-              else rope_cos_sin(p.epi.pos[n0 + nl], k, p.epi.d_rope, p.epi.rope_base, q.x, q.y);
-              v = (m & 1) ? fmaf(w, q.y, v * q.x) : fmaf(v, q.x, -w * q.y);
+          for (int j = 0; j < 32; ++j) {
+            float v = u2f(ra[j]);
+            const int nl = c0 + j;
+            if (MODE != kEpiPlain && rope_warp) {  // warp-uniform: every lane takes part in the exchange
+              const float w = __shfl_xor_sync(0xffffffffu, v, 1);  // the pair partner's value
+              if (rot && nl < nv) {
+                float2 q;
+                if (tab_cs) q = cs_tab[nl * half_rope + k];
+                else q = rope_cs_out_of_line(p.epi.pos[n0 + nl], k, p.epi.d_rope, p.epi.rope_base);
+                v = (m & 1) ? fmaf(w, q.y, v * q.x) : fmaf(v, q.x, -w * q.y);
+              }
             }
+            if (nl < nv && row_ok)
+              dst.put(n0 + nl, v, MODE != kEpiAppend ? 0 : tab_row ? row_tab[nl] : append_row_base(p.epi, n0 + nl));
           }
-          if (nl < nv && row_ok)
-            dst.put(n0 + nl, v, MODE != kEpiAppend ? 0 : tab_row ? row_tab[nl] : append_row_base(p.epi, n0 + nl));
+        }
+        if (more) {
+          tmem_wait_ld();
+#pragma unroll
+          for (int j = 0; j < 32; ++j) ra[j] = rb[j];
         }
       }
       tc_fence_before();
@@ -406,6 +435,9 @@ __global__ void __launch_bounds__(192, 1)
   }
   tc_fence_before();
   __syncthreads();
+  // Dependents may launch only now: a small-block dependent (the split reduction) resident
+  // early would share the SMs with the epilogue warps while they still work.
+  if (threadIdx.x == 0) griddep_launch();
   if (warp == 5) {
     tc_fence_after();
     tmem_dealloc(tmem, C::TMEM_COLS);
@@ -421,8 +453,8 @@ __global__ void __launch_bounds__(256) k_sk_reduce(const SkParams p, int G) {
   const int tile = blockIdx.x;
   const long t0 = (long)tile * p.kb;
   const int c_lo = sk_owner(p, t0, G), c_hi = sk_owner(p, t0 + p.kb - 1, G);
-  if (c_lo == c_hi) return;  // finished whole by its CTA
   const int nt = tile % p.n_tiles, mt = (tile / p.n_tiles) % p.m_tiles, z = tile / (p.n_tiles * p.m_tiles);
+  if (c_lo == c_hi && !(p.epi.rope_in_reduce && mt * 128 + 128 > p.epi.rope_lo)) return;  // finished by its CTA
   const int q = threadIdx.x & 63;
   const int m = mt * 128 + 2 * q;
   const int nl = blockIdx.y * 4 + (threadIdx.x >> 6);

@@ -316,7 +316,7 @@ inline AbsorbLayout absorb_layout(const mla_dims* d, int B, void* ws) {
   size_t part = 0;
   if (!simt) part = std::max(L.g1.part_bytes, std::max(L.g2.part_bytes, L.tc_uk ? L.g3.part_bytes : 0));
   L.part = part ? c.take<float>(part / sizeof(float)) : nullptr;
-  L.cs = (!simt && L.g2.split && L.g2.n_tiles == 1) ? c.take<float2>((size_t)B * (d->d_rope / 2)) : nullptr;
+  L.cs = (!simt && L.g2.n_tiles == 1) ? c.take<float2>((size_t)B * (d->d_rope / 2)) : nullptr;
   L.bytes = c.off;
   return L;
 }
@@ -339,9 +339,14 @@ int absorb_run(const mla_dims* d, const void* h, const void* w_dq, const void* w
         d->rope_base);
     ++n;
   } else {
-    // c^Q = W^DQ h
-    int r = gemm_sk<T>({w_dq, d->d_cq, d->d_model, 0}, false, {h, B, d->d_model, 0}, d->d_cq, B, d->d_model, L.g1,
-                       epi_plain(cq, d->d_cq, 0), L.part, st, n);
+    // c^Q = W^DQ h; its CTAs also tabulate the query's RoPE cos/sin for the next product
+    tc::EpiParams e1 = epi_plain(cq, d->d_cq, 0);
+    e1.cs_prefill = L.cs;
+    e1.pos = pos;
+    e1.d_rope = d->d_rope;
+    e1.rope_base = d->rope_base;
+    int r = gemm_sk<T>({w_dq, d->d_cq, d->d_model, 0}, false, {h, B, d->d_model, 0}, d->d_cq, B, d->d_model, L.g1, e1,
+                       L.part, st, n);
     if (r != MLA_OK) return r;
     // [q^C ; q^] = [W^UQ ; W^QR] c^Q; q^C -> qc, q^R_i = RoPE(q^_i) -> q_out[b][i][d_c:]
     tc::EpiParams e{};
@@ -355,6 +360,8 @@ int absorb_run(const mla_dims* d, const void* h, const void* w_dq, const void* w
     e.n_h = d->n_heads;
     e.d_c = d->d_c;
     e.cs_glob = L.cs;
+    e.cs_ready = L.cs != nullptr;
+    e.rope_in_reduce = L.g2.split && L.cs != nullptr;  // the reduction runs anyway
     r = gemm_sk<T>({w_uq_qr, nq, d->d_cq, 0}, false, {cq, B, d->d_cq, 0}, nq, B, d->d_cq, L.g2, e, L.part, st, n);
     if (r != MLA_OK) return r;
   }
