@@ -76,11 +76,6 @@ __device__ __forceinline__ float warp_sum(float v) {
   for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
   return v;
 }
-__device__ __forceinline__ float warp_max(float v) {
-#pragma unroll
-  for (int o = 16; o > 0; o >>= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, o));
-  return v;
-}
 
 // cos/sin of the RoPE angle of pair k at position pos: pos * base^(-2k/d_rope). The angle is
 // formed and reduced in double precision (an fp32 angle at position 131072 would be off by

@@ -12,7 +12,8 @@
 // projection's output step and stores. A partial segment is written as fp32 to slot
 // (tile + cta) of the partial buffer — unique, because both the tile and the CTA index only
 // grow along the iteration space — and k_sk_reduce sums a tile's slots in CTA order (a fixed
-// order, so results repeat bit for bit) before applying the same output step.
+// order, so results repeat bit for bit) before applying the same output step. With
+// rope_in_reduce, tiles holding rope rows go that way even when one CTA finishes them.
 //
 // Output steps (EpiParams::mode):
 //   plain   out[z * batch_off + n * ld + m]

@@ -113,23 +113,15 @@ __device__ __forceinline__ uint32_t mapa(uint32_t saddr, uint32_t rank) {
 }
 __device__ __forceinline__ void cluster_arrive() { asm volatile("barrier.cluster.arrive.release.aligned;" ::: "memory"); }
 __device__ __forceinline__ void cluster_wait() { asm volatile("barrier.cluster.wait.acquire.aligned;" ::: "memory"); }
-__device__ __forceinline__ void st_cluster_v4(uint32_t caddr, uint4 v) {
-  asm volatile("st.shared::cluster.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(caddr), "r"(v.x), "r"(v.y), "r"(v.z),
-               "r"(v.w)
-               : "memory");
-}
 __device__ __forceinline__ void st_cluster_f32(uint32_t caddr, float v) {
   asm volatile("st.shared::cluster.f32 [%0], %1;" ::"r"(caddr), "f"(v) : "memory");
 }
 __device__ __forceinline__ void st_cluster_u32(uint32_t caddr, uint32_t v) {
   asm volatile("st.shared::cluster.u32 [%0], %1;" ::"r"(caddr), "r"(v) : "memory");
 }
-// Order this thread's generic-proxy writes to shared memory (local or a peer's) before later
-// async-proxy reads of it (TMA / tcgen05.mma operands).
+// Order this thread's generic-proxy writes to this CTA's shared memory before later async-proxy
+// reads of it (bulk copies, tcgen05.mma operands).
 __device__ __forceinline__ void fence_proxy_async_cta() { asm volatile("fence.proxy.async.shared::cta;" ::: "memory"); }
-__device__ __forceinline__ void fence_proxy_async_cluster() {
-  asm volatile("fence.proxy.async.shared::cluster;" ::: "memory");
-}
 
 // Arrive on a peer CTA's barrier and add `bytes` to the transaction count its current phase
 // waits for (releasing this thread's prior writes at cluster scope).
@@ -229,12 +221,6 @@ __device__ __forceinline__ void tmem_ld32(uint32_t taddr, uint32_t (&r)[32]) {
       : MLA_R8(0), MLA_R8(8), MLA_R8(16), MLA_R8(24)
       : "r"(taddr)
       : "memory");
-}
-__device__ __forceinline__ void tmem_ld8(uint32_t taddr, uint32_t (&r)[8]) {
-  asm volatile("tcgen05.ld.sync.aligned.32x32b.x8.b32 {%0,%1,%2,%3,%4,%5,%6,%7}, [%8];"
-               : MLA_R8(0)
-               : "r"(taddr)
-               : "memory");
 }
 #undef MLA_R8
 // 2^x with the hardware's approximate exponential (flushes subnormal results to zero); the
