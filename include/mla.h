@@ -163,6 +163,18 @@ const char* mla_error_string(int code);
  * (for launch accounting in benchmarks). */
 int32_t mla_last_launch_count(int32_t call);
 
+typedef struct CUevent_st* mla_event_t;
+
+/* Profiling hook (not part of the method): from this call on, every mla_decode_attention (and
+ * _noalloc) call made by this host thread records `before` on its stream immediately before the
+ * attention kernel and `after` immediately after it, so that the kernel's own duration can be
+ * read with cudaEventElapsedTime apart from the planner and the split-KV merge launched in the
+ * same call. Pass NULL for both to stop. The events belong to the caller, who creates them
+ * (with timing) and destroys them. An event recorded between two launches keeps the second
+ * from starting early into the first one's tail, so leave the hook off where throughput
+ * matters. Returns MLA_OK, or MLA_ERR_INVALID_ARG if exactly one of the two is NULL. */
+int mla_set_decode_timing_events(mla_event_t before, mla_event_t after);
+
 /*
  * mla_decode_attention_noalloc — mla_decode_attention without a caller-supplied workspace.
  * The paper has no counterpart: it is a convenience for callers that cannot allocate device

@@ -54,6 +54,7 @@ _SIGS = {
     "mla_error_string": (ctypes.c_char_p, [ctypes.c_int]),
     "mla_last_launch_count": (_I32, [_I32]),
     "mla_decode_attention_noalloc": (ctypes.c_int, [_P, _P, _P, _I32, _P, _I32, _P, _I32, _I32, _P, _P, _P]),
+    "mla_set_decode_timing_events": (ctypes.c_int, [_P, _P]),
 }
 
 
@@ -245,6 +246,17 @@ def read_device_status(stream=None) -> int:
 
 def last_launch_count(call: int) -> int:
     return int(_lib().mla_last_launch_count(call))
+
+
+def set_decode_timing_events(before=None, after=None):
+    """mla_set_decode_timing_events: record two torch.cuda.Event objects around the attention
+    kernel of this thread's later decode calls (None, None: stop). The events must have been
+    recorded once (so that they exist) before they are handed over."""
+    h = lambda e: None if e is None else ctypes.c_void_p(e.cuda_event)
+    r = _lib().mla_set_decode_timing_events(h(before), h(after))
+    if r != 0:
+        raise MLAError(r, "mla_set_decode_timing_events")
+
 
 
 @dataclass

@@ -16,6 +16,14 @@ using namespace mla;
 namespace {
 
 thread_local int32_t t_launches[4] = {0, 0, 0, 0};
+// Profiling hook: events recorded around the attention kernel of this thread's decode calls.
+thread_local cudaEvent_t t_ev_before = nullptr, t_ev_after = nullptr;
+inline void mark_before(cudaStream_t st) {
+  if (t_ev_before != nullptr) cudaEventRecord(t_ev_before, st);
+}
+inline void mark_after(cudaStream_t st) {
+  if (t_ev_after != nullptr) cudaEventRecord(t_ev_after, st);
+}
 
 constexpr int kMaxDevices = 64;
 
@@ -201,8 +209,10 @@ int decode_tc_impl(const mla_dims* d, const void* q, const void* pool, int32_t n
   p.lse_out = lse_out;
   p.o_part = o_part;
   p.lse_part = lse_part;
+  mark_before(st);
   if (launch_pdl(tc::k_decode_tc<T>, dim3(2 * C), dim3(tc::dec::kThreads), tc::dec::kSmem, st, map, p) != cudaSuccess)
     return MLA_ERR_CUDA;
+  mark_after(st);
   if (launch_pdl(tc::k_decode_tc_merge<T>, dim3(B, (d->n_heads + 7) / 8), dim3(256), 0, st,
                  static_cast<const float*>(o_part), static_cast<const float*>(lse_part),
                  static_cast<const int*>(prefix), (int)B, C, (int)d->n_heads, static_cast<T*>(o_lat),
@@ -217,10 +227,12 @@ void launch_decode_simt(const mla_dims* d, const DecodePlan& p, const void* q, c
                         void* o_lat, float* lse_out, float* o_part, float* lse_part, cudaStream_t st) {
   const float scale_log2 = (float)(1.0 / std::sqrt((double)(d->d_head + d->d_rope)) * 1.4426950408889634);
   dim3 grid(p.n_splits, B, p.head_groups);
+  mark_before(st);
   k_decode_simt<T, NPAIR><<<grid, 256, 0, st>>>(
       static_cast<const T*>(q), static_cast<const T*>(pool), bt, max_pages, seq_lens, max_seq_len, num_pages,
       d->n_heads, d->d_c, d->d_c + d->d_rope, d->page_size, scale_log2, p.split_len, p.n_splits,
       static_cast<T*>(o_lat), lse_out, o_part, lse_part);
+  mark_after(st);
 }
 
 template <typename T>
@@ -403,6 +415,13 @@ const char* mla_error_string(int code) {
 }
 
 int32_t mla_last_launch_count(int32_t call) { return (call >= 0 && call < 4) ? t_launches[call] : -1; }
+
+int mla_set_decode_timing_events(mla_event_t before, mla_event_t after) {
+  if ((before == nullptr) != (after == nullptr)) return MLA_ERR_INVALID_ARG;
+  t_ev_before = reinterpret_cast<cudaEvent_t>(before);
+  t_ev_after = reinterpret_cast<cudaEvent_t>(after);
+  return MLA_OK;
+}
 
 }  // extern "C"
 

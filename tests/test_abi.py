@@ -120,6 +120,13 @@ def test_append_absorb_out_argument_errors(lib):
     assert lib.mla_out_proj(ctypes.byref(cd), FAKE, FAKE, FAKE, FAKE, -1, FAKE, 1 << 20, None) == -1
 
 
+def test_decode_timing_hook_arguments(lib):
+    fake = ctypes.c_void_p(0x100000)
+    assert lib.mla_set_decode_timing_events(fake, None) == -1
+    assert lib.mla_set_decode_timing_events(None, fake) == -1
+    assert lib.mla_set_decode_timing_events(None, None) == 0
+
+
 def test_workspace_sizes_are_consistent(lib):
     for d in (synth.RUNNING, synth.PRODUCTION):
         for call in range(4):

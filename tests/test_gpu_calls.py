@@ -194,6 +194,29 @@ def test_decode_needle_tokens(fam):
         assert_parity(to64(o_lat[b]), want, f"{fam} needle row b={b} j={j}")
 
 
+def test_decode_timing_hook_brackets_the_attention_kernel():
+    w = W_PROD
+    lens = np.array([3000, 17, 4097])
+    case = CacheCase(w, cached=lens, paging="shuffled")
+    q = synth.synthetic_query(w, 3)
+    ref_o, ref_l = run_decode(case, q)
+    ev = [torch.cuda.Event(enable_timing=True) for _ in range(4)]
+    for e in ev:
+        e.record()
+    M.set_decode_timing_events(ev[1], ev[2])
+    try:
+        ev[0].record()
+        o, l = run_decode(case, q)
+        ev[3].record()
+    finally:
+        M.set_decode_timing_events(None, None)
+    torch.cuda.synchronize()
+    assert M.read_device_status() == 0
+    assert torch.equal(o, ref_o) and torch.equal(l, ref_l)
+    kernel_ms, call_ms = ev[1].elapsed_time(ev[2]), ev[0].elapsed_time(ev[3])
+    assert 0.0 < kernel_ms <= call_ms
+
+
 def test_decode_all_equal_rows_and_single_token_are_exact():
     for w in (W_RUN16, W_PROD):
         d = w.dims
