@@ -154,7 +154,7 @@ __device__ __forceinline__ long append_row_base(const EpiParams& e, int n) {
 }
 
 template <typename T, int BN, bool A_MN, int MODE>
-__global__ void __launch_bounds__(192, 1)
+__global__ void __launch_bounds__(192, 2)
     k_gemm_sk(const __grid_constant__ CUtensorMap tma_a, const __grid_constant__ CUtensorMap tma_b,
               const SkParams p) {
   using C = SkCfg<BN>;

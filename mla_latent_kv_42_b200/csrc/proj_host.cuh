@@ -96,6 +96,7 @@ struct SkPlan {
 constexpr int kSkMinIters = 8;       // k blocks per CTA at least, when tiles are split
 constexpr int kSkLongTile = 16;      // tiles of at least this many k blocks are split (stream-K)
 constexpr size_t kSkSmemMax = 232448;
+constexpr size_t kSkSmemHalf = 113 * 1024;  // two CTAs per SM (228 KB per SM, 1 KB reserved per CTA)
 
 inline SkPlan plan_sk(int M, int N, int K, int batch, bool fused_epi, int d_rope) {
   SkPlan g;
@@ -122,6 +123,16 @@ inline SkPlan plan_sk(int M, int N, int K, int batch, bool fused_epi, int d_rope
   const size_t table = fused_epi ? (size_t)g.bn * (d_rope / 2) * 8 + (size_t)g.bn * 8 : 0;
   const size_t fixed = 1024 + table + 256;
   g.stages = (int)std::min<size_t>(12, (kSkSmemMax - fixed) / stage);
+  // Many short tiles (the per-head products): when a CTA's whole range fits a half-size ring,
+  // run two CTAs per SM, so that two sets of epilogue warps drain tiles side by side.
+  if (g.aligned && g.tiles > sms) {
+    const int per2 = (g.tiles + 2 * sms - 1) / (2 * sms);
+    const int need = per2 * g.kb;  // every stage of the range resident at once
+    if (need >= 2 && fixed + (size_t)need * stage <= kSkSmemHalf) {
+      g.G = (g.tiles + per2 - 1) / per2;
+      g.stages = need;
+    }
+  }
   g.smem = fixed + (size_t)g.stages * stage;
   g.part_bytes = g.split ? (size_t)(g.tiles + g.G) * 128 * g.bn * sizeof(float) : 0;
   return g;
