@@ -35,7 +35,7 @@ def up_to_date() -> bool:
     if not os.path.exists(LIB):
         return False
     t = os.path.getmtime(LIB)
-    deps = sources() + [os.path.join(INCLUDE, "mla.h"), __file__]
+    deps = sources() + [os.path.join(INCLUDE, f) for f in os.listdir(INCLUDE) if f.endswith(".h")] + [__file__]
     return all(os.path.getmtime(p) <= t for p in deps)
 
 

@@ -1,7 +1,8 @@
-// libmla — C ABI of the MLA absorbed-decode path (declared in include/mla.h).
+// libmla — C ABI of the MLA absorbed-decode path (declared in include/mla.h and include/mla_debug.h).
 // One translation unit: the kernels are included from the .cuh files beside this one.
 // Host code here validates arguments (before anything is queued), carves the caller's
 // workspace, picks kernels and launches them on the caller's stream. It allocates nothing.
+#include "mla_debug.h"
 #include <cmath>
 #include <cstring>
 #include <mutex>
@@ -415,6 +416,16 @@ const char* mla_error_string(int code) {
 }
 
 int32_t mla_last_launch_count(int32_t call) { return (call >= 0 && call < 4) ? t_launches[call] : -1; }
+
+int mla_debug_gemm_plan(int32_t M, int32_t N, int32_t K, int32_t batch, int32_t fused_rope, int32_t d_rope,
+                        int64_t* out) {
+  if (M <= 0 || N <= 0 || K <= 0 || batch <= 0 || d_rope <= 0 || out == nullptr) return MLA_ERR_INVALID_ARG;
+  const host::SkPlan g = host::plan_sk(M, N, K, batch, fused_rope != 0, d_rope);
+  const int64_t v[11] = {g.bn, g.m_tiles, g.n_tiles, g.kb, g.tiles, g.G, g.stages, g.aligned ? 1 : 0,
+                         g.split ? 1 : 0, (int64_t)g.smem, (int64_t)g.part_bytes};
+  for (int i = 0; i < 11; ++i) out[i] = v[i];
+  return MLA_OK;
+}
 
 int mla_set_decode_timing_events(mla_event_t before, mla_event_t after) {
   if ((before == nullptr) != (after == nullptr)) return MLA_ERR_INVALID_ARG;
