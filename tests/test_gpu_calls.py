@@ -262,6 +262,43 @@ def test_out_proj(fam):
     assert_parity(to64(u), ref, "u")
 
 
+@pytest.mark.parametrize("fam", ["running_bf16", "production_bf16"])
+def test_projections_beyond_one_n_tile(fam):
+    """300 tokens: the GEMMs run two n tiles of 256, with RoPE computed per element (no shared
+    table) and the append's scatter per token."""
+    w = FAMILIES[fam]
+    d = w.dims
+    W, W64 = weights64(w)
+    T = 300
+    # append: 5 sequences x 60 new tokens, crossing page boundaries, shuffled pages
+    seq_idx = np.repeat(np.arange(5), 60).astype(np.int32)
+    pos = np.concatenate([np.arange(o, o + 60) for o in (0, 40, 100, 1000, 4090)]).astype(np.int32)
+    bt, num_pages = synth.page_table(np.array([60, 100, 160, 1060, 4150]), d.page_size, "shuffled", seed=5)
+    h = synth.hidden(w, step=7, batch=T)
+    pool = torch.zeros((num_pages, d.page_size, d.D), dtype=synth.storage_dtype(d), device="cuda")
+    M.append_kv(d, h.cuda(), W["w_dkv_kr"].cuda(), torch.from_numpy(seq_idx).cuda(), torch.from_numpy(pos).cuda(),
+                torch.from_numpy(bt).cuda(), pool)
+    assert M.read_device_status() == 0
+    slots = np.array([O.page_slot(bt, s_, p_, d.page_size) for s_, p_ in zip(seq_idx, pos)])
+    got = to64(pool.view(-1, d.D)[torch.from_numpy(slots).cuda()])
+    ref = O.kv_rows(W64["w_dkv_kr"], O.as64(h), pos, d)
+    assert_parity(got[:, :d.d_c], ref[:, :d.d_c], "c^KV, 300 tokens")
+    assert_parity(got[:, d.d_c:], ref[:, d.d_c:], "k^R, 300 tokens")
+    # absorb: 300 queries at positions up to 131072
+    qpos = (np.arange(T, dtype=np.int64) * 437) % 131073
+    q = M.absorb_query(d, h.cuda(), W["w_dq"].cuda(), W["w_uq_qr"].cuda(), W["w_uk"].cuda(),
+                       torch.from_numpy(qpos.astype(np.int32)).cuda())
+    refq = O.absorb_query(W64["w_dq"], W64["w_uq_qr"], W64["w_uk"], O.as64(h), qpos.astype(np.int32), d)
+    assert_parity(to64(q)[..., :d.d_c], refq[..., :d.d_c], "q~, 300 tokens")
+    assert_parity(to64(q)[..., d.d_c:], refq[..., d.d_c:], "q^R, 300 tokens")
+    # out_proj of 300 rows
+    rng = np.random.default_rng(11)
+    o_lat = synth.to_storage(rng.standard_normal((T, d.n_heads, d.d_c), dtype=np.float32) * 0.05, d)
+    u = M.out_proj(d, o_lat.cuda(), W["w_uv"].cuda(), W["w_o"].cuda())
+    assert_parity(to64(u), O.out_proj_absorbed(W64["w_uv"], W64["w_o"], O.as64(o_lat)), "u, 300 tokens")
+    assert M.read_device_status() == 0
+
+
 # ---------------------------------------------------------------------------------------- one layer step
 def test_layer_step_running_model_fp16():
     """The pages' running model, one layer, B=1, 256 cached tokens, fp16 (positions 0..255, new at 256)."""
