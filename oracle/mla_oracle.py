@@ -23,7 +23,7 @@ Sources (page title, section or equation):
   [S2] DeepSeek-V2 paper review (velog): §2.1 latency model; §2.3 decoupled RoPE.
   [S4] DeepSeek-V2 visual explainer: 576 vs 32,768 numbers per token; the toy 512 -> 64.
 
-Readings where the pages are silent (each also listed in the design doc):
+Readings where the pages are silent:
   R1 RoPE rotates adjacent pairs (x_2k, x_2k+1) by the standard 2x2 rotation matrix.
   R2 Angle of pair k at position t is t * base^(-2k/d_h^R), formed in float64.
   R3 Positions are 0-based; cached tokens sit at 0..N-1 and the new token at N.
