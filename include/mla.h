@@ -21,6 +21,14 @@
  *   - Asynchrony: work is queued on `stream` (NULL = the legacy default stream) and the call
  *     returns without synchronising. Calls on different streams may run concurrently if their
  *     buffers (including workspaces) do not overlap.
+ *   - Overlap of consecutive kernels: every kernel is launched with programmatic dependent
+ *     launch, so it may start while the kernel queued just before it on `stream` still runs.
+ *     Each kernel waits for that predecessor to complete, with its memory visible, before it
+ *     touches activations, caches, workspaces or outputs. The one read issued earlier is the
+ *     first few k blocks of a projection's WEIGHT matrix (W^DKV, W^KR, W^DQ, W^UQ, W^QR, W^UK,
+ *     W^UV, W^O). So a kernel that writes a weight buffer must be separated from the calls that
+ *     read it by an event record on `stream` or a host synchronisation (weights loaded once and
+ *     synchronised meet this); no library call writes a weight.
  *   - Errors: calls return MLA_OK (0) or a negative mla_status. Argument checks run before
  *     anything is queued, so an error return from a check means no work was queued. A launch
  *     failure returns MLA_ERR_CUDA. Kernels never trap or assert: a bad page id or sequence
