@@ -1,4 +1,4 @@
-"""CPU fp64 oracle for Multi-head Latent Attention at decode time.
+"""CPU fp64 oracle for Multi-head Latent Attention at decode time (one or several new tokens per sequence).
 
 TEST INFRASTRUCTURE ONLY. Nothing on the product path may import, call or execute this
 package: only the tests, ``__graft_entry__.smoke()`` and the CPU-baseline / reference arm
@@ -31,6 +31,9 @@ Readings where the pages are silent:
   R5 No normalisation of the latent (none is given on [S1]).
   R6 Split-KV partials hold the normalised partial output and the log-sum-exp of the
      scaled scores (natural log); merging them is exact softmax algebra.
+  R7 A step may bring several new tokens of one sequence (the attention sum of [S1] §6 for a
+     general t): they take the consecutive positions after the prefix, all their rows are
+     cached first, and each token attends to the rows up to its own position (causal).
 
 Every function has pins in ``tests/test_oracle_pins.py``; none is "parity unpinned".
 """
@@ -43,6 +46,7 @@ __all__ = [
     "mla_cache_elems", "mha_cache_elems", "gqa_cache_elems", "gqa_equivalent_groups",
     "kv_rows", "query_path", "attention_naive", "output_naive", "layer_step_naive",
     "absorb_query", "latent_attention", "lse_merge", "out_proj_absorbed", "layer_step_absorbed",
+    "chunk_positions", "chunk_step_naive", "chunk_latent_attention", "chunk_step_absorbed",
     "page_slot", "as64",
 ]
 
@@ -268,4 +272,62 @@ def layer_step_absorbed(W: dict, h, prefix: list, dims) -> dict:
     o_lat = np.stack([o for o, _ in outs])
     lse = np.stack([l for _, l in outs])
     return {"rows": new_rows, "q": q, "o_lat": o_lat, "lse": lse,
+            "u": out_proj_absorbed(W["w_uv"], W["w_o"], o_lat)}
+
+
+# --------------------------------------------------------------------------- chunked step ([S1] §6, t general)
+def chunk_positions(prefix_lens, chunk_lens):
+    """Sequence and position of every new token of a multi-token step (R3, R7).
+
+    Sequence b holds ``prefix_lens[b]`` cached rows and brings ``chunk_lens[b]`` new tokens at
+    the positions that follow them. Tokens are listed sequence by sequence. Returns
+    (seq_idx [T], pos [T]) as int64.
+    """
+    seq_idx = np.repeat(np.arange(len(prefix_lens), dtype=np.int64), np.asarray(chunk_lens, dtype=np.int64))
+    pos = np.concatenate([n + np.arange(q, dtype=np.int64) for n, q in zip(prefix_lens, chunk_lens)]
+                         + [np.zeros(0, dtype=np.int64)])
+    return seq_idx, pos
+
+
+def chunk_step_naive(W: dict, h, prefix: list, chunk_lens, dims) -> dict:
+    """One step that brings several new tokens per sequence, in the naive form ([S1] §6).
+
+    ``h`` stacks the new tokens' hidden states in ``chunk_positions`` order. Every new row is
+    computed and appended first. The token at position t of sequence b then attends to rows
+    0..t of b: the prefix, the new tokens before it and itself (R4, R7), none after it.
+    Returns seq_idx, pos, the new rows, q^C, q^R, o and u per new token.
+    """
+    seq_idx, pos = chunk_positions([len(p) for p in prefix], chunk_lens)
+    new_rows = kv_rows(W["w_dkv_kr"], h, pos, dims)
+    _, q_c, q_r = query_path(W["w_dq"], W["w_uq_qr"], h, pos, dims)
+    full = [np.vstack([as64(prefix[b]).reshape(-1, dims.d_c + dims.d_rope), new_rows[seq_idx == b]])
+            for b in range(len(prefix))]
+    o = np.stack([attention_naive(q_c[t], q_r[t], full[seq_idx[t]][:pos[t] + 1], W["w_uk"], W["w_uv"], dims)
+                  for t in range(len(pos))])
+    return {"seq_idx": seq_idx, "pos": pos, "rows": new_rows, "q_c": q_c, "q_r": q_r, "o": o,
+            "u": output_naive(W["w_o"], o)}
+
+
+def chunk_latent_attention(q, seq_rows: list, seq_idx, pos, dims):
+    """Absorbed attention for the new tokens of a multi-token step ([S1] §5.3 steps 2-3 for
+    every new token of §6): token t attends to rows 0..pos[t] of sequence seq_idx[t] (R7).
+
+    ``q`` [T, n_h, D]; ``seq_rows[b]`` holds at least pos[t] + 1 rows [., D] of sequence b.
+    Returns (o_lat [T, n_h, d_c], lse [T, n_h]).
+    """
+    outs = [latent_attention(q[t], as64(seq_rows[seq_idx[t]])[:pos[t] + 1], dims) for t in range(len(pos))]
+    if not outs:
+        return np.zeros((0, dims.n_heads, dims.d_c)), np.zeros((0, dims.n_heads))
+    return np.stack([o for o, _ in outs]), np.stack([l for _, l in outs])
+
+
+def chunk_step_absorbed(W: dict, h, prefix: list, chunk_lens, dims) -> dict:
+    """The same multi-token step as ``chunk_step_naive`` through the absorbed route ([S1] §5.3)."""
+    seq_idx, pos = chunk_positions([len(p) for p in prefix], chunk_lens)
+    new_rows = kv_rows(W["w_dkv_kr"], h, pos, dims)
+    q = absorb_query(W["w_dq"], W["w_uq_qr"], W["w_uk"], h, pos, dims)
+    full = [np.vstack([as64(prefix[b]).reshape(-1, dims.d_c + dims.d_rope), new_rows[seq_idx == b]])
+            for b in range(len(prefix))]
+    o_lat, lse = chunk_latent_attention(q, full, seq_idx, pos, dims)
+    return {"seq_idx": seq_idx, "pos": pos, "rows": new_rows, "q": q, "o_lat": o_lat, "lse": lse,
             "u": out_proj_absorbed(W["w_uv"], W["w_o"], o_lat)}

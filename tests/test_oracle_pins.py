@@ -441,3 +441,95 @@ def test_pins_catch_planted_mistakes():
     o_lat, _ = O.latent_attention(q_abs[0], rows, dims)
     u_bad = O.out_proj_absorbed(W["w_uv"], W["w_o"], o_lat[None])
     assert np.abs(u_bad - good["u"]).max() > 1e-6 * np.abs(good["u"]).max()
+
+
+# ----------------------------------------------------------------------------- multi-token step
+CHUNK_CASES = [([0, 3, 5], [4, 1, 3]), ([2], [6]), ([0], [1]), ([7, 0], [0, 2])]
+
+
+@pytest.mark.parametrize("dims", [TINY, RUNNING], ids=["tiny", "running"])
+@pytest.mark.parametrize("prefix_lens,chunk_lens", CHUNK_CASES)
+def test_chunk_equals_one_token_at_a_time(dims, prefix_lens, chunk_lens):
+    """§6 with a general t: a step that brings q tokens of a sequence at once gives each of them
+    what q single-token decode steps give, taken in position order, each appending its own row
+    before it attends (causal: a token never sees a later one)."""
+    rng = np.random.default_rng(21)
+    W = rand_weights(dims, rng, scale=0.5)
+    prefix = [rng.standard_normal((n, dims.D)) for n in prefix_lens]
+    seq_idx, pos = O.chunk_positions(prefix_lens, chunk_lens)
+    h = rng.standard_normal((len(pos), dims.d_model))
+    got = O.chunk_step_naive(W, h, prefix, chunk_lens, dims)
+    grown = [p.copy() for p in prefix]
+    for t in range(len(pos)):
+        b = int(seq_idx[t])
+        assert pos[t] == len(grown[b])
+        one = O.layer_step_naive(W, h[t:t + 1], [grown[b]], dims)
+        np.testing.assert_allclose(got["rows"][t], one["rows"][0], rtol=1e-12, atol=1e-14)
+        # fp64 roundoff only: the two routes multiply matrices of different shapes
+        np.testing.assert_allclose(got["o"][t], one["o"][0], rtol=0, atol=1e-10 * np.abs(one["o"]).max())
+        np.testing.assert_allclose(got["u"][t], one["u"][0], rtol=0, atol=1e-10 * np.abs(one["u"]).max())
+        grown[b] = np.vstack([grown[b], one["rows"]])
+
+
+@pytest.mark.parametrize("dims", [TINY, RUNNING], ids=["tiny", "running"])
+def test_chunk_absorbed_equals_naive(dims):
+    """§5.1-§5.3 hold token by token, so the absorbed multi-token step equals the naive one."""
+    rng = np.random.default_rng(22)
+    W = rand_weights(dims, rng, scale=0.5)
+    prefix_lens, chunk_lens = [0, 3, 5], [4, 1, 3]
+    prefix = [rng.standard_normal((n, dims.D)) for n in prefix_lens]
+    h = rng.standard_normal((sum(chunk_lens), dims.d_model))
+    naive = O.chunk_step_naive(W, h, prefix, chunk_lens, dims)
+    absorbed = O.chunk_step_absorbed(W, h, prefix, chunk_lens, dims)
+    np.testing.assert_array_equal(naive["pos"], absorbed["pos"])
+    np.testing.assert_allclose(absorbed["u"], naive["u"], rtol=1e-10, atol=1e-12 * np.abs(naive["u"]).max())
+
+
+def test_chunk_attention_equals_library_sdpa_with_a_causal_mask():
+    """torch's scaled_dot_product_attention with a boolean mask that admits key j for query t
+    exactly when j <= pos[t] gives the absorbed chunk attention (values = the latents)."""
+    dims = RUNNING
+    rng = np.random.default_rng(23)
+    L, q_len = 29, 6
+    rows = rng.standard_normal((L, dims.D))
+    pos = np.arange(L - q_len, L)
+    q = rng.standard_normal((q_len, dims.n_heads, dims.D)) * 0.3
+    o_lat, _ = O.chunk_latent_attention(q, [rows], np.zeros(q_len, dtype=np.int64), pos, dims)
+    mask = torch.from_numpy(np.arange(L)[None, :] <= pos[:, None])
+    t = lambda a: torch.from_numpy(np.ascontiguousarray(a))
+    ref = torch.nn.functional.scaled_dot_product_attention(
+        t(q.transpose(1, 0, 2)), t(rows)[None], t(rows[:, :dims.d_c])[None], attn_mask=mask,
+        scale=1.0 / math.sqrt(dims.d_head + dims.d_rope)).numpy().transpose(1, 0, 2)
+    np.testing.assert_allclose(o_lat, ref, rtol=1e-11, atol=1e-13)
+
+
+def test_chunk_first_token_of_an_empty_sequence_sees_only_itself():
+    """At position 0 the softmax runs over one row, so o_lat is that token's own latent and the
+    log-sum-exp its own scaled score (§4.4 with a single term)."""
+    dims = RUNNING
+    rng = np.random.default_rng(24)
+    W = rand_weights(dims, rng, scale=0.5)
+    h = rng.standard_normal((3, dims.d_model))
+    out = O.chunk_step_absorbed(W, h, [np.zeros((0, dims.D))], [3], dims)
+    np.testing.assert_allclose(out["o_lat"][0], np.broadcast_to(out["rows"][0, :dims.d_c], (dims.n_heads, dims.d_c)),
+                               rtol=1e-13, atol=1e-14)
+    s0 = out["q"][0] @ out["rows"][0] / math.sqrt(dims.d_head + dims.d_rope)
+    np.testing.assert_allclose(out["lse"][0], s0, rtol=1e-12, atol=1e-14)
+
+
+def test_chunk_pins_catch_a_causal_off_by_one():
+    """An attention bound one row short (the token misses itself) or one row long (it sees the
+    next token) breaks the token-at-a-time pin; the correct bound passes it."""
+    dims = RUNNING
+    rng = np.random.default_rng(25)
+    W = rand_weights(dims, rng, scale=0.5)
+    prefix = [rng.standard_normal((4, dims.D))]
+    h = rng.standard_normal((3, dims.d_model))
+    good = O.chunk_step_absorbed(W, h, prefix, [3], dims)
+    full = np.vstack([prefix[0], good["rows"]])
+    seq0 = np.zeros(3, dtype=np.int64)
+    step = O.layer_step_absorbed(W, h[1:2], [full[:5]], dims)     # the middle token, decoded alone
+    for shift, ok in ((0, True), (-1, False), (1, False)):
+        o_lat, _ = O.chunk_latent_attention(good["q"], [full], seq0, good["pos"] + shift, dims)
+        err = np.abs(o_lat[1] - step["o_lat"][0]).max()
+        assert (err < 1e-12) if ok else (err > 1e-6)
