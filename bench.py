@@ -5,7 +5,9 @@
 
 A step is one pass of the whole hot path over one batch: append the new token's latent row,
 absorb the query, latent attention over every cached token, output projection (for the
-12-layer running-model workload: all 12 layers). Inputs (weights, caches, new hidden states)
+12-layer running-model workload: all 12 layers). A workload whose sequences each bring a chunk
+of several new tokens (``chunk`` > 1, e.g. production_b8_n4096_chunk128_bf16) runs the same
+step for all of them with causal mla_prefill_attention in place of mla_decode_attention. Inputs (weights, caches, new hidden states)
 are seeded synthetic data resident in HBM before timing. With N > 1 (torchrun, one process per
 GPU) every rank runs its own replica of the workload: sequences are independent, so there is no
 data-path collective; ``value`` aggregates the ranks and the time is the max over ranks.
@@ -13,7 +15,7 @@ data-path collective; ``value`` aggregates the ranks and the time is the max ove
 One JSON line on rank 0. ``value`` is µs per layer-step of the whole job (step time divided by
 layers and by N). ``e2e`` is the same metric with host buffers: the step's inputs copied from
 pinned host memory and its output copied back inside the timed region. ``roofline`` reports
-the dominant call, mla_decode_attention, against max(bytes / HBM, flops / tensor peak) with the
+the dominant call, the attention call, against max(bytes / HBM, flops / tensor peak) with the
 measured peaks. ``cpu_baseline`` times the fp64 oracle on a bounded sample (rank 0, N = 1).
 """
 from __future__ import annotations
@@ -111,7 +113,9 @@ class ClockSampler:
 
 # ----------------------------------------------------------------------------------- CPU oracle
 class OracleSample:
-    """A bounded sample of the workload for the fp64 oracle: the first ``n`` sequences of one layer."""
+    """A bounded sample of the workload for the fp64 oracle, one layer: the first ``n`` sequences
+    of a decode step, or the first ``n`` new tokens of sequence 0 of a multi-token step. ``frac``
+    is the sample's share of the step's attended tokens (the oracle's cost is linear in them)."""
 
     def __init__(self, w, n, layer=0):
         import oracle as O
@@ -119,35 +123,49 @@ class OracleSample:
         self.O, self.w = O, w
         self.cached = synth.cached_lengths(w)
         self.W64 = {k: O.as64(v) for k, v in synth.weights(w, layer).items()}
-        self.picks = list(range(min(n, w.batch)))
-        sub = self.cached[self.picks]
+        c = w.chunk
+        total = float(np.sum(c * (self.cached + 1) + c * (c - 1) // 2))
+        if c == 1:
+            self.picks = list(range(min(n, w.batch)))
+            self.k = len(self.picks)
+            sub = self.cached[self.picks]
+            self.attended = int(np.sum(sub + 1))
+            self.h = O.as64(synth.hidden(w))[self.picks]
+            self.what = f"{self.k} of {w.batch} sequences"
+        else:
+            self.picks = [0]
+            self.k = min(n, c)
+            sub = self.cached[:1]
+            self.attended = int(sum(int(sub[0]) + i + 1 for i in range(self.k)))
+            self.h = O.as64(synth.hidden(w, batch=w.batch * c))[:self.k]
+            self.what = f"the first {self.k} of {c} new tokens of sequence 0 of {w.batch}"
         rows = synth.prefix_rows(w, sub, layer=layer, device="cpu")
         offs = np.concatenate([[0], np.cumsum(sub)])
-        self.prefix = [O.as64(rows[offs[i]:offs[i + 1]]) for i in range(len(self.picks))]
-        self.h = O.as64(synth.hidden(w))[self.picks]
-        self.frac = float(np.sum(sub + 1)) / float(np.sum(self.cached + 1))
+        self.prefix = [O.as64(rows[offs[i]:offs[i + 1]]) for i in range(len(sub))]
+        self.frac = self.attended / total
 
-    def run(self, n=None):
-        """Seconds for the naive oracle's layer-step over the first ``n`` sampled sequences."""
-        k = len(self.picks) if n is None else n
+    def run(self):
+        """Seconds for the naive oracle over the sample."""
         t = time.perf_counter()
-        self.O.layer_step_naive(self.W64, self.h[:k], self.prefix[:k], self.w.dims)
+        if self.w.chunk == 1:
+            self.O.layer_step_naive(self.W64, self.h, self.prefix, self.w.dims)
+        else:
+            self.O.chunk_step_naive(self.W64, self.h, self.prefix, [self.k], self.w.dims)
         return time.perf_counter() - t
 
 
 def cpu_baseline(w, target_s=12.0):
-    """Time the naive oracle on a bounded sample of whole sequences; extrapolate to the step."""
+    """Time the naive oracle on a bounded sample (whole sequences, or the first new tokens of
+    one sequence for a multi-token step); extrapolate to the step by attended tokens."""
     probe = OracleSample(w, 1)
     t1 = probe.run()
-    n = max(1, min(w.batch, int(target_s / max(t1, 1e-3))))
+    n = max(1, min(w.batch if w.chunk == 1 else w.chunk, int(target_s / max(t1, 1e-3))))
     smp = OracleSample(w, n)
     t = smp.run()
     cores = len(os.sched_getaffinity(0))
-    attended = int(np.sum(smp.cached[smp.picks] + 1))
     return {"value": t / smp.frac * 1e6, "unit": UNIT, "cores": cores, "kind": "oracle",
-            "sample": (f"naive fp64 oracle, one layer, {len(smp.picks)} of {w.batch} sequences (all heads, "
-                       f"{attended} attended tokens), extrapolated by attended tokens x{1 / smp.frac:.1f}; "
-                       f"{t:.1f} s of CPU time")}
+            "sample": (f"naive fp64 oracle, one layer, {smp.what} (all heads, {smp.attended} attended tokens), "
+                       f"extrapolated by attended tokens x{1 / smp.frac:.1f}; {t:.1f} s of CPU time")}
 
 
 def run_reference(args):
@@ -158,7 +176,6 @@ def run_reference(args):
     from mla_latent_kv_42_b200 import synth
     w = synth.workload(args.workload)
     smp = OracleSample(w, 1)
-    cached = smp.cached
     per = []
     for i in range(args.warmup + args.steps):
         t = smp.run()
@@ -166,8 +183,8 @@ def run_reference(args):
             per.append(t / smp.frac)
     us = float(np.mean(per)) * 1e6
     cores = len(os.sched_getaffinity(0))
-    sample = (f"naive fp64 oracle on sequence 0 of {w.batch} each step (all heads, {int(cached[0]) + 1} attended "
-              f"tokens), extrapolated by attended tokens to the whole batch")
+    sample = (f"naive fp64 oracle on {smp.what} each step (all heads, {smp.attended} attended tokens), "
+              f"extrapolated by attended tokens to the whole step")
     line = {
         "impl": "reference", "metric": METRIC, "value": us, "unit": UNIT, "n_gpus": args.gpus, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": us * w.layers / 1e3, "higher_is_better": False, "scaling": "weak",
@@ -247,17 +264,24 @@ def run_mla(args):
     w = rank_workload(synth.workload(args.workload), rank)
     d = w.dims
     cached = synth.cached_lengths(w)
-    ix = harness.step_index(cached, device=dev)
-    layers = [harness.make_layer(w, cached, layer=l, device=dev) for l in range(w.layers)]
+    chunk = w.chunk                  # new tokens per sequence per step; > 1 runs mla_prefill_attention
+    ix = harness.step_index(cached, device=dev, chunk=chunk)
+    layers = [harness.make_layer(w, cached, layer=l, device=dev, spare_tokens=chunk) for l in range(w.layers)]
     B = w.batch
-    h0 = synth.hidden(w).to(dev)
+    T = B * chunk                    # new tokens per step
+    h0 = synth.hidden(w, batch=T).to(dev)
     h = h0.clone()
-    ws = torch.empty(M.step_workspace_bytes(d, B, ix.max_seq_len), dtype=torch.uint8, device=dev)
+    attn_call = M.CALL_PREFILL_ATTENTION if chunk > 1 else M.CALL_DECODE_ATTENTION
+    calls = (M.CALL_APPEND_KV, M.CALL_ABSORB_QUERY, attn_call, M.CALL_OUT_PROJ)
+    ws = torch.empty(max(M.workspace_size(d, c, T, ix.max_seq_len) for c in calls), dtype=torch.uint8, device=dev)
+    # per-step index input besides the positions: the attended lengths (decode) or each new
+    # token's sequence (prefill)
+    aux0 = ix.seq_idx if chunk > 1 else ix.seq_lens
     e = synth.storage_dtype(d)
-    outs = [{"q": torch.empty((B, d.n_heads, d.D), dtype=e, device=dev),
-             "o_lat": torch.empty((B, d.n_heads, d.d_c), dtype=e, device=dev),
-             "lse": torch.empty((B, d.n_heads), dtype=torch.float32, device=dev),
-             "u": torch.empty((B, d.d_model), dtype=e, device=dev)} for _ in layers]
+    outs = [{"q": torch.empty((T, d.n_heads, d.D), dtype=e, device=dev),
+             "o_lat": torch.empty((T, d.n_heads, d.d_c), dtype=e, device=dev),
+             "lse": torch.empty((T, d.n_heads), dtype=torch.float32, device=dev),
+             "u": torch.empty((T, d.d_model), dtype=e, device=dev)} for _ in layers]
     stream = torch.cuda.current_stream(dev)
     EV = lambda: torch.cuda.Event(enable_timing=True)
     call_ms = np.zeros(4)
@@ -265,13 +289,14 @@ def run_mla(args):
     kernel_events = []
 
     def one_step(record=False, inp=None, outs_=None):
-        x, pos, lens = inp if inp is not None else (h, ix.pos, ix.seq_lens)
+        x, pos, aux = inp if inp is not None else (h, ix.pos, aux0)
+        seq_idx = aux if chunk > 1 else ix.seq_idx
         for L, o in zip(layers, outs if outs_ is None else outs_):
             st, w_ = L.state, L.state.w
             if record:
                 ev = [EV() for _ in range(5)]
                 ev[0].record(stream)
-            M.append_kv(d, x, w_["w_dkv_kr"], ix.seq_idx, pos, st.block_table, st.pool, ws=ws, stream=stream)
+            M.append_kv(d, x, w_["w_dkv_kr"], seq_idx, pos, st.block_table, st.pool, ws=ws, stream=stream)
             n = M.last_launch_count(0)
             if record:
                 ev[1].record(stream)
@@ -284,12 +309,16 @@ def run_mla(args):
                 for x_ in kev:
                     x_.record(stream)
                 M.set_decode_timing_events(kev[0], kev[1])
-            M.decode_attention(d, o["q"], st.pool, st.block_table, lens, ix.max_seq_len, o_lat=o["o_lat"],
-                               lse=o["lse"], ws=ws, stream=stream)
+            if chunk > 1:
+                M.prefill_attention(d, o["q"], st.pool, st.block_table, seq_idx, pos, ix.max_seq_len,
+                                    o_lat=o["o_lat"], lse=o["lse"], ws=ws, stream=stream)
+            else:
+                M.decode_attention(d, o["q"], st.pool, st.block_table, aux, ix.max_seq_len, o_lat=o["o_lat"],
+                                   lse=o["lse"], ws=ws, stream=stream)
             if record:
                 M.set_decode_timing_events(None, None)
                 kernel_events.append(kev)
-            n += M.last_launch_count(2)
+            n += M.last_launch_count(attn_call)
             if record:
                 ev[3].record(stream)
             M.out_proj(d, o["o_lat"], w_["w_uv"], w_["w_o"], u=o["u"], ws=ws, stream=stream)
@@ -353,8 +382,8 @@ def run_mla(args):
     # ---- e2e: host buffers through the public API (pinned h in, u out, inside the timed region)
     h_host = h0.cpu().pin_memory()
     pos_host = ix.pos.cpu().pin_memory()
-    lens_host = ix.seq_lens.cpu().pin_memory()
-    u_host = torch.empty((B, d.d_model), dtype=e).pin_memory()
+    aux_host = aux0.cpu().pin_memory()
+    u_host = torch.empty((T, d.d_model), dtype=e).pin_memory()
     if world > 1:
         dist.barrier()
     # Pipelined as a serving loop would run it: step k+1's inputs go up on a copy stream and
@@ -363,7 +392,7 @@ def run_mla(args):
     # outputs (a set is rewritten once its read-back has finished). Every step's copies lie
     # inside the timed region, which spans both streams.
     copy_stream = torch.cuda.Stream(dev)
-    ins = [(torch.empty_like(h), torch.empty_like(ix.pos), torch.empty_like(ix.seq_lens)) for _ in range(2)]
+    ins = [(torch.empty_like(h), torch.empty_like(ix.pos), torch.empty_like(aux0)) for _ in range(2)]
     outs_pp = [outs, [{k: torch.empty_like(v) for k, v in o.items()} for o in outs]]
     ev_in = [torch.cuda.Event() for _ in range(2)]
     ev_done = [torch.cuda.Event() for _ in range(2)]
@@ -380,7 +409,7 @@ def run_mla(args):
             hb, pb, lb = ins[k % 2]
             hb.copy_(h_host, non_blocking=True)
             pb.copy_(pos_host, non_blocking=True)
-            lb.copy_(lens_host, non_blocking=True)
+            lb.copy_(aux_host, non_blocking=True)
             ev_in[k % 2].record(copy_stream)
 
     upload(0)
@@ -414,9 +443,8 @@ def run_mla(args):
         ms_step = ms_total / args.steps
         us_layer_job = job_us_per_layer_step(ms_total, args.steps, len(layers), world)
         us_e2e_job = job_us_per_layer_step(ms_e2e, args.steps, len(layers), world)
-        seq_lens = cached + 1
-        dbytes, dflops = harness.decode_work(d, seq_lens)
-        sbytes, sflops = harness.step_work(d, seq_lens)
+        dbytes, dflops = harness.attention_work(d, cached, chunk)
+        sbytes, sflops = harness.layer_work(d, cached, chunk)
         dec_s = decode_ms * 1e-3    # the whole call: planner + attention kernel + merge
         ker_s = kernel_ms * 1e-3    # the attention kernel alone (events around its launch)
         t_mem = dbytes / (peaks["hbm_gbs"] * 1e9)
@@ -431,7 +459,9 @@ def run_mla(args):
         roof["frac"] = roof["achieved"] / roof["peak"]
         roof["frac_whole_call"] = call_frac  # counting the planner and merge launches too
         roof["traffic"] = measured_decode_traffic(w.name)
-        roof["kernel"] = "attention kernel of mla_decode_attention (k_decode_tc; CUDA-core k_decode_simt at small n_h)"
+        roof["kernel"] = ("attention kernel of mla_prefill_attention (k_decode_tc, one item per new token)" if chunk > 1
+                          else "attention kernel of mla_decode_attention (k_decode_tc; CUDA-core k_decode_simt at "
+                               "small n_h)")
         roof["kernel_us"] = kernel_ms * 1e3
         roof["peak_source"] = peak_src + " (burst; MEASURED_PEAKS.json)" if peak_src == "measured" else peak_src
         roof["roofline_us"] = max(t_mem, t_flop) * 1e6
@@ -446,6 +476,7 @@ def run_mla(args):
                                                                          f"U[{w.cached[0]},{w.cached[1]}], sum "
                                                                          f"{int(cached.sum())}"),
                        "layers": len(layers), "dims": dims_desc(d), "paging": w.paging,
+                       **({"chunk": chunk, "new_tokens": T} if chunk > 1 else {}),
                        "l2": "inputs larger than L2" if sbytes > 126e6 else "L2 not flushed (inputs below L2)",
                        "parallelism": f"replicas x{world} (sequence-independent, no collective)"},
             "tflops": sflops / step_s / 1e12,
@@ -453,12 +484,14 @@ def run_mla(args):
             "decode_us": decode_ms * 1e3,
             "decode_kernel_us": kernel_ms * 1e3,
             "per_call_us": {"append_kv": call_ms[0] * 1e3, "absorb_query": call_ms[1] * 1e3,
-                            "decode_attention": call_ms[2] * 1e3, "out_proj": call_ms[3] * 1e3},
+                            ("prefill_attention" if chunk > 1 else "decode_attention"): call_ms[2] * 1e3,
+                            "out_proj": call_ms[3] * 1e3},
             "layer_step_roofline_us": max(sbytes / (peaks["hbm_gbs"] * 1e9), sflops / (peaks["bf16_tflops"] * 1e12))
             * 1e6,
             "roofline": roof,
-            "e2e": {"value": us_e2e_job, "unit": UNIT, "h2d_bytes_per_step": int(h0.numel() * 2 + 2 * B * 4),
-                    "d2h_bytes_per_step": int(B * d.d_model * 2)},
+            "e2e": {"value": us_e2e_job, "unit": UNIT,
+                    "h2d_bytes_per_step": int(h0.numel() * 2 + ix.pos.numel() * 4 + aux0.numel() * 4),
+                    "d2h_bytes_per_step": int(T * d.d_model * 2)},
             "gpu_launches": int(gpu_launches),
             "clocks": sampler.summary(t_wall0 - 0.1, t_wall1 + 0.1),
         }

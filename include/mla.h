@@ -79,7 +79,8 @@ enum mla_call {
   MLA_CALL_APPEND_KV = 0,
   MLA_CALL_ABSORB_QUERY = 1,
   MLA_CALL_DECODE_ATTENTION = 2,
-  MLA_CALL_OUT_PROJ = 3
+  MLA_CALL_OUT_PROJ = 3,
+  MLA_CALL_PREFILL_ATTENTION = 4
 };
 
 /* Returns MLA_OK if every call supports `dims`, else MLA_ERR_UNSUPPORTED_DIMS or
@@ -92,8 +93,9 @@ int mla_check_dims(const mla_dims* dims);
  * §4.5; 160 for the running model, 576 at DeepSeek-V2 dims). Negative on invalid dims. */
 int32_t mla_cache_elems_per_token(const mla_dims* dims);
 
-/* Bytes of workspace the call `call` needs for batch B (tokens T for append) and longest
- * attended length max_seq_len, on the current device. 0 on invalid arguments. */
+/* Bytes of workspace the call `call` needs for batch B (new tokens T for append and prefill
+ * attention) and longest attended length max_seq_len, on the current device. 0 on invalid
+ * arguments. */
 size_t mla_workspace_size(const mla_dims* dims, int32_t call, int32_t B, int32_t max_seq_len);
 
 /*
@@ -148,6 +150,32 @@ int mla_decode_attention(const mla_dims* dims, const void* q, const void* pool, 
                          const int32_t* block_table, int32_t max_pages, const int32_t* seq_lens,
                          int32_t B, int32_t max_seq_len, void* o_lat, float* lse_out,
                          void* ws, size_t ws_bytes, mla_stream_t stream);
+
+/*
+ * mla_prefill_attention — latent attention for a step that brings several new tokens per
+ * sequence (chunked prefill), causal (from-scratch page §6: the attention sum of the token at
+ * position t runs over the cached positions j <= t; §5.3 steps 2-3 for each new token).
+ * For every new token t and head i, over j = 0 .. pos[t] of sequence seq_idx[t]:
+ *   s_j = (q~_i . c_j + q^R_i . k^R_j) / sqrt(d_head + d_rope);  p = softmax_j(s)
+ *   o_lat[t][i] = sum_j p_j c_j;   lse_out[t][i] = log sum_j exp(s_j)   (skipped if NULL)
+ * So a token sees its sequence's prefix, the new tokens before it and itself, and no later
+ * token. Every new token's cache row must already be written (mla_append_kv with the same
+ * seq_idx and pos), and q is mla_absorb_query's output for the same tokens and positions.
+ * q [T, n_heads, d_c + d_rope]; seq_idx int32 [T] in [0, num_seqs); pos int32 [T] in
+ * [0, max_seq_len); block_table int32 [num_seqs, max_pages] and pool as in mla_append_kv,
+ * max_pages * page_size >= max_seq_len; o_lat [T, n_heads, d_c] element type; lse_out float
+ * [T, n_heads] or NULL; ws at least mla_workspace_size(dims, MLA_CALL_PREFILL_ATTENTION, T,
+ * max_seq_len) bytes. Tokens may come in any order; each is computed on its own, with the
+ * arithmetic of mla_decode_attention for a sequence of length pos[t] + 1 (where split-KV
+ * boundaries fall may differ, so agreement is to rounding). The result is bitwise
+ * reproducible run to run. A token with an out-of-range seq_idx or pos gets a zero
+ * output (lse -inf) and records MLA_ERR_BAD_SEQ_LEN in the device status; a bad page id
+ * records MLA_ERR_BAD_PAGE. T == 0 is a no-op.
+ */
+int mla_prefill_attention(const mla_dims* dims, const void* q, const void* pool, int32_t num_pages,
+                          const int32_t* block_table, int32_t num_seqs, int32_t max_pages,
+                          const int32_t* seq_idx, const int32_t* pos, int32_t T, int32_t max_seq_len,
+                          void* o_lat, float* lse_out, void* ws, size_t ws_bytes, mla_stream_t stream);
 
 /*
  * mla_out_proj — output projection with W^UV absorbed (from-scratch page §5.2, step 4 of

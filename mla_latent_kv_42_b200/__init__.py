@@ -16,11 +16,12 @@ from dataclasses import dataclass
 
 __all__ = [
     "MLAError", "load_library", "library_path", "c_dims", "workspace_size", "cache_elems_per_token",
-    "append_kv", "absorb_query", "decode_attention", "decode_attention_noalloc", "out_proj", "read_device_status", "last_launch_count",
-    "LayerState", "layer_step", "CALL_APPEND_KV", "CALL_ABSORB_QUERY", "CALL_DECODE_ATTENTION", "CALL_OUT_PROJ",
+    "append_kv", "absorb_query", "decode_attention", "decode_attention_noalloc", "prefill_attention", "out_proj",
+    "read_device_status", "last_launch_count", "LayerState", "layer_step",
+    "CALL_APPEND_KV", "CALL_ABSORB_QUERY", "CALL_DECODE_ATTENTION", "CALL_OUT_PROJ", "CALL_PREFILL_ATTENTION",
 ]
 
-CALL_APPEND_KV, CALL_ABSORB_QUERY, CALL_DECODE_ATTENTION, CALL_OUT_PROJ = 0, 1, 2, 3
+CALL_APPEND_KV, CALL_ABSORB_QUERY, CALL_DECODE_ATTENTION, CALL_OUT_PROJ, CALL_PREFILL_ATTENTION = 0, 1, 2, 3, 4
 _PKG = os.path.dirname(os.path.abspath(__file__))
 
 
@@ -49,6 +50,8 @@ _SIGS = {
     "mla_append_kv": (ctypes.c_int, [_P, _P, _P, _P, _P, _P, _I32, _I32, _P, _I32, _I32, _P, _SZ, _P]),
     "mla_absorb_query": (ctypes.c_int, [_P, _P, _P, _P, _P, _P, _P, _I32, _P, _SZ, _P]),
     "mla_decode_attention": (ctypes.c_int, [_P, _P, _P, _I32, _P, _I32, _P, _I32, _I32, _P, _P, _P, _SZ, _P]),
+    "mla_prefill_attention": (ctypes.c_int, [_P, _P, _P, _I32, _P, _I32, _I32, _P, _P, _I32, _I32, _P, _P, _P, _SZ,
+                                             _P]),
     "mla_out_proj": (ctypes.c_int, [_P, _P, _P, _P, _P, _I32, _P, _SZ, _P]),
     "mla_read_device_status": (ctypes.c_int, [_P, ctypes.POINTER(_I32)]),
     "mla_error_string": (ctypes.c_char_p, [ctypes.c_int]),
@@ -187,6 +190,35 @@ def decode_attention(dims, q, pool, block_table, seq_lens, max_seq_len, o_lat=No
     _check(_lib().mla_decode_attention(ctypes.byref(cd), _ptr(q), _ptr(pool), pool.shape[0], _ptr(block_table),
                                        block_table.shape[1], _ptr(seq_lens), B, int(max_seq_len), _ptr(o_lat),
                                        _ptr(lse), _ptr(ws), nbytes, _stream(stream)), "mla_decode_attention")
+    return o_lat, lse
+
+
+def prefill_attention(dims, q, pool, block_table, seq_idx, pos, max_seq_len, o_lat=None, lse=None, want_lse=True,
+                      ws=None, stream=None):
+    """mla_prefill_attention: causal latent attention of several new tokens per sequence.
+
+    Token t (sequence ``seq_idx[t]``, position ``pos[t]``) attends to its sequence's cached
+    positions 0..pos[t]; the new tokens' rows must already be appended.
+    """
+    import torch
+    e = _elem(dims)
+    for t, n, dt in ((q, "q", e), (pool, "pool", e), (block_table, "block_table", torch.int32),
+                     (seq_idx, "seq_idx", torch.int32), (pos, "pos", torch.int32)):
+        _need(t, dt, n)
+    T = q.shape[0]
+    if o_lat is None:
+        o_lat = torch.empty((T, dims.n_heads, dims.d_c), dtype=e, device=q.device)
+    if lse is None and want_lse:
+        lse = torch.empty((T, dims.n_heads), dtype=torch.float32, device=q.device)
+    _need(o_lat, e, "o_lat")
+    if lse is not None:
+        _need(lse, torch.float32, "lse")
+    ws, nbytes = _ws(dims, CALL_PREFILL_ATTENTION, T, max_seq_len, ws, q.device)
+    cd = c_dims(dims)
+    _check(_lib().mla_prefill_attention(ctypes.byref(cd), _ptr(q), _ptr(pool), pool.shape[0], _ptr(block_table),
+                                        block_table.shape[0], block_table.shape[1], _ptr(seq_idx), _ptr(pos), T,
+                                        int(max_seq_len), _ptr(o_lat), _ptr(lse), _ptr(ws), nbytes,
+                                        _stream(stream)), "mla_prefill_attention")
     return o_lat, lse
 
 

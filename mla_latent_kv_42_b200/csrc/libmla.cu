@@ -10,13 +10,14 @@
 #include "common.cuh"
 #include "decode_simt.cuh"
 #include "decode_tc.cuh"
+#include "prefill.cuh"
 #include "proj_host.cuh"
 
 using namespace mla;
 
 namespace {
 
-thread_local int32_t t_launches[4] = {0, 0, 0, 0};
+thread_local int32_t t_launches[5] = {0, 0, 0, 0, 0};
 // Profiling hook: events recorded around the attention kernel of this thread's decode calls.
 thread_local cudaEvent_t t_ev_before = nullptr, t_ev_after = nullptr;
 inline void mark_before(cudaStream_t st) {
@@ -183,7 +184,7 @@ size_t ws_decode(const mla_dims* d, int B, int max_seq_len) {
 template <typename T>
 int decode_tc_impl(const mla_dims* d, const void* q, const void* pool, int32_t num_pages, const int32_t* bt,
                    int32_t max_pages, const int32_t* seq_lens, int32_t B, int32_t max_seq_len, void* o_lat,
-                   float* lse_out, void* ws, cudaStream_t st) {
+                   float* lse_out, void* ws, cudaStream_t st, int32_t& launches) {
   const int C = decode_clusters();
   if (!decode_tc_set_smem<T>()) return MLA_ERR_CUDA;
   Carve c{static_cast<char*>(ws)};
@@ -219,7 +220,8 @@ int decode_tc_impl(const mla_dims* d, const void* q, const void* pool, int32_t n
                  static_cast<const int*>(prefix), (int)B, C, (int)d->n_heads, static_cast<T*>(o_lat),
                  lse_out) != cudaSuccess)
     return MLA_ERR_CUDA;
-  return finish_launches(MLA_CALL_DECODE_ATTENTION, 3);
+  launches += 3;
+  return MLA_OK;
 }
 
 template <typename T, int NPAIR>
@@ -239,9 +241,10 @@ void launch_decode_simt(const mla_dims* d, const DecodePlan& p, const void* q, c
 template <typename T>
 int decode_impl(const mla_dims* d, const void* q, const void* pool, int32_t num_pages, const int32_t* bt,
                 int32_t max_pages, const int32_t* seq_lens, int32_t B, int32_t max_seq_len, void* o_lat,
-                float* lse_out, void* ws, cudaStream_t st) {
+                float* lse_out, void* ws, cudaStream_t st, int32_t& launches) {
   if (decode_tc_eligible(d))
-    return decode_tc_impl<T>(d, q, pool, num_pages, bt, max_pages, seq_lens, B, max_seq_len, o_lat, lse_out, ws, st);
+    return decode_tc_impl<T>(d, q, pool, num_pages, bt, max_pages, seq_lens, B, max_seq_len, o_lat, lse_out, ws, st,
+                             launches);
   const DecodePlan p = plan_decode(d, B, max_seq_len);
   const size_t bh = (size_t)B * d->n_heads;
   float* o_part = nullptr;
@@ -252,7 +255,7 @@ int decode_impl(const mla_dims* d, const void* q, const void* pool, int32_t num_
     lse_part = c.take<float>(bh * p.n_splits);
   }
   const int D = d->d_c + d->d_rope;
-  int32_t n = 0;
+  int32_t& n = launches;
   if (D <= 192)
     launch_decode_simt<T, 3>(d, p, q, pool, num_pages, bt, max_pages, seq_lens, B, max_seq_len, o_lat, lse_out,
                              o_part, lse_part, st);
@@ -268,7 +271,51 @@ int decode_impl(const mla_dims* d, const void* q, const void* pool, int32_t num_
                                                  lse_out);
     ++n;
   }
-  return finish_launches(MLA_CALL_DECODE_ATTENTION, n);
+  return cudaGetLastError() == cudaSuccess ? MLA_OK : MLA_ERR_CUDA;
+}
+
+// New tokens per group of attention launches in mla_prefill_attention: bounds its workspace
+// (per-token items and split-KV partials) while leaving thousands of attention tiles per launch.
+constexpr int kPrefillGroup = 1024;
+
+size_t ws_prefill(const mla_dims* d, int T, int max_seq_len) {
+  if (T <= 0 || max_seq_len <= 0) return 0;
+  const int G = T < kPrefillGroup ? T : kPrefillGroup;
+  const size_t item_pages = ((size_t)max_seq_len + d->page_size - 1) / d->page_size;
+  size_t dec = ws_decode(d, G, max_seq_len);
+  if (T % G != 0) {  // the last, smaller group may split sequences further
+    const size_t last = ws_decode(d, T % G, max_seq_len);
+    if (last > dec) dec = last;
+  }
+  return align256((size_t)G * item_pages * 4) + align256((size_t)G * 4) + dec;
+}
+
+template <typename T>
+int prefill_impl(const mla_dims* d, const void* q, const void* pool, int32_t num_pages, const int32_t* bt,
+                 int32_t num_seqs, int32_t max_pages, const int32_t* seq_idx, const int32_t* pos, int32_t T_,
+                 int32_t max_seq_len, void* o_lat, float* lse_out, void* ws, cudaStream_t st) {
+  const int G = T_ < kPrefillGroup ? T_ : kPrefillGroup;
+  const int item_pages = (int)(((long)max_seq_len + d->page_size - 1) / d->page_size);
+  Carve c{static_cast<char*>(ws)};
+  int* item_bt = c.take<int>((size_t)G * item_pages);
+  int* item_len = c.take<int>((size_t)G);
+  void* dec_ws = static_cast<char*>(ws) + c.off;
+  const size_t q_row = (size_t)d->n_heads * (d->d_c + d->d_rope) * sizeof(T);
+  const size_t o_row = (size_t)d->n_heads * d->d_c * sizeof(T);
+  int32_t n = 0;
+  for (int g0 = 0; g0 < T_; g0 += G) {
+    const int g = T_ - g0 < G ? T_ - g0 : G;
+    if (launch_pdl(k_prefill_items, dim3((g + 7) / 8), dim3(256), 0, st, seq_idx + g0, pos + g0, bt, (int)num_seqs,
+                   (int)max_pages, (int)d->page_size, (int)max_seq_len, g, item_pages, item_bt,
+                   item_len) != cudaSuccess)
+      return MLA_ERR_CUDA;
+    ++n;
+    const int r = decode_impl<T>(d, static_cast<const char*>(q) + g0 * q_row, pool, num_pages, item_bt, item_pages,
+                                 item_len, g, max_seq_len, static_cast<char*>(o_lat) + g0 * o_row,
+                                 lse_out != nullptr ? lse_out + (size_t)g0 * d->n_heads : nullptr, dec_ws, st, n);
+    if (r != MLA_OK) return r;
+  }
+  return finish_launches(MLA_CALL_PREFILL_ATTENTION, n);
 }
 
 template <typename T>
@@ -299,6 +346,7 @@ size_t mla_workspace_size(const mla_dims* dims, int32_t call, int32_t B, int32_t
     case MLA_CALL_ABSORB_QUERY: return ws_absorb(dims, B);
     case MLA_CALL_DECODE_ATTENTION: return ws_decode(dims, B, max_seq_len);
     case MLA_CALL_OUT_PROJ: return ws_out(dims, B);
+    case MLA_CALL_PREFILL_ATTENTION: return ws_prefill(dims, B, max_seq_len);
     default: return 0;
   }
 }
@@ -364,11 +412,38 @@ int mla_decode_attention(const mla_dims* dims, const void* q, const void* pool, 
   if (ws_bytes < need) return MLA_ERR_WORKSPACE_TOO_SMALL;
   if (need > 0 && !ws) return MLA_ERR_INVALID_ARG;
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  int32_t n = 0;
+  r = dims->dtype == MLA_BF16
+          ? decode_impl<__nv_bfloat16>(dims, q, pool, num_pages, block_table, max_pages, seq_lens, B, max_seq_len,
+                                       o_lat, lse_out, ws, st, n)
+          : decode_impl<__half>(dims, q, pool, num_pages, block_table, max_pages, seq_lens, B, max_seq_len, o_lat,
+                                lse_out, ws, st, n);
+  if (r != MLA_OK) return r;
+  return finish_launches(MLA_CALL_DECODE_ATTENTION, n);
+}
+
+int mla_prefill_attention(const mla_dims* dims, const void* q, const void* pool, int32_t num_pages,
+                          const int32_t* block_table, int32_t num_seqs, int32_t max_pages, const int32_t* seq_idx,
+                          const int32_t* pos, int32_t T, int32_t max_seq_len, void* o_lat, float* lse_out, void* ws,
+                          size_t ws_bytes, mla_stream_t stream) {
+  const int r = check_dims_impl(dims);
+  if (r != MLA_OK) return r;
+  if (T < 0 || max_seq_len < 1 || num_seqs <= 0 || max_pages <= 0 || num_pages <= 0) return MLA_ERR_INVALID_ARG;
+  if ((long)max_pages * dims->page_size < (long)max_seq_len) return MLA_ERR_INVALID_ARG;
+  if (T == 0) {
+    t_launches[MLA_CALL_PREFILL_ATTENTION] = 0;
+    return MLA_OK;
+  }
+  if (!q || !pool || !block_table || !seq_idx || !pos || !o_lat || !ws) return MLA_ERR_INVALID_ARG;
+  if (!aligned16(q) || !aligned16(pool) || !aligned16(o_lat) || !aligned16(ws) || !aligned16(lse_out))
+    return MLA_ERR_ALIGNMENT;
+  if (ws_bytes < ws_prefill(dims, T, max_seq_len)) return MLA_ERR_WORKSPACE_TOO_SMALL;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
   if (dims->dtype == MLA_BF16)
-    return decode_impl<__nv_bfloat16>(dims, q, pool, num_pages, block_table, max_pages, seq_lens, B, max_seq_len,
-                                      o_lat, lse_out, ws, st);
-  return decode_impl<__half>(dims, q, pool, num_pages, block_table, max_pages, seq_lens, B, max_seq_len, o_lat,
-                             lse_out, ws, st);
+    return prefill_impl<__nv_bfloat16>(dims, q, pool, num_pages, block_table, num_seqs, max_pages, seq_idx, pos, T,
+                                       max_seq_len, o_lat, lse_out, ws, st);
+  return prefill_impl<__half>(dims, q, pool, num_pages, block_table, num_seqs, max_pages, seq_idx, pos, T,
+                              max_seq_len, o_lat, lse_out, ws, st);
 }
 
 int mla_out_proj(const mla_dims* dims, const void* o_lat, const void* w_uv, const void* w_o, void* u, int32_t B,
@@ -415,7 +490,7 @@ const char* mla_error_string(int code) {
   }
 }
 
-int32_t mla_last_launch_count(int32_t call) { return (call >= 0 && call < 4) ? t_launches[call] : -1; }
+int32_t mla_last_launch_count(int32_t call) { return (call >= 0 && call < 5) ? t_launches[call] : -1; }
 
 int mla_debug_gemm_plan(int32_t M, int32_t N, int32_t K, int32_t batch, int32_t fused_rope, int32_t d_rope,
                         int64_t* out) {

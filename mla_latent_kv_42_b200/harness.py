@@ -25,30 +25,32 @@ class Layer:
 @dataclass
 class StepIndex:
     cached: np.ndarray    # N_b
-    pos: torch.Tensor     # int32 [B], the new token's position = N_b
-    seq_idx: torch.Tensor  # int32 [B] = arange(B)
-    seq_lens: torch.Tensor  # int32 [B] = N_b + 1
+    chunk: int            # new tokens per sequence in the step (1 = decode)
+    pos: torch.Tensor     # int32 [T], positions of the new tokens: N_b, N_b + 1, ..., N_b + chunk - 1
+    seq_idx: torch.Tensor  # int32 [T], the sequence of each new token
+    seq_lens: torch.Tensor  # int32 [T] = pos + 1, the length each new token attends
     max_seq_len: int
 
 
-def step_index(cached: np.ndarray, device="cuda") -> StepIndex:
+def step_index(cached: np.ndarray, device="cuda", chunk: int = 1) -> StepIndex:
+    """Index tensors of a step that brings ``chunk`` new tokens to every sequence, listed
+    sequence by sequence (T = B * chunk). With chunk = 1 it is a decode step: pos = N_b,
+    seq_idx = b, seq_lens = N_b + 1."""
     cached = np.asarray(cached, dtype=np.int64)
     B = len(cached)
-    return StepIndex(
-        cached=cached,
-        pos=torch.from_numpy(cached.astype(np.int32)).to(device),
-        seq_idx=torch.arange(B, dtype=torch.int32, device=device),
-        seq_lens=torch.from_numpy((cached + 1).astype(np.int32)).to(device),
-        max_seq_len=int(cached.max()) + 1,
-    )
+    seq = np.repeat(np.arange(B, dtype=np.int64), chunk)
+    pos = cached[seq] + np.tile(np.arange(chunk, dtype=np.int64), B)
+    i32 = lambda a: torch.from_numpy(a.astype(np.int32)).to(device)
+    return StepIndex(cached=cached, chunk=chunk, pos=i32(pos), seq_idx=i32(seq), seq_lens=i32(pos + 1),
+                     max_seq_len=int(cached.max()) + chunk)
 
 
 def make_layer(w: synth.Workload, cached: np.ndarray, layer: int = 0, device="cuda", fill: float = 0.0,
-               block_table: np.ndarray | None = None, num_pages: int | None = None) -> Layer:
+               block_table: np.ndarray | None = None, num_pages: int | None = None, spare_tokens: int = 1) -> Layer:
     d = w.dims
     W = synth.weights(w, layer)
     if block_table is None:
-        block_table, num_pages = synth.page_table(cached, d.page_size, w.paging, w.seed)
+        block_table, num_pages = synth.page_table(cached, d.page_size, w.paging, w.seed, spare_tokens=spare_tokens)
     rows = synth.prefix_rows(w, cached, layer=layer, device=device)
     pool = synth.paged_pool(rows, cached, block_table, num_pages, d.page_size, fill=fill)
     st = LayerState(dims=d, w={k: v.to(device) for k, v in W.items()}, pool=pool,
@@ -86,3 +88,34 @@ def step_work(d: synth.Dims, seq_lens: np.ndarray) -> tuple[int, int]:
                           + 2 * n_h * d.d_head * d.d_c + d.d_model * n_h * d.d_head)
     act_bytes = 2 * B * (2 * d.d_model + (d.d_c + d.d_rope))  # h in, u out, the appended row
     return db + weight_bytes(d) + act_bytes, df + proj_flops
+
+
+def attention_work(d: synth.Dims, cached: np.ndarray, chunk: int = 1) -> tuple[int, int]:
+    """Algorithmic bytes and flops of the attention call of a step bringing ``chunk`` new tokens
+    to every sequence (chunk = 1: decode; equals ``decode_work(d, cached + 1)``).
+
+    Bytes: each sequence's N_b + chunk cache rows read once (the new tokens of a sequence share
+    them), q read and o_lat written per new token. Flops: the token at position t attends t + 1
+    rows, 2 n_h (d_c + d_h^R) for its scores and 2 n_h d_c for its weighted sum per row.
+    """
+    cached = np.asarray(cached, dtype=np.int64)
+    D = d.d_c + d.d_rope
+    T = len(cached) * chunk
+    rows = int(np.sum(cached + chunk))
+    attended = int(np.sum(chunk * (cached + 1) + chunk * (chunk - 1) // 2))
+    byts = 2 * (rows * D + T * d.n_heads * D + T * d.n_heads * d.d_c)
+    flops = 2 * attended * d.n_heads * (D + d.d_c)
+    return byts, flops
+
+
+def layer_work(d: synth.Dims, cached: np.ndarray, chunk: int = 1) -> tuple[int, int]:
+    """Algorithmic bytes and flops of a whole layer step bringing ``chunk`` new tokens to every
+    sequence: weights read once, the projections of every new token, and the attention call
+    (chunk = 1: equals ``step_work(d, cached + 1)``)."""
+    T = len(cached) * chunk
+    ab, af = attention_work(d, cached, chunk)
+    n_h = d.n_heads
+    proj_flops = 2 * T * ((d.d_c + d.d_rope) * d.d_model + d.d_cq * d.d_model + n_h * (d.d_head + d.d_rope) * d.d_cq
+                          + 2 * n_h * d.d_head * d.d_c + d.d_model * n_h * d.d_head)
+    act_bytes = 2 * T * (2 * d.d_model + (d.d_c + d.d_rope))
+    return ab + weight_bytes(d) + act_bytes, af + proj_flops

@@ -70,6 +70,7 @@ class Workload:
     sigma_w: float
     paging: str                     # "contiguous" or "shuffled"
     seed: int = 0
+    chunk: int = 1                  # new tokens per sequence per step (1 = decode; more = chunked prefill)
 
     @property
     def ragged(self) -> bool:
@@ -84,6 +85,7 @@ WORKLOADS = {
         Workload("production_b64_n4096_bf16", PRODUCTION, 64, 4096, 1, 0.006, "contiguous"),
         Workload("production_b128_ragged_paged_bf16", PRODUCTION, 128, (512, 32768), 1, 0.006, "shuffled"),
         Workload("production_b4_n131072_bf16", PRODUCTION, 4, 131072, 1, 0.006, "contiguous"),
+        Workload("production_b8_n4096_chunk128_bf16", PRODUCTION, 8, 4096, 1, 0.006, "contiguous", chunk=128),
     ]
 }
 

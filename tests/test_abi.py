@@ -25,9 +25,9 @@ def declared_functions():
     return sorted(set(re.findall(r"\b(mla_[a-z_0-9]+)\s*\(", text)))
 
 
-def test_header_declares_the_four_calls():
+def test_header_declares_the_calls():
     names = declared_functions()
-    for n in ("mla_append_kv", "mla_absorb_query", "mla_decode_attention", "mla_out_proj"):
+    for n in ("mla_append_kv", "mla_absorb_query", "mla_decode_attention", "mla_out_proj", "mla_prefill_attention"):
         assert n in names
 
 
@@ -130,7 +130,7 @@ def test_decode_timing_hook_arguments(lib):
 
 def test_workspace_sizes_are_consistent(lib):
     for d in (synth.RUNNING, synth.PRODUCTION):
-        for call in range(4):
+        for call in range(5):
             a = M.workspace_size(d, call, 64, 4097)
             b = M.workspace_size(d, call, 128, 32769)
             assert a >= 0 and b >= a
@@ -148,3 +148,45 @@ def test_error_strings(lib):
 def test_product_path_fails_loudly_without_the_library(tmp_path):
     with pytest.raises(RuntimeError, match="not built"):
         M.load_library(str(tmp_path / "missing.so"))
+
+
+def test_prefill_argument_errors_queue_nothing(lib):
+    cd = dims(synth.PRODUCTION)
+    f = lib.mla_prefill_attention
+    # dims, q, pool, num_pages, block_table, num_seqs, max_pages, seq_idx, pos, T, max_seq_len, o_lat, lse,
+    # ws, ws_bytes, stream
+    args = [ctypes.byref(cd), FAKE, FAKE, 10, FAKE, 2, 4, FAKE, FAKE, 5, 256, FAKE, None, FAKE, 1 << 30, None]
+
+    def call(**kw):
+        a = list(args)
+        for k, v in kw.items():
+            a[int(k[1:])] = v
+        return f(*a)
+
+    assert call(a7=None) == -1                            # null seq_idx
+    assert call(a8=None) == -1                            # null pos
+    assert call(a13=None) == -1                           # the per-token tables need a workspace
+    assert call(a12=MISALIGNED) == -4                     # misaligned lse_out
+    assert call(a5=0) == -1                               # no sequences
+    assert call(a9=-1) == -1                              # negative token count
+    assert call(a10=257) == -1                            # max_pages * page_size < max_seq_len
+    assert call(a14=16) == -3                             # too-small workspace
+    assert call(a9=0, a1=None, a13=None) == 0             # T == 0 is a no-op
+    assert lib.mla_last_launch_count(M.CALL_PREFILL_ATTENTION) == 0
+    assert lib.mla_last_launch_count(5) == -1
+
+
+def test_prefill_workspace_covers_decode_and_stops_growing():
+    """Tokens run in launch groups of at most 1024, so past one group the workspace stays put,
+    and it always holds a decode call's workspace for one group plus the per-token tables."""
+    for d in (synth.RUNNING, synth.PRODUCTION):
+        for T in (1, 7, 1000, 1024, 1025, 5000):
+            g = min(T, 1024)
+            need = M.workspace_size(d, M.CALL_PREFILL_ATTENTION, T, 4097)
+            assert need % 256 == 0
+            assert need >= M.workspace_size(d, M.CALL_DECODE_ATTENTION, g, 4097) + 4 * g * (-(-4097 // d.page_size))
+            assert need >= M.workspace_size(d, M.CALL_DECODE_ATTENTION, T % 1024 or g, 4097)
+    P = synth.PRODUCTION
+    assert (M.workspace_size(P, M.CALL_PREFILL_ATTENTION, 1024, 4097)
+            == M.workspace_size(P, M.CALL_PREFILL_ATTENTION, 4096, 4097)
+            == M.workspace_size(P, M.CALL_PREFILL_ATTENTION, 100000, 4097))

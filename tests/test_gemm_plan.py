@@ -80,7 +80,7 @@ def products(d):
 
 
 @pytest.mark.parametrize("dims", [synth.RUNNING, synth.PRODUCTION], ids=["running", "production"])
-@pytest.mark.parametrize("N", [1, 4, 16, 64, 128, 257, 300])
+@pytest.mark.parametrize("N", [1, 4, 16, 64, 128, 257, 300, 1024, 4096])
 def test_projection_plans(lib, dims, N):
     for Mr, K, batch, fused in products(dims):
         check_plan(plan(lib, Mr, N, K, batch, fused, dims.d_rope), Mr, N, K, batch, fused, dims.d_rope)
