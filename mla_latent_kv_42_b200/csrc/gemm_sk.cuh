@@ -134,12 +134,15 @@ struct RowDest {
   }
 };
 
-// cos/sin of one RoPE angle, kept out of line: the epilogue loop that may call it is unrolled and
-// runs with cold instruction fetch, so an inlined double-precision pow and sincos in its (rarely
-// taken) branch would slow every pass through it.
-__device__ __noinline__ float2 rope_cs_out_of_line(int pos, int k, int d_rope, double base) {
+// cos/sin of the RoPE angle of token n, pair k: read from the per-token table `tab`
+// ([N][d_rope/2]) when an earlier kernel filled it, else computed. Kept out of line: the epilogue
+// loop that may call it is unrolled and runs with cold instruction fetch, so an inlined
+// double-precision pow and sincos in its branch would slow every pass through it.
+__device__ __noinline__ float2 rope_cs_out_of_line(const float2* tab, const int* pos, int n, int k, int d_rope,
+                                                   double base) {
+  if (tab != nullptr) return tab[(long)n * (d_rope / 2) + k];
   float2 q;
-  rope_cos_sin(pos, k, d_rope, base, q.x, q.y);
+  rope_cos_sin(pos[n], k, d_rope, base, q.x, q.y);
   return q;
 }
 
@@ -414,7 +417,8 @@ __global__ void __launch_bounds__(192, 2)
               if (rot && nl < nv) {
                 float2 q;
                 if (tab_cs) q = cs_tab[nl * half_rope + k];
-                else q = rope_cs_out_of_line(p.epi.pos[n0 + nl], k, p.epi.d_rope, p.epi.rope_base);
+                else q = rope_cs_out_of_line(p.epi.cs_ready ? p.epi.cs_glob : nullptr, p.epi.pos, n0 + nl, k,
+                                             p.epi.d_rope, p.epi.rope_base);
                 v = (m & 1) ? fmaf(w, q.y, v * q.x) : fmaf(v, q.x, -w * q.y);
               }
             }

@@ -308,7 +308,7 @@ struct AbsorbLayout {
   void* qc;     // q^C, element type [B, n_h*d_h]
   float* Y2;    // CUDA-core route: [q^C ; q^R before RoPE] fp32 [B, nq]
   float* part;  // stream-K partials, shared by the three products (they run one after another)
-  float2* cs;   // RoPE cos/sin per token for the reduction of split query tiles
+  float2* cs;   // RoPE cos/sin per token, filled by the W^DQ product for the query product
   size_t bytes;
   bool tc_uk;   // the per-head (W^UK_i)^T product runs on the tensor-core GEMM
 };
@@ -327,7 +327,7 @@ inline AbsorbLayout absorb_layout(const mla_dims* d, int B, void* ws) {
   size_t part = 0;
   if (!simt) part = std::max(L.g1.part_bytes, std::max(L.g2.part_bytes, L.tc_uk ? L.g3.part_bytes : 0));
   L.part = part ? c.take<float>(part / sizeof(float)) : nullptr;
-  L.cs = (!simt && L.g2.n_tiles == 1) ? c.take<float2>((size_t)B * (d->d_rope / 2)) : nullptr;
+  L.cs = !simt ? c.take<float2>((size_t)B * (d->d_rope / 2)) : nullptr;
   L.bytes = c.off;
   return L;
 }
@@ -372,7 +372,10 @@ int absorb_run(const mla_dims* d, const void* h, const void* w_dq, const void* w
     e.d_c = d->d_c;
     e.cs_glob = L.cs;
     e.cs_ready = L.cs != nullptr;
-    e.rope_in_reduce = L.g2.split && L.cs != nullptr;  // the reduction runs anyway
+    // one n tile: rope tiles go through the reduction, which runs anyway, instead of rotating from
+    // a shared-memory table while the next tile streams in; several n tiles: whole tiles read the
+    // cos/sin per element from the global table
+    e.rope_in_reduce = L.g2.split && L.g2.n_tiles == 1 && L.cs != nullptr;
     r = gemm_sk<T>({w_uq_qr, nq, d->d_cq, 0}, false, {cq, B, d->d_cq, 0}, nq, B, d->d_cq, L.g2, e, L.part, st, n);
     if (r != MLA_OK) return r;
   }
