@@ -203,7 +203,8 @@ typedef struct CUevent_st* mla_event_t;
 
 /* Profiling hook (not part of the method): from this call on, every mla_decode_attention (and
  * _noalloc) call made by this host thread records `before` on its stream immediately before the
- * attention kernel and `after` immediately after it, so that the kernel's own duration can be
+ * attention kernel and `after` immediately after it (mla_prefill_attention records them around the
+ * attention kernel of each of its launch groups, so afterwards they bracket the last group's), so that the kernel's own duration can be
  * read with cudaEventElapsedTime apart from the planner and the split-KV merge launched in the
  * same call. Pass NULL for both to stop. The events belong to the caller, who creates them
  * (with timing) and destroys them. An event recorded between two launches keeps the second

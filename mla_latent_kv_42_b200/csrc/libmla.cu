@@ -303,6 +303,9 @@ int prefill_impl(const mla_dims* d, const void* q, const void* pool, int32_t num
   const size_t q_row = (size_t)d->n_heads * (d->d_c + d->d_rope) * sizeof(T);
   const size_t o_row = (size_t)d->n_heads * d->d_c * sizeof(T);
   int32_t n = 0;
+  // The groups reuse the item tables and the attention workspace. Each group's k_prefill_items
+  // waits (griddep_wait) for the kernel before it, the previous group's last launch, which itself
+  // waited for that group's attention kernel, the last reader of those buffers.
   for (int g0 = 0; g0 < T_; g0 += G) {
     const int g = T_ - g0 < G ? T_ - g0 : G;
     if (launch_pdl(k_prefill_items, dim3((g + 7) / 8), dim3(256), 0, st, seq_idx + g0, pos + g0, bt, (int)num_seqs,
