@@ -21,6 +21,9 @@
  *   - Asynchrony: work is queued on `stream` (NULL = the legacy default stream) and the call
  *     returns without synchronising. Calls on different streams may run concurrently if their
  *     buffers (including workspaces) do not overlap.
+ *   - Threads: any host thread may call at any time. The library's own host state is per-device
+ *     caches of device properties (atomic) and, per thread, the launch counts and the timing
+ *     hook below; mla_decode_attention_noalloc's static scratch is the one shared buffer.
  *   - Overlap of consecutive kernels: every kernel is launched with programmatic dependent
  *     launch, so it may start while the kernel queued just before it on `stream` still runs.
  *     Each kernel waits for that predecessor to complete, with its memory visible, before it

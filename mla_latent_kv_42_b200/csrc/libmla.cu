@@ -3,6 +3,7 @@
 // Host code here validates arguments (before anything is queued), carves the caller's
 // workspace, picks kernels and launches them on the caller's stream. It allocates nothing.
 #include "mla_debug.h"
+#include <atomic>
 #include <cmath>
 #include <cstring>
 #include <mutex>
@@ -29,16 +30,18 @@ inline void mark_after(cudaStream_t st) {
 
 constexpr int kMaxDevices = 64;
 
+// Per-device values cached on first use. Host threads may call concurrently: the caches are
+// atomics, and a race only computes the same value twice.
 int device_sm_count() {
-  static int cache[kMaxDevices] = {0};
+  static std::atomic<int> cache[kMaxDevices];
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return 148;
-  if (cache[dev] == 0) {
-    int n = 0;
-    if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0) n = 148;
-    cache[dev] = n;
+  int v = cache[dev].load(std::memory_order_relaxed);
+  if (v == 0) {
+    if (cudaDeviceGetAttribute(&v, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || v <= 0) v = 148;
+    cache[dev].store(v, std::memory_order_relaxed);
   }
-  return cache[dev];
+  return v;
 }
 
 inline bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
@@ -123,35 +126,35 @@ int absorb_impl(const mla_dims* d, const void* h, const void* w_dq, const void* 
 // The tcgen05 path serves DeepSeek-V2-shaped caches (d_c = 512, d_h^R = 64, 64-token pages,
 // 65..128 heads); MLA_DECODE_IMPL=simt selects the CUDA-core kernel instead.
 bool decode_tc_eligible(const mla_dims* d) {
-  static int forced_simt = -1;
-  if (forced_simt < 0) {
+  static const bool forced_simt = [] {
     const char* e = std::getenv("MLA_DECODE_IMPL");
-    forced_simt = (e != nullptr && std::strcmp(e, "simt") == 0) ? 1 : 0;
-  }
+    return e != nullptr && std::strcmp(e, "simt") == 0;
+  }();
   return !forced_simt && d->n_heads > 64 && d->n_heads <= 128 && d->d_c == tc::dec::kDc &&
          d->d_c + d->d_rope == tc::dec::kD && d->page_size == tc::dec::kPage;
 }
 
 template <typename T>
 bool decode_tc_set_smem() {
-  static bool done[kMaxDevices] = {};
+  static std::atomic<bool> done[kMaxDevices];
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return false;
-  if (!done[dev]) {
+  if (!done[dev].load(std::memory_order_acquire)) {
     if (cudaFuncSetAttribute(tc::k_decode_tc<T>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)tc::dec::kSmem) !=
         cudaSuccess)
       return false;
-    done[dev] = true;
+    done[dev].store(true, std::memory_order_release);
   }
   return true;
 }
 
 // Clusters of two CTAs that can be resident at once: the work is split statically over them.
 int decode_clusters() {
-  static int cache[kMaxDevices] = {0};
+  static std::atomic<int> cache[kMaxDevices];
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return device_sm_count() / 2;
-  if (cache[dev] == 0) {
+  int c = cache[dev].load(std::memory_order_relaxed);
+  if (c == 0) {
     int n = 0;
     if (decode_tc_set_smem<__nv_bfloat16>()) {
       cudaLaunchConfig_t cfg = {};
@@ -161,9 +164,10 @@ int decode_clusters() {
       if (cudaOccupancyMaxActiveClusters(&n, tc::k_decode_tc<__nv_bfloat16>, &cfg) != cudaSuccess) n = 0;
     }
     cudaGetLastError();
-    cache[dev] = n > 0 ? n : device_sm_count() / 2;
+    c = n > 0 ? n : device_sm_count() / 2;
+    cache[dev].store(c, std::memory_order_relaxed);
   }
-  return cache[dev];
+  return c;
 }
 
 size_t ws_decode_tc(const mla_dims* d, int B) {

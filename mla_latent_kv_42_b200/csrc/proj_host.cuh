@@ -8,6 +8,7 @@
 #include <cudaTypedefs.h>
 
 #include <algorithm>
+#include <atomic>
 #include <cstdlib>
 #include <cstring>
 #include <mutex>
@@ -20,16 +21,18 @@ namespace host {
 
 constexpr int kMaxDev = 64;
 
+// Per-device values cached on first use; atomics, since host threads may call concurrently (a race
+// only computes the same value twice).
 inline int sm_count() {
-  static int cache[kMaxDev] = {0};
+  static std::atomic<int> cache[kMaxDev];
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDev) return 148;
-  if (cache[dev] == 0) {
-    int n = 0;
-    if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0) n = 148;
-    cache[dev] = n;
+  int v = cache[dev].load(std::memory_order_relaxed);
+  if (v == 0) {
+    if (cudaDeviceGetAttribute(&v, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || v <= 0) v = 148;
+    cache[dev].store(v, std::memory_order_relaxed);
   }
-  return cache[dev];
+  return v;
 }
 
 inline size_t a256(size_t x) { return (x + 255) & ~size_t(255); }
@@ -46,12 +49,11 @@ struct Carver {
 };
 
 inline bool proj_uses_simt() {
-  static int v = -1;
-  if (v < 0) {
+  static const bool v = [] {
     const char* e = std::getenv("MLA_PROJ_IMPL");
-    v = (e != nullptr && std::strcmp(e, "simt") == 0) ? 1 : 0;
-  }
-  return v == 1;
+    return e != nullptr && std::strcmp(e, "simt") == 0;
+  }();
+  return v;
 }
 
 // ------------------------------------------------------------------ TMA tensor maps
@@ -151,14 +153,14 @@ struct Operand {
 template <typename T, int BN, bool MN, int MODE>
 cudaError_t run_sk(const CUtensorMap& ma, const CUtensorMap& mb, const tc::SkParams& p, const SkPlan& g,
                    cudaStream_t st, int32_t& n) {
-  static bool attr_done[kMaxDev] = {};
+  static std::atomic<bool> attr_done[kMaxDev];
   int dev = 0;
   cudaGetDevice(&dev);
-  if (dev >= 0 && dev < kMaxDev && !attr_done[dev]) {
+  if (dev >= 0 && dev < kMaxDev && !attr_done[dev].load(std::memory_order_acquire)) {
     cudaError_t e = cudaFuncSetAttribute(tc::k_gemm_sk<T, BN, MN, MODE>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          (int)kSkSmemMax);
     if (e != cudaSuccess) return e;
-    attr_done[dev] = true;
+    attr_done[dev].store(true, std::memory_order_release);
   }
   cudaError_t e = launch_pdl(tc::k_gemm_sk<T, BN, MN, MODE>, dim3(g.G), dim3(192), g.smem, st, ma, mb, p);
   if (e != cudaSuccess) return e;
