@@ -22,6 +22,9 @@ Sources (page title, section or equation):
        §8.2 the worked softmax example.
   [S2] DeepSeek-V2 paper review (velog): §2.1 latency model; §2.3 decoupled RoPE.
   [S4] DeepSeek-V2 visual explainer: 576 vs 32,768 numbers per token; the toy 512 -> 64.
+  [S5] "DeepSeek-V2: A Strong, Economical, and Efficient Mixture-of-Experts Language Model
+       (Multi-head Latent Attention)" summary: "The Model: DeepSeek-V2" (a 6-bit KV cache and
+       FP8 weights in deployment).
 
 Readings where the pages are silent:
   R1 RoPE rotates adjacent pairs (x_2k, x_2k+1) by the standard 2x2 rotation matrix.
@@ -34,6 +37,10 @@ Readings where the pages are silent:
   R7 A step may bring several new tokens of one sequence (the attention sum of [S1] §6 for a
      general t): they take the consecutive positions after the prefix, all their rows are
      cached first, and each token attends to the rows up to its own position (causal).
+  R8 A quantised latent cache ([S2] §4.2 and [S5] give a KV cache of about 6 bits per element
+     without its format): e4m3 bytes with two float32 scales per token, max|part| / 448 for c and for k^R,
+     values divided by their scale in float32 and rounded to the nearest e4m3 value, ties to
+     even. Attention over it is the attention over the rows it stands for.
 
 Every function has pins in ``tests/test_oracle_pins.py``; none is "parity unpinned".
 """
@@ -47,6 +54,7 @@ __all__ = [
     "kv_rows", "query_path", "attention_naive", "output_naive", "layer_step_naive",
     "absorb_query", "latent_attention", "lse_merge", "out_proj_absorbed", "layer_step_absorbed",
     "chunk_positions", "chunk_step_naive", "chunk_latent_attention", "chunk_step_absorbed",
+    "E4M3_MAX", "e4m3_values", "quantize_e4m3", "fp8_row_scales", "quantize_rows_fp8", "dequantize_rows_fp8",
     "page_slot", "as64",
 ]
 
@@ -331,3 +339,66 @@ def chunk_step_absorbed(W: dict, h, prefix: list, chunk_lens, dims) -> dict:
     o_lat, lse = chunk_latent_attention(q, full, seq_idx, pos, dims)
     return {"seq_idx": seq_idx, "pos": pos, "rows": new_rows, "q": q, "o_lat": o_lat, "lse": lse,
             "u": out_proj_absorbed(W["w_uv"], W["w_o"], o_lat)}
+
+
+# --------------------------------------------------------------------------- FP8 latent cache (reading R8)
+E4M3_MAX = 448.0
+
+
+def e4m3_values() -> np.ndarray:
+    """The 256 values of the e4m3 ("fn") byte format, indexed by code, decoded from its fields:
+    sign bit 7, exponent bits 6-3 with bias 7, fraction bits 2-0. Exponent field 0 holds the
+    subnormals f/8 * 2^-6; exponent 15 with fraction 7 is NaN; there are no infinities."""
+    v = np.empty(256, dtype=np.float64)
+    for code in range(256):
+        s, e, f = code >> 7, (code >> 3) & 15, code & 7
+        if e == 15 and f == 7:
+            v[code] = np.nan
+            continue
+        mag = (f / 8.0) * 2.0 ** -6 if e == 0 else (1.0 + f / 8.0) * 2.0 ** (e - 7)
+        v[code] = -mag if s else mag
+    return v
+
+
+def quantize_e4m3(y) -> np.ndarray:
+    """Nearest e4m3 value to each finite y with |y| <= 448, ties to the even fraction (R8).
+
+    The grid spacing is 2^(E-3) for |y| in [2^E, 2^(E+1)), E >= -6, and 2^-9 below 2^-6."""
+    y = np.asarray(y, dtype=np.float64)
+    assert np.all(np.abs(y) <= E4M3_MAX), "scale the values into range first"
+    a = np.abs(y)
+    E = np.floor(np.log2(np.where(a > 0, a, 1.0)))
+    step = 2.0 ** (np.maximum(E, -6.0) - 3.0)
+    return np.sign(y) * np.round(a / step) * step      # np.round rounds halves to even
+
+
+def fp8_row_scales(rows, d_c: int):
+    """Per-token scales of the FP8 latent cache (R8): one for the latent part c (d_c values) and one
+    for the RoPE key k^R, each max|part| / 448 computed in float32 (the precision the cache writer
+    uses, so that both sides take the same rounding decisions); 1 for an all-zero part.
+    Returns float32 [T, 2]."""
+    rows = np.asarray(rows, dtype=np.float32)
+    out = np.empty((rows.shape[0], 2), dtype=np.float32)
+    for j, part in enumerate((rows[:, :d_c], rows[:, d_c:])):
+        m = np.abs(part).max(axis=1) if part.shape[1] else np.zeros(rows.shape[0], np.float32)
+        out[:, j] = np.where(m > 0, m / np.float32(E4M3_MAX), np.float32(1.0))
+    return out
+
+
+def quantize_rows_fp8(rows, d_c: int):
+    """FP8 cache rows (R8): each part divided by its scale in float32, then rounded to e4m3.
+    The part's largest value divides to 448 up to one float32 rounding, so the quotient is
+    clamped to +-448 first (a saturating conversion). ``rows`` [T, D] (the element-type rows the
+    bf16 cache would hold). Returns (values [T, D] as float64, the exact e4m3 values; scales
+    float32 [T, 2])."""
+    rows32 = np.asarray(rows, dtype=np.float32)
+    sc = fp8_row_scales(rows32, d_c)
+    y = np.concatenate([rows32[:, :d_c] / sc[:, :1], rows32[:, d_c:] / sc[:, 1:]], axis=1)
+    return quantize_e4m3(np.clip(y.astype(np.float64), -E4M3_MAX, E4M3_MAX)), sc
+
+
+def dequantize_rows_fp8(values, scales, d_c: int) -> np.ndarray:
+    """Rows the FP8 cache stands for: each part's e4m3 values times its scale, in float64."""
+    values = np.asarray(values, dtype=np.float64)
+    sc = np.asarray(scales, dtype=np.float64)
+    return np.concatenate([values[:, :d_c] * sc[:, :1], values[:, d_c:] * sc[:, 1:]], axis=1)

@@ -533,3 +533,80 @@ def test_chunk_pins_catch_a_causal_off_by_one():
         o_lat, _ = O.chunk_latent_attention(good["q"], [full], seq0, good["pos"] + shift, dims)
         err = np.abs(o_lat[1] - step["o_lat"][0]).max()
         assert (err < 1e-12) if ok else (err > 1e-6)
+
+
+# ----------------------------------------------------------------------------- FP8 latent cache
+def _torch_e4m3(y):
+    return torch.from_numpy(np.asarray(y, dtype=np.float32)).to(torch.float8_e4m3fn).double().numpy()
+
+
+def test_e4m3_decoding_matches_the_library_format():
+    """The 256 codes decoded from the format's fields equal torch's float8_e4m3fn bytes; closed
+    forms: largest 448, smallest normal 2^-6, smallest subnormal 2^-9, NaN only at S.1111.111."""
+    v = O.e4m3_values()
+    lib = torch.arange(256, dtype=torch.uint8).view(torch.float8_e4m3fn).double().numpy()
+    np.testing.assert_array_equal(np.isnan(v), np.isnan(lib))
+    np.testing.assert_array_equal(v[~np.isnan(v)], lib[~np.isnan(lib)])
+    assert np.flatnonzero(np.isnan(v)).tolist() == [127, 255]
+    assert np.nanmax(v) == O.E4M3_MAX == 448.0
+    assert v[0b00001000] == 2.0 ** -6 and v[1] == 2.0 ** -9
+
+
+def test_e4m3_rounding_nearest_even_against_the_library_and_brute_force():
+    """Every value, every midpoint between neighbours (ties go to the even fraction) and random
+    values across the normal and subnormal range round as torch's conversion does, and as an
+    exhaustive nearest-value search with ties to the even code does."""
+    v = O.e4m3_values()
+    pos = np.unique(v[(~np.isnan(v)) & (v >= 0)])
+    mids = (pos[1:] + pos[:-1]) / 2
+    rng = np.random.default_rng(40)
+    rnd = np.concatenate([rng.uniform(-448, 448, 2000), rng.uniform(-2 ** -5, 2 ** -5, 2000),
+                          np.exp2(rng.uniform(-12, 8.8, 2000)) * rng.choice([-1, 1], 2000)])
+    rnd = rnd[np.abs(rnd) <= 448]
+    for y in (pos, -pos, mids, -mids, rnd):
+        y32 = y.astype(np.float32).astype(np.float64)        # the quantiser sees float32 inputs
+        np.testing.assert_array_equal(O.quantize_e4m3(y32), _torch_e4m3(y32))
+    finite = np.flatnonzero(~np.isnan(v))
+    for y in rnd[:300].astype(np.float32).astype(np.float64):
+        d = np.abs(v[finite] - y)
+        best = finite[d == d.min()]
+        code = best[0] if len(best) == 1 else best[(best & 1) == 0][0]
+        assert O.quantize_e4m3(y) == v[code], y
+    np.testing.assert_array_equal(O.quantize_e4m3(pos), pos)  # representable values are fixed points
+
+
+def test_fp8_rows_error_bound_scales_and_zero_parts():
+    """Per token and part, max|part| maps to 448 and every value is within half an e4m3 spacing:
+    2^-4 of its magnitude for normals, 2^-10 of the scale for subnormals (plus float32 division
+    rounding). An all-zero part gets scale 1 and zero values."""
+    d = PRODUCTION
+    rng = np.random.default_rng(41)
+    rows = (rng.standard_normal((50, d.D)) * np.exp2(rng.uniform(-6, 6, (50, 1)))).astype(np.float32)
+    rows[3, d.d_c:] = 0.0
+    rows[4, :d.d_c] = 0.0
+    vals, sc = O.quantize_rows_fp8(rows, d.d_c)
+    assert sc.dtype == np.float32 and sc.shape == (50, 2)
+    assert sc[3, 1] == 1.0 and sc[4, 0] == 1.0
+    assert not vals[3, d.d_c:].any() and not vals[4, :d.d_c].any()
+    for j, part in enumerate((slice(0, d.d_c), slice(d.d_c, d.D))):
+        m = np.abs(vals[:, part]).max(axis=1)
+        live = np.abs(rows[:, part]).max(axis=1) > 0
+        assert np.all(m[live] == 448.0)
+        y = rows[:, part].astype(np.float64) / sc[:, j:j + 1].astype(np.float64)
+        err = np.abs(vals[:, part] - y)
+        bound = np.maximum(np.abs(y) * 2.0 ** -4, 2.0 ** -10) * (1 + 1e-6) + np.abs(y) * 2.0 ** -23
+        assert np.all(err <= bound)
+    back = O.dequantize_rows_fp8(vals, sc, d.d_c)
+    rel = np.abs(back - rows) / np.maximum(np.abs(rows), 1e-30)
+    assert np.median(rel[rows != 0]) < 2.0 ** -5
+
+
+def test_fp8_pins_catch_ties_away_from_zero():
+    """Rounding halves away from zero (a plausible slip) disagrees with the library at midpoints."""
+    v = O.e4m3_values()
+    pos = np.unique(v[(~np.isnan(v)) & (v >= 0)])
+    mids = (pos[1:] + pos[:-1]) / 2
+    a = np.abs(mids)
+    step = 2.0 ** (np.maximum(np.floor(np.log2(a)), -6.0) - 3.0)
+    away = np.floor(a / step + 0.5) * step
+    assert np.any(away != _torch_e4m3(mids))
