@@ -190,3 +190,16 @@ def test_prefill_workspace_covers_decode_and_stops_growing():
     assert (M.workspace_size(P, M.CALL_PREFILL_ATTENTION, 1024, 4097)
             == M.workspace_size(P, M.CALL_PREFILL_ATTENTION, 4096, 4097)
             == M.workspace_size(P, M.CALL_PREFILL_ATTENTION, 100000, 4097))
+
+
+def test_binding_refuses_host_tensors_before_calling_the_library(lib):
+    """The binding checks placement, layout and dtype itself: host, strided or mistyped tensors
+    raise ValueError and reach no C call (so nothing is queued)."""
+    import torch
+    d = synth.RUNNING
+    q = torch.zeros((3, d.n_heads, d.D), dtype=torch.bfloat16)
+    i32 = torch.zeros(3, dtype=torch.int32)
+    with pytest.raises(ValueError, match="CUDA"):
+        M.prefill_attention(d, q, q, i32.view(1, 3), i32, i32, 4)
+    with pytest.raises(ValueError, match="CUDA"):
+        M.decode_attention(d, q, q, i32.view(1, 3), i32, 4)
