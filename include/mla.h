@@ -130,7 +130,8 @@ int mla_append_kv(const mla_dims* dims, const void* h, const void* w_dkv_kr,
  *   q_out[b][i] = [q~_i (d_c) ‖ q^R_i (d_rope)]   — the same layout as a cache row.
  * h [B, d_model]; w_dq [d_cq, d_model]; w_uq_qr [n_heads*(d_head + d_rope), d_cq] (W^UQ rows
  * then W^QR rows); w_uk [n_heads*d_head, d_c]; pos int32 [B]; q_out [B, n_heads, d_c + d_rope].
- * c^Q and q^C are rounded to the element type before their next product.
+ * c^Q and q^C are rounded to the element type before their next product. 0 <= B <= 65535
+ * (MLA_ERR_INVALID_ARG otherwise); B == 0 is a no-op.
  */
 int mla_absorb_query(const mla_dims* dims, const void* h, const void* w_dq, const void* w_uq_qr,
                      const void* w_uk, const int32_t* pos, void* q_out, int32_t B,
@@ -147,7 +148,8 @@ int mla_absorb_query(const mla_dims* dims, const void* h, const void* w_dq, cons
  * o_lat [B, n_heads, d_c] element type; lse_out float [B, n_heads] or NULL.
  * Long sequences are split across SMs and the partials merged by log-sum-exp; the result is
  * bitwise reproducible run to run. A bad seq_len or page id zeroes that sequence's output and
- * records the error in the device status.
+ * records the error in the device status. 0 <= B <= 65535 and max_pages * page_size >=
+ * max_seq_len >= 1 (MLA_ERR_INVALID_ARG otherwise); B == 0 is a no-op.
  */
 int mla_decode_attention(const mla_dims* dims, const void* q, const void* pool, int32_t num_pages,
                          const int32_t* block_table, int32_t max_pages, const int32_t* seq_lens,
@@ -186,7 +188,7 @@ int mla_prefill_attention(const mla_dims* dims, const void* q, const void* pool,
  *   o_i = W^UV_i o_lat_i   (d_head values, rounded to the element type)
  *   u   = W^O [o_1 ; ... ; o_n_h]
  * o_lat [B, n_heads, d_c]; w_uv [n_heads*d_head, d_c]; w_o [d_model, n_heads*d_head];
- * u [B, d_model].
+ * u [B, d_model]. 0 <= B <= 65535 (MLA_ERR_INVALID_ARG otherwise); B == 0 is a no-op.
  */
 int mla_out_proj(const mla_dims* dims, const void* o_lat, const void* w_uv, const void* w_o,
                  void* u, int32_t B, void* ws, size_t ws_bytes, mla_stream_t stream);
