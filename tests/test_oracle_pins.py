@@ -270,6 +270,22 @@ def test_zero_query_gives_the_mean_latent():
     np.testing.assert_allclose(lse, math.log(301), rtol=1e-15)
 
 
+def test_latent_attention_lse_and_weights_against_scipy():
+    """§5.3 steps 2-3 with the §4.4 scale through scipy's logsumexp and softmax: the log-sum-exp
+    (natural log, over the scaled scores) and the weighted sum of latents, on scores wide enough
+    that a missing max shift would overflow."""
+    import scipy.special as sp
+    dims = PRODUCTION
+    rng = np.random.default_rng(16)
+    rows = rng.standard_normal((97, dims.D))
+    q = rng.standard_normal((dims.n_heads, dims.D)) * 120.0
+    o_lat, lse = O.latent_attention(q, rows, dims)
+    s = (q @ rows.T) / math.sqrt(dims.d_head + dims.d_rope)
+    assert np.abs(s).max() > 710.0                       # exp would overflow without the shift
+    np.testing.assert_allclose(lse, sp.logsumexp(s, axis=1), rtol=1e-14)
+    np.testing.assert_allclose(o_lat, sp.softmax(s, axis=1) @ rows[:, :dims.d_c], rtol=1e-10, atol=1e-12)
+
+
 def test_all_equal_rows_return_that_row():
     dims = RUNNING
     rng = np.random.default_rng(13)
