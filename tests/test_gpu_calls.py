@@ -264,8 +264,9 @@ def test_out_proj(fam):
 
 @pytest.mark.parametrize("fam", ["running_bf16", "production_bf16"])
 def test_projections_beyond_one_n_tile(fam):
-    """300 tokens: the GEMMs run two n tiles of 256, with RoPE computed per element (no shared
-    table) and the append's scatter per token."""
+    """300 tokens: the GEMMs run two n tiles of 256 with no shared-memory RoPE table: the query's
+    q^R reads each cos/sin from the global per-token table the W^DQ product fills, the append's
+    k^R computes its own, and the append scatters per token."""
     w = FAMILIES[fam]
     d = w.dims
     W, W64 = weights64(w)
