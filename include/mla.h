@@ -148,8 +148,8 @@ int mla_absorb_query(const mla_dims* dims, const void* h, const void* w_dq, cons
  * o_lat [B, n_heads, d_c] element type; lse_out float [B, n_heads] or NULL.
  * Long sequences are split across SMs and the partials merged by log-sum-exp; the result is
  * bitwise reproducible run to run. A bad seq_len or page id zeroes that sequence's output and
- * records the error in the device status. 0 <= B <= 65535 and max_pages * page_size >=
- * max_seq_len >= 1 (MLA_ERR_INVALID_ARG otherwise); B == 0 is a no-op.
+ * records the error in the device status. 0 <= B <= 65535, 1 <= max_seq_len <= 2^30 and
+ * max_pages * page_size >= max_seq_len (MLA_ERR_INVALID_ARG otherwise); B == 0 is a no-op.
  */
 int mla_decode_attention(const mla_dims* dims, const void* q, const void* pool, int32_t num_pages,
                          const int32_t* block_table, int32_t max_pages, const int32_t* seq_lens,
@@ -168,7 +168,7 @@ int mla_decode_attention(const mla_dims* dims, const void* q, const void* pool, 
  * seq_idx and pos), and q is mla_absorb_query's output for the same tokens and positions.
  * q [T, n_heads, d_c + d_rope]; seq_idx int32 [T] in [0, num_seqs); pos int32 [T] in
  * [0, max_seq_len); block_table int32 [num_seqs, max_pages] and pool as in mla_append_kv,
- * max_pages * page_size >= max_seq_len; o_lat [T, n_heads, d_c] element type; lse_out float
+ * max_pages * page_size >= max_seq_len, 1 <= max_seq_len <= 2^30; o_lat [T, n_heads, d_c] element type; lse_out float
  * [T, n_heads] or NULL; ws at least mla_workspace_size(dims, MLA_CALL_PREFILL_ATTENTION, T,
  * max_seq_len) bytes. Tokens may come in any order; each is computed on its own, with the
  * arithmetic of mla_decode_attention for a sequence of length pos[t] + 1 (where split-KV

@@ -29,6 +29,9 @@ inline void mark_after(cudaStream_t st) {
 }
 
 constexpr int kMaxDevices = 64;
+// Longest attended length the attention calls accept: page counts and token indices stay far
+// from int32 overflow in every kernel.
+constexpr int32_t kMaxSeqLen = 1 << 30;
 
 // Per-device values cached on first use. Host threads may call concurrently: the caches are
 // atomics, and a race only computes the same value twice.
@@ -406,7 +409,8 @@ int mla_decode_attention(const mla_dims* dims, const void* q, const void* pool, 
                          mla_stream_t stream) {
   int r = check_dims_impl(dims);
   if (r != MLA_OK) return r;
-  if (B < 0 || B > 65535 || max_seq_len < 1 || max_pages <= 0 || num_pages <= 0) return MLA_ERR_INVALID_ARG;
+  if (B < 0 || B > 65535 || max_seq_len < 1 || max_seq_len > kMaxSeqLen || max_pages <= 0 || num_pages <= 0)
+    return MLA_ERR_INVALID_ARG;
   if ((long)max_pages * dims->page_size < (long)max_seq_len) return MLA_ERR_INVALID_ARG;
   if (B == 0) {
     t_launches[MLA_CALL_DECODE_ATTENTION] = 0;
@@ -435,7 +439,8 @@ int mla_prefill_attention(const mla_dims* dims, const void* q, const void* pool,
                           size_t ws_bytes, mla_stream_t stream) {
   const int r = check_dims_impl(dims);
   if (r != MLA_OK) return r;
-  if (T < 0 || max_seq_len < 1 || num_seqs <= 0 || max_pages <= 0 || num_pages <= 0) return MLA_ERR_INVALID_ARG;
+  if (T < 0 || max_seq_len < 1 || max_seq_len > kMaxSeqLen || num_seqs <= 0 || max_pages <= 0 || num_pages <= 0)
+    return MLA_ERR_INVALID_ARG;
   if ((long)max_pages * dims->page_size < (long)max_seq_len) return MLA_ERR_INVALID_ARG;
   if (T == 0) {
     t_launches[MLA_CALL_PREFILL_ATTENTION] = 0;

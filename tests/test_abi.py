@@ -99,6 +99,10 @@ def test_decode_argument_errors_queue_nothing(lib):
     need = lib.mla_workspace_size(ctypes.byref(cd), M.CALL_DECODE_ATTENTION, 2, 256)
     assert f(*bad) == (-3 if need > 0 else f(*bad))        # too-small workspace
     bad = list(args)
+    bad[8] = (1 << 30) + 1
+    bad[5] = 1 << 25
+    assert f(*bad) == -1                                  # max_seq_len beyond 2^30
+    bad = list(args)
     bad[7] = 0
     assert f(*bad) == 0                                   # B == 0 is a no-op
 
@@ -170,6 +174,7 @@ def test_prefill_argument_errors_queue_nothing(lib):
     assert call(a5=0) == -1                               # no sequences
     assert call(a9=-1) == -1                              # negative token count
     assert call(a10=257) == -1                            # max_pages * page_size < max_seq_len
+    assert call(a10=(1 << 30) + 1, a6=1 << 25) == -1      # max_seq_len beyond 2^30
     assert call(a14=16) == -3                             # too-small workspace
     assert call(a9=0, a1=None, a13=None) == 0             # T == 0 is a no-op
     assert lib.mla_last_launch_count(M.CALL_PREFILL_ATTENTION) == 0
