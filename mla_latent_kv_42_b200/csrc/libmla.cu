@@ -87,7 +87,7 @@ DecodePlan plan_decode(const mla_dims* d, int B, int max_seq_len) {
   const long blocks_wanted = 4L * device_sm_count();
   const long base = (long)B * p.head_groups;
   long s = (blocks_wanted + base - 1) / base;
-  const long by_len = (max_seq_len + 255) / 256;  // at least 256 tokens per split
+  const long by_len = ((long)max_seq_len + 255) / 256;  // at least 256 tokens per split
   if (s > by_len) s = by_len;
   if (s < 1) s = 1;
   p.n_splits = (int)s;
@@ -179,8 +179,17 @@ size_t ws_decode_tc(const mla_dims* d, int B) {
          align256(slots * d->n_heads * 4);
 }
 
+// Pages of the longest sequence; the planner's page counts, summed over a launch, must stay in
+// int32.
+inline long pages_of(const mla_dims* d, int32_t max_seq_len) {
+  return ((long)max_seq_len + d->page_size - 1) / d->page_size;
+}
+inline bool page_total_fits(const mla_dims* d, long items, int32_t max_seq_len) {
+  return items * pages_of(d, max_seq_len) <= (long)INT32_MAX;
+}
+
 size_t ws_decode(const mla_dims* d, int B, int max_seq_len) {
-  if (B <= 0 || max_seq_len <= 0) return 0;
+  if (B <= 0 || max_seq_len < 1 || max_seq_len > kMaxSeqLen) return 0;
   if (decode_tc_eligible(d)) return ws_decode_tc(d, B);
   const DecodePlan p = plan_decode(d, B, max_seq_len);
   if (p.n_splits == 1) return 0;
@@ -285,9 +294,18 @@ int decode_impl(const mla_dims* d, const void* q, const void* pool, int32_t num_
 // (per-token items and split-KV partials) while leaving thousands of attention tiles per launch.
 constexpr int kPrefillGroup = 1024;
 
+// Tokens per launch group: at most kPrefillGroup, and few enough that the group's page count
+// (tokens x pages of the longest sequence) stays in int32.
+inline int prefill_group(const mla_dims* d, int T, int max_seq_len) {
+  long G = T < kPrefillGroup ? T : kPrefillGroup;
+  const long cap = (long)INT32_MAX / pages_of(d, max_seq_len);
+  if (G > cap) G = cap;
+  return G < 1 ? 1 : (int)G;
+}
+
 size_t ws_prefill(const mla_dims* d, int T, int max_seq_len) {
-  if (T <= 0 || max_seq_len <= 0) return 0;
-  const int G = T < kPrefillGroup ? T : kPrefillGroup;
+  if (T <= 0 || max_seq_len < 1 || max_seq_len > kMaxSeqLen) return 0;
+  const int G = prefill_group(d, T, max_seq_len);
   const size_t item_pages = ((size_t)max_seq_len + d->page_size - 1) / d->page_size;
   size_t dec = ws_decode(d, G, max_seq_len);
   if (T % G != 0) {  // the last, smaller group may split sequences further
@@ -301,7 +319,7 @@ template <typename T>
 int prefill_impl(const mla_dims* d, const void* q, const void* pool, int32_t num_pages, const int32_t* bt,
                  int32_t num_seqs, int32_t max_pages, const int32_t* seq_idx, const int32_t* pos, int32_t T_,
                  int32_t max_seq_len, void* o_lat, float* lse_out, void* ws, cudaStream_t st) {
-  const int G = T_ < kPrefillGroup ? T_ : kPrefillGroup;
+  const int G = prefill_group(d, T_, max_seq_len);
   const int item_pages = (int)(((long)max_seq_len + d->page_size - 1) / d->page_size);
   Carve c{static_cast<char*>(ws)};
   int* item_bt = c.take<int>((size_t)G * item_pages);
@@ -412,6 +430,7 @@ int mla_decode_attention(const mla_dims* dims, const void* q, const void* pool, 
   if (B < 0 || B > 65535 || max_seq_len < 1 || max_seq_len > kMaxSeqLen || max_pages <= 0 || num_pages <= 0)
     return MLA_ERR_INVALID_ARG;
   if ((long)max_pages * dims->page_size < (long)max_seq_len) return MLA_ERR_INVALID_ARG;
+  if (!page_total_fits(dims, B, max_seq_len)) return MLA_ERR_INVALID_ARG;
   if (B == 0) {
     t_launches[MLA_CALL_DECODE_ATTENTION] = 0;
     return MLA_OK;
@@ -555,8 +574,12 @@ int mla_decode_attention_noalloc(const mla_dims* dims, const void* q, const void
                                  int32_t max_seq_len, void* o_lat, float* lse_out, mla_stream_t stream) {
   const int r = check_dims_impl(dims);
   if (r != MLA_OK) return r;
-  if (B > 0 && max_seq_len >= 1 && ws_decode(dims, B, max_seq_len) > kStaticScratchBytes)
-    return MLA_ERR_WORKSPACE_TOO_SMALL;
+  // the argument checks of mla_decode_attention come first, so that the size below is defined
+  if (B < 0 || B > 65535 || max_seq_len < 1 || max_seq_len > kMaxSeqLen || max_pages <= 0 || num_pages <= 0)
+    return MLA_ERR_INVALID_ARG;
+  if ((long)max_pages * dims->page_size < (long)max_seq_len || !page_total_fits(dims, B, max_seq_len))
+    return MLA_ERR_INVALID_ARG;
+  if (ws_decode(dims, B, max_seq_len) > kStaticScratchBytes) return MLA_ERR_WORKSPACE_TOO_SMALL;
   void* ws = nullptr;
   const int s = static_scratch_address(&ws);
   if (s != MLA_OK) return s;

@@ -208,3 +208,39 @@ def test_binding_refuses_host_tensors_before_calling_the_library(lib):
         M.prefill_attention(d, q, q, i32.view(1, 3), i32, i32, 4)
     with pytest.raises(ValueError, match="CUDA"):
         M.decode_attention(d, q, q, i32.view(1, 3), i32, 4)
+
+
+def test_page_totals_beyond_int32_are_rejected(lib):
+    """The attention planner sums page counts over a launch in int32: a batch whose worst case
+    (B x pages of max_seq_len) passes INT32_MAX is rejected before anything is queued, by both the
+    workspace and the allocation-free entry point."""
+    cd = dims(synth.PRODUCTION)
+    big = 1 << 30                     # 2^24 pages of 64 tokens
+    args = [ctypes.byref(cd), FAKE, FAKE, 10, FAKE, 1 << 24, FAKE, 128, big, FAKE, None, FAKE, 1 << 40, None]
+    assert lib.mla_decode_attention(*args) == -1           # 128 x 2^24 = 2^31 pages
+    na = [ctypes.byref(cd), FAKE, FAKE, 10, FAKE, 1 << 24, FAKE, 128, big, FAKE, None, None]
+    assert lib.mla_decode_attention_noalloc(*na) == -1
+    na[8] = big + 1                                         # beyond the 2^30 length limit
+    na[7] = 1
+    assert lib.mla_decode_attention_noalloc(*na) == -1
+    na[8] = 0
+    assert lib.mla_decode_attention_noalloc(*na) == -1
+
+
+def test_workspace_size_is_zero_for_out_of_range_lengths(lib):
+    for call in (M.CALL_DECODE_ATTENTION, M.CALL_PREFILL_ATTENTION):
+        for d in (synth.RUNNING, synth.PRODUCTION):
+            assert M.workspace_size(d, call, 4, 2**31 - 1) == 0
+            assert M.workspace_size(d, call, 4, 0) == 0
+
+
+def test_prefill_groups_shrink_to_keep_page_totals_in_int32():
+    """At max_seq_len = 2^30 (2^24 pages) a launch group holds at most INT32_MAX // 2^24 = 127
+    tokens, so the workspace stops growing there instead of at 1024 tokens."""
+    P = synth.PRODUCTION
+    big = 1 << 30
+    a = M.workspace_size(P, M.CALL_PREFILL_ATTENTION, 127, big)
+    assert a > 0
+    assert a == M.workspace_size(P, M.CALL_PREFILL_ATTENTION, 128, big) == M.workspace_size(
+        P, M.CALL_PREFILL_ATTENTION, 4096, big)
+    assert a >= 127 * (1 << 24) * 4
