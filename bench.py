@@ -23,7 +23,6 @@ from __future__ import annotations
 import argparse
 import json
 import os
-import re
 import statistics
 import subprocess
 import sys
@@ -100,9 +99,10 @@ class ClockSampler:
             if len(parts) < 8:
                 continue
             rows.append((ts, parts))
-        inside = [r for r in rows if t0 <= r[0] <= t1] or rows
+        inside = [r for r in rows if t0 <= r[0] <= t1]
         if not inside:
-            return None
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "samples": 0,
+                    "note": "no nvidia-smi sample fell inside the timed region"}
         sm = [float(p[0]) for _, p in inside if p[0].replace(".", "").isdigit()]
         mx = [float(p[1]) for _, p in inside if p[1].replace(".", "").isdigit()]
         names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
@@ -205,21 +205,20 @@ def rank_workload(w, rank: int):
 
 
 def measured_decode_traffic(workload: str):
-    """DRAM bytes (read + write) of one decode-kernel launch from the committed ncu summary, if it was
-    taken on this workload and the kernel source is unchanged since; otherwise None."""
+    """DRAM bytes (read + write) of one attention-kernel launch on this workload, from the table of
+    ncu captures in profiles/decode_tc_traffic.txt (lines ``workload sha256-prefix bytes``), if the
+    capture was taken with the kernel source as it is now; otherwise None."""
     import hashlib
-    prof = os.path.join(ROOT, "profiles", f"ncu_decode_tc_{workload.replace('_bf16', '').replace('_fp16', '')}.md")
+    table = os.path.join(ROOT, "profiles", "decode_tc_traffic.txt")
     src = os.path.join(ROOT, "mla_latent_kv_42_b200", "csrc", "decode_tc.cuh")
-    if not os.path.exists(prof):
+    if not os.path.exists(table):
         return None
-    text = open(prof).read()
-    m_hash = re.search(r"decode_tc.cuh sha256 prefix at capture: ([0-9a-f]+)", text)
-    m_bytes = re.search(r"^traffic_bytes: (\d+)", text, re.M)
-    if not m_hash or not m_bytes:
-        return None
-    if hashlib.sha256(open(src, "rb").read()).hexdigest()[:len(m_hash.group(1))] != m_hash.group(1):
-        return None
-    return int(m_bytes.group(1))
+    digest = hashlib.sha256(open(src, "rb").read()).hexdigest()
+    for line in open(table):
+        parts = line.split()
+        if len(parts) == 3 and not line.startswith("#") and parts[0] == workload and digest.startswith(parts[1]):
+            return int(parts[2])
+    return None
 
 
 def max_over_ranks(values, device, world: int):
@@ -344,24 +343,56 @@ def run_mla(args):
     sampler.start()
     time.sleep(0.3)
 
-    # ---- timed region: K steps, device time, barrier + synchronize on both sides
-    launches[0] = 0
+    # ---- timed region: K steps, device time, barrier + synchronize on both sides. The K-step
+    # region is repeated (at least 3 times, until about half a second has been timed, so that the
+    # clock sampler sees it) and the median repetition is reported; every rank runs the same number
+    # of repetitions (the count is agreed from rank 0's first one).
+    # With --flush-l2 every step runs cold: a 256 MiB write (twice L2) precedes it, outside its
+    # own pair of events, and the region's time is the sum of the steps' times.
+    flush_buf = torch.empty(256 << 20, dtype=torch.uint8, device=dev) if args.flush_l2 else None
+
+    def timed_block():
+        if world > 1:
+            dist.barrier()
+        torch.cuda.synchronize(dev)
+        if flush_buf is not None:
+            total = 0.0
+            evs = []
+            for _ in range(args.steps):
+                flush_buf.fill_(1)
+                a, b = EV(), EV()
+                a.record(stream)
+                one_step()
+                b.record(stream)
+                evs.append((a, b))
+            torch.cuda.synchronize(dev)
+            total = sum(a.elapsed_time(b) for a, b in evs)
+        else:
+            start, end = EV(), EV()
+            start.record(stream)
+            for _ in range(args.steps):
+                one_step()
+            end.record(stream)
+            torch.cuda.synchronize(dev)
+            total = start.elapsed_time(end)
+        if world > 1:
+            dist.barrier()
+        return total
+
     pending.clear()
-    if world > 1:
-        dist.barrier()
-    torch.cuda.synchronize(dev)
     t_wall0 = time.time()
-    start, end = EV(), EV()
-    start.record(stream)
-    for _ in range(args.steps):
-        one_step()
-    end.record(stream)
-    torch.cuda.synchronize(dev)
-    t_wall1 = time.time()
-    if world > 1:
-        dist.barrier()
-    ms_total = start.elapsed_time(end)
+    launches[0] = 0
+    rep_ms = [timed_block()]
     n_timed_launches = launches[0]
+    reps = int(min(args.max_reps, max(3, -(-args.min_timed_s * 1e3 // max(rep_ms[0], 1e-3)))))
+    if world > 1:
+        r_t = torch.tensor([reps], dtype=torch.int64, device=dev)
+        dist.broadcast(r_t, 0)
+        reps = int(r_t.item())
+    while len(rep_ms) < reps:
+        rep_ms.append(timed_block())
+    t_wall1 = time.time()
+    ms_total = float(np.median(rep_ms))
 
     # ---- per-call breakdown, a separate pass: events between the calls stop each call's first
     # kernel from launching early into the previous call's tail, so this pass runs a little
@@ -477,8 +508,13 @@ def run_mla(args):
                                                                          f"{int(cached.sum())}"),
                        "layers": len(layers), "dims": dims_desc(d), "paging": w.paging,
                        **({"chunk": chunk, "new_tokens": T} if chunk > 1 else {}),
-                       "l2": "inputs larger than L2" if sbytes > 126e6 else "L2 not flushed (inputs below L2)",
-                       "parallelism": f"replicas x{world} (sequence-independent, no collective)"},
+                       "l2": ("flushed before every step (256 MiB write, outside the step's events)" if args.flush_l2
+                              else "inputs larger than L2" if sbytes > 126e6 else "L2 not flushed (inputs below L2)"),
+                       "parallelism": f"replicas x{world} (sequence-independent, no collective)",
+                       "timed_reps": len(rep_ms),
+                       "timing": (f"median of {len(rep_ms)} repetitions of the {args.steps}-step timed region "
+                                  f"(min {min(rep_ms) / args.steps * 1e3 / len(layers):.1f}, max "
+                                  f"{max(rep_ms) / args.steps * 1e3 / len(layers):.1f} us per layer-step)")},
             "tflops": sflops / step_s / 1e12,
             "cache_gbs": dbytes / dec_s / 1e9,
             "decode_us": decode_ms * 1e3,
@@ -512,6 +548,10 @@ def main():
     ap.add_argument("--workload", default=DEFAULT_WORKLOAD)
     ap.add_argument("--impl", choices=["mla", "reference"], default="mla")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--min-timed-s", type=float, default=0.5,
+                    help="repeat the K-step timed region until this many seconds are timed (at least 3 times)")
+    ap.add_argument("--max-reps", type=int, default=1000)
+    ap.add_argument("--flush-l2", action="store_true", help="write 256 MiB before every timed step (cold L2)")
     args = ap.parse_args()
     args.warmup = max(3, args.warmup)     # at least 3 untimed warm-up steps
     if args.impl == "reference":

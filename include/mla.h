@@ -13,8 +13,9 @@
  *     row block [i*d_rope, (i+1)*d_rope); head i of W^O its column block [i*d_h, (i+1)*d_h).
  *   - Element type of every activation, weight and cache buffer is dims->dtype (bf16 or
  *     fp16); accumulation is fp32. Results are rounded to the element type to nearest even.
- *   - RoPE rotates adjacent pairs (x[2k], x[2k+1]) by the angle pos * rope_base^(-2k/d_rope),
- *     formed in double precision; positions are 0-based.
+ *   - RoPE rotates adjacent pairs (x[2k], x[2k+1]) by the angle pos * theta_k with
+ *     theta_k = rope_base^(-2k/d_rope) (or the caller's table, mla_dims.rope_inv_freq), formed in
+ *     double precision; positions are 0-based.
  *   - Ownership: the caller owns every buffer. All pointer arguments are DEVICE pointers,
  *     16-byte aligned, on the current device. The library allocates no device memory and
  *     keeps no per-call state besides one device status word per device.
@@ -63,6 +64,13 @@ typedef struct mla_dims {
   int32_t page_size; /* tokens per cache page */
   int32_t dtype;     /* enum mla_dtype */
   double rope_base;  /* RoPE frequency base, e.g. 10000 */
+  /* Optional RoPE frequency table: DEVICE pointer to d_rope/2 doubles theta_k (8-byte aligned),
+   * used in place of rope_base^(-2k/d_rope) by mla_append_kv (k^R) and mla_absorb_query (q^R),
+   * e.g. YaRN-interpolated frequencies for context extension (the velog DeepSeek-V2 review §4.1
+   * applies YaRN to the decoupled key; its constants are not on the pages, so the caller supplies
+   * the table; an amplitude factor of YaRN folds into W^QR and W^KR). NULL: the base formula. The
+   * table must stay valid until the calls that read it have completed. */
+  const double* rope_inv_freq;
 } mla_dims;
 /* The softmax scale is derived, 1/sqrt(d_head + d_rope) (from-scratch page, §4.4). */
 
@@ -87,9 +95,9 @@ enum mla_call {
 };
 
 /* Returns MLA_OK if every call supports `dims`, else MLA_ERR_UNSUPPORTED_DIMS or
- * MLA_ERR_INVALID_ARG. Supported: all widths positive multiples of 8 (d_rope a multiple of 8),
- * n_heads <= 128, d_c <= 512, d_c + d_rope <= 576, page_size >= 1, dtype bf16/fp16,
- * rope_base > 0. */
+ * MLA_ERR_INVALID_ARG (MLA_ERR_ALIGNMENT for a rope_inv_freq table not 8-byte aligned).
+ * Supported: all widths positive multiples of 8 (d_rope a multiple of 8), n_heads <= 128,
+ * d_c <= 512, d_c + d_rope <= 576, page_size >= 1, dtype bf16/fp16, rope_base > 0. */
 int mla_check_dims(const mla_dims* dims);
 
 /* Elements cached per token per layer, d_c + d_rope ("What Gets Cached", from-scratch page

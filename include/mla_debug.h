@@ -30,6 +30,19 @@ extern "C" {
 int mla_debug_gemm_plan(int32_t M, int32_t N, int32_t K, int32_t batch, int32_t fused_rope, int32_t d_rope,
                         int64_t* out);
 
+/* Fault injection for testing the bounded waits (not part of the method). In the library built
+ * with MLA_FAULT_INJECT (libmla_faultinj.so, used only by tests), every wait inside a kernel gives
+ * up after 20 ms instead of 2 s, and this call makes the next mla_decode_attention calls on the
+ * current device leave one cache load unissued: the first latent load of 128-token tile `tile` of
+ * the call's concatenated tile list (the tiles of sequence 0, then of sequence 1, ...; -1: none).
+ * The waits of the SM pair that owns it then run out; its kernel records MLA_ERR_TIMEOUT
+ * in the device status, waits for the loads it did issue, releases its tensor memory and
+ * returns, and later calls on the stream run normally once the injection is cleared (-1). The
+ * output of the call with a missing load is undefined. Returns 0 (set), MLA_ERR_INVALID_ARG in
+ * the regular library (which has no injection) or for tile < -1, MLA_ERR_CUDA if the copy to the
+ * device fails. */
+int mla_debug_inject_missing_load(int32_t tile);
+
 #ifdef __cplusplus
 }
 #endif

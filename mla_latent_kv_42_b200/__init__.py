@@ -38,7 +38,8 @@ class MLAError(RuntimeError):
 class _Dims(ctypes.Structure):
     _fields_ = [("d_model", ctypes.c_int32), ("n_heads", ctypes.c_int32), ("d_head", ctypes.c_int32),
                 ("d_c", ctypes.c_int32), ("d_cq", ctypes.c_int32), ("d_rope", ctypes.c_int32),
-                ("page_size", ctypes.c_int32), ("dtype", ctypes.c_int32), ("rope_base", ctypes.c_double)]
+                ("page_size", ctypes.c_int32), ("dtype", ctypes.c_int32), ("rope_base", ctypes.c_double),
+                ("rope_inv_freq", ctypes.c_void_p)]
 
 
 _LIB = None
@@ -58,6 +59,7 @@ _SIGS = {
     "mla_last_launch_count": (_I32, [_I32]),
     "mla_decode_attention_noalloc": (ctypes.c_int, [_P, _P, _P, _I32, _P, _I32, _P, _I32, _I32, _P, _P, _P]),
     "mla_set_decode_timing_events": (ctypes.c_int, [_P, _P]),
+    "mla_debug_inject_missing_load": (ctypes.c_int, [_I32]),
 }
 
 
@@ -81,10 +83,31 @@ def load_library(path: str | None = None):
 _lib = load_library
 
 
+_ROPE_TABLES = {}
+
+
+def _rope_table_ptr(d):
+    """Device copy (float64, current device) of a dims' RoPE frequency table, or None. The copies are
+    kept for the life of the process so that queued kernels can still read them."""
+    table = getattr(d, "rope_inv_freq", None)
+    if table is None:
+        return None
+    import torch
+    key = (tuple(float(x) for x in table), torch.cuda.current_device())
+    t = _ROPE_TABLES.get(key)
+    if t is None:
+        if len(key[0]) != d.d_rope // 2:
+            raise ValueError(f"rope_inv_freq has {len(key[0])} entries, d_rope/2 = {d.d_rope // 2}")
+        t = torch.tensor(key[0], dtype=torch.float64, device="cuda")
+        _ROPE_TABLES[key] = t
+    return t.data_ptr()
+
+
 def c_dims(d) -> _Dims:
-    """mla_dims from a ``synth.Dims`` (or anything with the same attributes)."""
+    """mla_dims from a ``synth.Dims`` (or anything with the same attributes). A dims with a RoPE
+    frequency table (``rope_inv_freq``, d_rope/2 floats) gets a device copy of it."""
     return _Dims(d.d_model, d.n_heads, d.d_head, d.d_c, d.d_cq, d.d_rope, d.page_size,
-                 {"bf16": 0, "fp16": 1}[d.dtype], float(d.rope_base))
+                 {"bf16": 0, "fp16": 1}[d.dtype], float(d.rope_base), _rope_table_ptr(d))
 
 
 def _ptr(t):

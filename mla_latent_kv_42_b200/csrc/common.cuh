@@ -77,11 +77,12 @@ __device__ __forceinline__ float warp_sum(float v) {
   return v;
 }
 
-// cos/sin of the RoPE angle of pair k at position pos: pos * base^(-2k/d_rope). The angle is
-// formed and reduced in double precision (an fp32 angle at position 131072 would be off by
-// up to ~1e-2 rad); only the final cos/sin are rounded to fp32.
-__device__ __forceinline__ double rope_inv_freq(int k, int d_rope, double base) {
-  return pow(base, -2.0 * (double)k / (double)d_rope);
+// cos/sin of the RoPE angle of pair k at position pos: pos * theta_k, with theta_k from the
+// caller's table when one is given (e.g. YaRN-scaled frequencies), else base^(-2k/d_rope). The
+// angle is formed and reduced in double precision (an fp32 angle at position 131072 would be off
+// by up to ~1e-2 rad); only the final cos/sin are rounded to fp32.
+__device__ __forceinline__ double rope_inv_freq(int k, int d_rope, double base, const double* table) {
+  return table != nullptr ? table[k] : pow(base, -2.0 * (double)k / (double)d_rope);
 }
 __device__ __forceinline__ void rope_cos_sin_at(int pos, double inv_freq, float& c, float& s) {
   double sd, cd;
@@ -89,8 +90,9 @@ __device__ __forceinline__ void rope_cos_sin_at(int pos, double inv_freq, float&
   c = (float)cd;
   s = (float)sd;
 }
-__device__ __forceinline__ void rope_cos_sin(int pos, int k, int d_rope, double base, float& c, float& s) {
-  rope_cos_sin_at(pos, rope_inv_freq(k, d_rope, base), c, s);
+__device__ __forceinline__ void rope_cos_sin(int pos, int k, int d_rope, double base, const double* table, float& c,
+                                             float& s) {
+  rope_cos_sin_at(pos, rope_inv_freq(k, d_rope, base, table), c, s);
 }
 
 // Launch `kern` on `st` with programmatic stream serialization: it may begin while the

@@ -1,18 +1,30 @@
-// Latent attention on tcgen05 for DeepSeek-V2 dims (n_h <= 128 heads, d_c = 512, d_h^R = 64,
+// Latent attention on tcgen05 for DeepSeek-V2 dims (65..128 heads, d_c = 512, d_h^R = 64,
 // 64-token pages): "DeepSeek-V2 from Scratch" §4.4 with the absorbed steps 2-3 of §5.3.
 //
-// For 128 heads the fp32 accumulator O = sum_j p_j c_j is 128 x 512 x 4 B = 256 KB, all of
-// one SM's tensor memory, so one work unit runs on a cluster of two CTAs:
-//   score CTA (rank 0): Q [128 x 576] lives in TMEM as the A operand; S = Q C^T for each
-//     64-token page (36 MMAs of K = 16, N = 64) from TMA-loaded 64 x 64 chunks; four warps
-//     run the online softmax in fp32 (one head per thread, lazy rescaling: the reference
-//     max moves only when a score exceeds it by 2^8) and write P (bf16) and the per-head
-//     rescale factor straight into the value CTA's shared memory.
-//   value CTA (rank 1): O in TMEM (512 columns); O += P C_lat per page (two N = 256
-//     halves, C_lat read MN-major from TMA-loaded chunks); four warps apply rescales and
-//     write the result (or a split-KV partial) out.
-// The pages of all sequences are split evenly over the clusters; a sequence that spans
-// clusters is merged afterwards by log-sum-exp in a fixed order.
+// A work unit is a pair of CTAs (a 2-CTA cluster, one TPC) that shares every MMA (tcgen05
+// cta_group::2, M = 128). CTA r owns heads [64r, 64r + 64): their absorbed queries Q_r
+// [64 x 576] sit in its shared memory and their fp32 accumulator O_r [64 x 512] in its tensor
+// memory (256 columns). Cached tokens go in 128-token tiles of two pages:
+//   S = Q C^T      N = 128 tokens. CTA r supplies page r of the tile, all 576 columns; each CTA
+//                  receives its 64 heads x 128 tokens (TMEM lanes 0-63: page 0, 64-127: page 1).
+//   softmax        eight warps per CTA, four threads per head (two pages x two halves of 32
+//                  tokens), online in fp32 with lazy rescaling (the reference max moves only
+//                  when a score exceeds it by 2^8); P (bf16) is written to shared memory.
+//   O += P C_lat   N = 256 latent columns per MMA, two of them: CTA r supplies columns
+//                  [256j + 128r, 256j + 128r + 128) of all 128 tokens.
+// So CTA r reads its own page whole and only the latent half it supplies of the other page:
+// 1.44x the unique bytes per SM, against 2x for two SMs that each stream whole pages. The own
+// page's latent half stays in shared memory from S to O, and the other page's half is loaded
+// into the slots that the own page's remaining latent half held during S.
+//
+// Shared memory (per CTA): Q (9 chunks of 64 rows x 64 columns, 128-byte swizzle), P (two
+// chunks: 64 heads x the tokens of page g), one rope slot (the own page's k^R columns, shared by
+// consecutive tiles) and two sets of 8 latent chunks (tile i uses set i & 1). Latent chunks
+// 2p and 2p+1 of a set form pair p = 2j + g: during S they hold the own page's columns
+// [128p, 128p + 128); during O they hold the columns CTA r supplies for n-half j of page g.
+//
+// The pages of all sequences are split evenly over the pairs by 128-token tile; a sequence that
+// spans pairs is merged afterwards by log-sum-exp in a fixed order.
 #pragma once
 
 #include "tc_common.cuh"
@@ -20,60 +32,67 @@
 namespace mla {
 namespace tc {
 
+#ifdef MLA_FAULT_INJECT
+// Fault-injection test builds only: the global tile (index in the concatenated tile list of the
+// call) whose first latent load the rank-0 loader of its pair leaves unissued, after arming its
+// barrier; -1 = none. The S MMAs then wait for bytes that never come, and every role of the pair
+// gives up after the build's short wait limit. Set with mla_debug_inject_missing_load.
+__device__ int g_inject_missing_tile = -1;
+#endif
+
 namespace dec {
-constexpr int kPage = 64;         // tokens per cache page
-constexpr int kTile = 128;        // tokens per tile: two pages (S = Q C^T with N = 128)
-constexpr int kDc = 512;          // latent width (O columns)
-constexpr int kD = 576;           // cache row width
-constexpr int kChunk = 8192;      // one 64 x 64 box of 16-bit elements
-constexpr int kPair = 2 * kChunk;  // column chunk kc of both pages of a tile, rows 0-63 then 64-127
-constexpr int kScoreSlots = 8;    // score ring: 8 x 16 KB
-constexpr int kValSlots = 4;      // value ring: 4 x 32 KB (one page's half latent: 4 chunks)
-constexpr int kPBufs = 2;         // P buffers in the value CTA
-constexpr int kPTile = 2 * 16384;  // P tile: 128 heads x 128 tokens bf16, two 64-token swizzled halves
-constexpr int kPBytes = kPTile + 512;  // + 128 rescale factors
-constexpr int kPStride = 33792;   // 1024-aligned stride of P buffers / staging buffers
-constexpr int kStg = 2;           // score CTA: P staging buffers
-constexpr int kStageOff = kScoreSlots * kPair;   // score CTA: kStg staging buffers
-constexpr int kPOff = kValSlots * 4 * kChunk;    // value CTA: kPBufs P buffers
-constexpr float kLazy = 8.f;      // rescale threshold in log2 units
-constexpr int kDataBytes = 204800;
-static_assert(kStageOff + kStg * kPStride <= kDataBytes, "score layout");
-static_assert(kPOff + kPBufs * kPStride <= kDataBytes, "value layout");
-constexpr int kThreads = 224;     // 7 warps
+constexpr int kPage = 64;          // tokens per cache page
+constexpr int kTile = 128;         // tokens per tile: page r of it is supplied by CTA r
+constexpr int kDc = 512;           // latent width (O columns)
+constexpr int kD = 576;            // cache row width
+constexpr int kChunk = 8192;       // 64 rows x 64 columns of 16-bit elements
+constexpr int kQOff = 0;           // Q: 9 chunks
+constexpr int kPOff = 9 * kChunk;  // P: 2 chunks (tokens of page 0, of page 1)
+constexpr int kRopeOff = kPOff + 2 * kChunk;  // own page's k^R columns
+constexpr int kSetOff = kRopeOff + kChunk;    // two sets of 8 latent chunks
+constexpr int kSetBytes = 8 * kChunk;
+constexpr int kDataBytes = kSetOff + 2 * kSetBytes;  // 229376
+constexpr float kLazy = 8.f;       // rescale threshold in log2 units
+constexpr int kSoftWarps = 8;      // warps 0-7: softmax, rescale, epilogue
+constexpr int kLoadWarp = 8;       // Q, rope and own-page latent loads
+constexpr int kMmaWarp = 9;        // TMEM allocation; rank 0: MMA issue
+constexpr int kPairWarp = 10;      // the other page's latent half; tail tiles' row clearing
+constexpr int kThreads = 11 * 32;
 // TMEM columns
-constexpr uint32_t kSCol = 0;     // score: S, 128 columns
-constexpr uint32_t kQCol = 128;   // score: Q, 288 columns
-constexpr uint32_t kOCol = 0;     // value: O, 512 columns
+constexpr uint32_t kOCol = 0;      // O: n-half j in columns [128j, 128j + 128)
+constexpr uint32_t kSCol = 256;    // S buffer b in columns [256 + 64b, 320 + 64b)
 constexpr uint32_t kTmemCols = 512;
 
 struct Ctrl {
-  uint64_t full[kScoreSlots];
-  uint64_t empty[kScoreSlots];
-  uint64_t s_full, s_empty, q_ready;
-  uint64_t stg_ready[kStg], stg_free[kStg];  // score CTA: staging buffers (softmax warps <-> sender warp)
-  uint64_t p_empty[kPBufs];  // score CTA; arrived by the value CTA's multicast commit
-  uint64_t stats_empty;      // score CTA; arrived remotely by the value CTA
-  uint64_t p_full[kPBufs];   // value CTA; armed and completed by the score CTA's bulk copy
-  uint64_t p_ready[kPBufs];  // value CTA
-  // value CTA: O complete through the last tile that used P buffer pb. One barrier per P buffer
-  // keeps every parity wait on it at most one phase behind: the P ring only guarantees that the
-  // MMAs of tile t-2 are done when tile t's P arrives, so one shared barrier could lag by two.
-  uint64_t o_done[kPBufs];
-  uint64_t stats_full, o_free, drain;
-  float stats[128][2];       // value CTA: reference max (log2 units) and denominator
+  // Barriers arrived by both CTAs (two arrivals, plus the TMA bytes) live in rank 0, the issuer.
+  uint64_t qk_full[2][2];  // set s, chunks [4h, 4h + 4) of the own page loaded in both CTAs
+  uint64_t pv_full[2][4];  // set s, pair p ready for O in both CTAs
+  uint64_t rope_full, q_full;
+  uint64_t s_free[2];      // S buffer b read by all 16 softmax warps
+  uint64_t p_full;         // P written (and O rescaled) by all 16 softmax warps
+  uint64_t o_free;         // O read out by all 16 softmax warps (end of a sequence's item)
+  // Barriers arrived by rank 0's MMA commits, multicast to both CTAs.
+  uint64_t qk_done[2][4];  // set s, the S MMAs of pair p are complete (its slots may be reused)
+  uint64_t set_free[2];    // the O MMAs of the tile using set s are complete
+  uint64_t rope_done, q_free;
+  uint64_t s_full[2], p_free;
+  // Local barriers.
+  uint64_t fix_full[2][4];  // tail tiles: this CTA's own load of pair p
+  uint64_t xm_full, xm_free;  // exchange of per-thread partial maxima / sums among the softmax warps
+  uint64_t drain;
+  float xm[2][128];          // [column half][TMEM lane]
   uint32_t tmem_slot;
   int abort_flag;
 };
 constexpr size_t kSmem = 1024 + kDataBytes + sizeof(Ctrl);
+static_assert(kSmem <= 232448, "decode kernel shared memory");
 }  // namespace dec
 
 struct DecodeTcParams {
-  const void* q;          // [B, n_h, 576]
   const int* bt;          // [B, max_pages]
   int max_pages;
   const int* seq_lens;    // [B]
-  const int* tile_prefix;  // [B + 1] pages before each sequence (0 pages for a rejected one)
+  const int* tile_prefix;  // [B + 1] 128-token tiles before each sequence (0 tiles for a rejected one)
   int B, n_h;
   float scale_log2;       // log2(e) / sqrt(d_h + d_h^R)
   void* o_lat;            // [B, n_h, 512] element type
@@ -82,7 +101,14 @@ struct DecodeTcParams {
   float* lse_part;        // [B + C][n_h]
 };
 
-// Pages [t0, t1) of sequence b handled by this cluster (n_b = pages of the sequence).
+// Tensor maps of the attention kernel: the paged pool viewed as [pages * 64 rows, 576] with one
+// 64 x 64 box (rope), and as (64 columns, rows, 9 column chunks) with boxes of 2 and 4 chunks;
+// the queries viewed as (64 columns, B * n_h rows, 9 chunks) with a box of 9 chunks.
+struct DecodeTcMaps {
+  CUtensorMap pool1, pool2, pool4, q9;
+};
+
+// Tiles [t0, t1) of sequence b handled by this pair (n_b = tiles of the sequence).
 struct Item {
   int b, t0, t1, n_b;
 };
@@ -116,12 +142,55 @@ __device__ __forceinline__ bool next_item(ItemIter& it, const int* prefix, Item&
   return true;
 }
 
-// Cluster owning global page g when T pages are split over C clusters as [T c / C, T (c+1) / C).
+// The pair's tiles in order. Every role walks the same sequence with a cursor of its own:
+// ti counts the pair's tiles, ii its items, t is the tile within sequence item.b (tokens
+// [128t, 128t + 128)).
+struct Cursor {
+  ItemIter it;
+  Item item;
+  int t, ti, ii;
+  bool valid;
+  __device__ __forceinline__ void start(const int* prefix, int B, int cluster, int nclusters) {
+    it = item_iter(prefix, B, cluster, nclusters);
+    valid = next_item(it, prefix, item);
+    t = valid ? item.t0 : 0;
+    ti = 0;
+    ii = 0;
+  }
+  __device__ __forceinline__ bool first() const { return t == item.t0; }
+  __device__ __forceinline__ bool last() const { return t + 1 == item.t1; }
+  __device__ __forceinline__ void advance(const int* prefix) {
+    ++ti;
+    if (++t == item.t1) {
+      ++ii;
+      valid = next_item(it, prefix, item);
+      if (valid) t = item.t0;
+    }
+  }
+};
+
+// Pair that owns global tile g when T tiles are split over C pairs as [T c / C, T (c+1) / C).
 __device__ __forceinline__ int cluster_of(long g, long T, int C) { return (int)(((g + 1) * C - 1) / T); }
+
+__device__ __forceinline__ void tma_load_3d(uint32_t dst, const CUtensorMap* map, uint32_t bar, int x, int y, int z) {
+  asm volatile(
+      "cp.async.bulk.tensor.3d.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%3, %4, %5}], [%2];" ::"r"(
+          dst),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(bar), "r"(x), "r"(y), "r"(z)
+      : "memory");
+}
+__device__ __forceinline__ void tma_load_3d_pair(uint32_t dst, const CUtensorMap* map, uint32_t cluster_bar, int x,
+                                                 int y, int z) {
+  asm volatile(
+      "cp.async.bulk.tensor.3d.cta_group::2.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%3, %4, "
+      "%5}], [%2];" ::"r"(dst),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(cluster_bar), "r"(x), "r"(y), "r"(z)
+      : "memory");
+}
 
 template <typename T>
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(dec::kThreads, 1)
-    k_decode_tc(const __grid_constant__ CUtensorMap pool_map, const DecodeTcParams p) {
+    k_decode_tc(const __grid_constant__ DecodeTcMaps maps, const DecodeTcParams p) {
   using namespace dec;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* data = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -129,39 +198,40 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(dec::kThreads, 1)
   volatile int* abort_flag = &ctl->abort_flag;
   const uint32_t data_u32 = smem_u32(data);
   const uint32_t rank = cluster_ctarank();
-  const uint32_t peer = rank ^ 1u;
   const int cluster = (int)cluster_id_x(), nclusters = (int)num_clusters_x();
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   auto bar = [&](uint64_t& b) { return smem_u32(&b); };
+  auto lead = [&](uint64_t& b) { return mapa(smem_u32(&b), 0u); };  // the barrier in rank 0
+  constexpr bool kBf16 = IsBf16<T>::value;
 
   if (threadIdx.x == 0) {
-    for (int i = 0; i < kScoreSlots; ++i) {
-      mbar_init(bar(ctl->full[i]), 1);
-      mbar_init(bar(ctl->empty[i]), 1);
+    for (int s = 0; s < 2; ++s) {
+      for (int h = 0; h < 2; ++h) mbar_init(bar(ctl->qk_full[s][h]), 2);
+      for (int q = 0; q < 4; ++q) {
+        mbar_init(bar(ctl->pv_full[s][q]), 2);
+        mbar_init(bar(ctl->qk_done[s][q]), 1);
+        mbar_init(bar(ctl->fix_full[s][q]), 1);
+      }
+      mbar_init(bar(ctl->s_free[s]), 2 * kSoftWarps);
+      mbar_init(bar(ctl->set_free[s]), 1);
+      mbar_init(bar(ctl->s_full[s]), 1);
     }
-    mbar_init(bar(ctl->s_full), 1);
-    mbar_init(bar(ctl->s_empty), 128);
-    for (int i = 0; i < kStg; ++i) {
-      mbar_init(bar(ctl->stg_ready[i]), 128);
-      mbar_init(bar(ctl->stg_free[i]), 1);
-    }
-    mbar_init(bar(ctl->q_ready), 128);
-    for (int i = 0; i < kPBufs; ++i) {
-      mbar_init(bar(ctl->p_empty[i]), 1);
-      mbar_init(bar(ctl->p_full[i]), 1);
-      mbar_init(bar(ctl->p_ready[i]), 128);
-      mbar_init(bar(ctl->o_done[i]), 1);
-    }
-    mbar_init(bar(ctl->stats_empty), 128);
-    mbar_init(bar(ctl->stats_full), 128);
-    mbar_init(bar(ctl->o_free), 128);
+    mbar_init(bar(ctl->rope_full), 2);
+    mbar_init(bar(ctl->q_full), 2);
+    mbar_init(bar(ctl->p_full), 2 * kSoftWarps);
+    mbar_init(bar(ctl->o_free), 2 * kSoftWarps);
+    mbar_init(bar(ctl->rope_done), 1);
+    mbar_init(bar(ctl->q_free), 1);
+    mbar_init(bar(ctl->p_free), 1);
+    mbar_init(bar(ctl->xm_full), kSoftWarps);
+    mbar_init(bar(ctl->xm_free), kSoftWarps);
     mbar_init(bar(ctl->drain), 1);
     ctl->abort_flag = 0;
     fence_mbar_init();
   }
-  if (warp == 5) {
-    tmem_alloc(smem_u32(&ctl->tmem_slot), kTmemCols);
-    tmem_relinquish();
+  if (warp == kMmaWarp) {
+    tmem_alloc2(smem_u32(&ctl->tmem_slot), kTmemCols);
+    tmem_relinquish2();
   }
   tc_fence_before();
   __syncthreads();
@@ -171,465 +241,433 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(dec::kThreads, 1)
   const uint32_t tmem = ctl->tmem_slot;
   if (threadIdx.x == 0) griddep_launch();
   griddep_wait();  // the plan, the query and the cache come from earlier kernels
+  const int* prefix = p.tile_prefix;
   const bool has_work = [&] {
-    const long T_ = p.tile_prefix[p.B];
+    const long T_ = prefix[p.B];
     return T_ * (cluster + 1) / nclusters > T_ * cluster / nclusters;
   }();
-  const uint32_t peer_abort = mapa(smem_u32(&ctl->abort_flag), peer);
-  // A wait that gives up also releases the peer CTA's waiters.
+  const uint32_t peer_abort = mapa(smem_u32(&ctl->abort_flag), rank ^ 1u);
+  // A wait that gives up also releases the peer CTA's waiters. The warp-uniform variant is for
+  // warps whose lanes then run warp-collective instructions: a give-up seen by any lane is taken
+  // by the whole warp.
   auto wait = [&](uint64_t& b, uint32_t parity) {
     if (mbar_wait(bar(b), parity, abort_flag)) return true;
     st_cluster_u32(peer_abort, 1u);
     return false;
   };
-  auto wait_cl = [&](uint64_t& b, uint32_t parity) {
-    if (mbar_wait_cluster(bar(b), parity, abort_flag)) return true;
-    st_cluster_u32(peer_abort, 1u);
-    return false;
-  };
-  // Warp-uniform variants for warps whose lanes all wait and then run warp-collective
-  // instructions: a give-up seen by any lane is taken by the whole warp.
   auto wwait = [&](uint64_t& b, uint32_t parity) {
     const bool ok = __all_sync(0xffffffffu, mbar_wait(bar(b), parity, abort_flag));
     if (!ok && lane == 0) st_cluster_u32(peer_abort, 1u);
     return ok;
   };
-  auto wwait_cl = [&](uint64_t& b, uint32_t parity) {
-    const bool ok = __all_sync(0xffffffffu, mbar_wait_cluster(bar(b), parity, abort_flag));
-    if (!ok && lane == 0) st_cluster_u32(peer_abort, 1u);
-    return ok;
-  };
-  constexpr bool kBf16 = IsBf16<T>::value;
+  const uint32_t set_u32 = data_u32 + kSetOff;
 
   if (has_work) {
-    if (rank == 0) {
-      // =========================================================== score CTA
-      if (warp == 4) {  // ---------------- TMA producer: chunk kc (64 columns) of both pages of a tile
-        if (lane == 0) {
-          tma_prefetch_map(&pool_map);
-          int slot_i = 0;
-          bool ok = true;
-          ItemIter it = item_iter(p.tile_prefix, p.B, cluster, nclusters);
-          Item item;
-          while (ok && next_item(it, p.tile_prefix, item)) {
-            const int* btb = p.bt + (long)item.b * p.max_pages;
-            int page_a = btb[item.t0];
-            int page_b = item.t0 + 1 < item.t1 ? btb[item.t0 + 1] : -1;
-            for (int t = item.t0; ok && t < item.t1; t += 2) {
-              const int next_a = t + 2 < item.t1 ? btb[t + 2] : 0;  // read ahead of their use
-              const int next_b = t + 3 < item.t1 ? btb[t + 3] : -1;
-              for (int kc = 0; kc < 9; ++kc, ++slot_i) {
-                const int s = slot_i % kScoreSlots;
-                if (!wait(ctl->empty[s], ((slot_i / kScoreSlots) & 1) ^ 1)) {
-                  ok = false;
-                  break;
-                }
-                mbar_arrive_expect_tx(bar(ctl->full[s]), page_b >= 0 ? kPair : kChunk);
-                tma_load_2d(data_u32 + s * kPair, &pool_map, bar(ctl->full[s]), kc * 64, page_a * kPage);
-                if (page_b >= 0)
-                  tma_load_2d(data_u32 + s * kPair + kChunk, &pool_map, bar(ctl->full[s]), kc * 64, page_b * kPage);
-              }
-              page_a = next_a;
-              page_b = next_b;
+    if (warp == kLoadWarp) {
+      // ---------------------------------------------------------------- Q, rope and own-page loads
+      if (lane == 0) {
+        tma_prefetch_map(&maps.pool1);
+        tma_prefetch_map(&maps.pool2);
+        tma_prefetch_map(&maps.pool4);
+        tma_prefetch_map(&maps.q9);
+        Cursor c;
+        c.start(prefix, p.B, cluster, nclusters);
+        while (c.valid) {
+          const int s = c.ti & 1, b = c.item.b, t = c.t;
+          const int L = p.seq_lens[b];
+          if (c.first()) {  // this CTA's 64 heads of the sequence's queries, after the last S MMA of the item before
+            if (!wait(ctl->q_free, (c.ii & 1) ^ 1)) break;
+            mbar_arrive_expect_tx_remote(lead(ctl->q_full), 9 * kChunk);
+            tma_load_3d_pair(data_u32 + kQOff, &maps.q9, lead(ctl->q_full), 0, b * p.n_h + 64 * (int)rank, 0);
+          }
+          const bool own = kTile * t + kPage * (int)rank < L;  // page r of the tile holds tokens
+          const int page = own ? p.bt[(long)b * p.max_pages + 2 * t + (int)rank] : 0;
+          if (!wait(ctl->rope_done, (c.ti & 1) ^ 1)) break;
+          if (own) {
+            mbar_arrive_expect_tx_remote(lead(ctl->rope_full), kChunk);
+            tma_load_2d_pair(data_u32 + kRopeOff, &maps.pool1, lead(ctl->rope_full), kDc, page * kPage);
+          } else {
+            mbar_arrive_remote(lead(ctl->rope_full));
+          }
+          if (!wait(ctl->set_free[s], ((c.ti >> 1) & 1) ^ 1)) break;  // the O MMAs of tile ti - 2 are done
+          for (int h = 0; h < 2; ++h) {
+#ifdef MLA_FAULT_INJECT
+            if (own && h == 0 && rank == 0 && prefix[b] + t == g_inject_missing_tile) {
+              mbar_arrive_expect_tx_remote(lead(ctl->qk_full[s][h]), 4 * kChunk);
+              continue;
+            }
+#endif
+            if (own) {
+              mbar_arrive_expect_tx_remote(lead(ctl->qk_full[s][h]), 4 * kChunk);
+              tma_load_3d_pair(set_u32 + s * kSetBytes + 4 * h * kChunk, &maps.pool4, lead(ctl->qk_full[s][h]), 0,
+                               page * kPage, 4 * h);
+            } else {
+              mbar_arrive_remote(lead(ctl->qk_full[s][h]));
             }
           }
-          if (!ok)  // copies in flight must land before the CTA exits
-            for (int i = max(0, slot_i - kScoreSlots); i < slot_i; ++i)
-              mbar_wait_slow<false>(bar(ctl->full[i % kScoreSlots]), (i / kScoreSlots) & 1, nullptr);
+          c.advance(prefix);
         }
-        __syncwarp();
-      } else if (warp == 5) {  // ---------------- MMA issue: S = Q C^T, 128 heads x 128 tokens
-        if (lane == 0) {
-          const uint32_t idesc = idesc_f16(128, kTile, kBf16, false, false);
-          int slot_i = 0, tile = 0, item_i = 0;
-          bool ok = true;
-          ItemIter it = item_iter(p.tile_prefix, p.B, cluster, nclusters);
-          Item item;
-          while (ok && next_item(it, p.tile_prefix, item)) {
-            if (!wait(ctl->q_ready, item_i & 1)) break;
-            tc_fence_after();
-            for (int t = item.t0; ok && t < item.t1; t += 2, ++tile) {
-              if (!wait(ctl->s_empty, (tile & 1) ^ 1)) {
+      }
+      __syncwarp();
+    } else if (warp == kPairWarp) {
+      // ---------------------------------------------------------------- the other page's latent half
+      // Pair p = 2j + g of set s holds, for O, the columns this CTA supplies for n-half j of page
+      // g. Page g = r is already there (loaded for S); page 1 - r is loaded once S is done with
+      // the own page's columns in those slots. In a tail tile (the sequence ends inside it) rows
+      // past the end may hold anything (even NaN): this warp zeroes them in both pages, loading
+      // the other page's half to a local barrier first.
+      Cursor c;
+      c.start(prefix, p.B, cluster, nclusters);
+      uint32_t fix_par = 0;
+      bool ok = true;
+      while (ok && c.valid) {
+        const int s = c.ti & 1, b = c.item.b, t = c.t;
+        const int L = p.seq_lens[b];
+        const uint32_t ph = (c.ti >> 1) & 1;
+        const int* btb = p.bt + (long)b * p.max_pages;
+        // the O MMAs of tile ti - 2 are complete, so every barrier of set s is in this tile's phase
+        if (!wwait(ctl->set_free[s], ph ^ 1)) break;
+        if (kTile * (t + 1) <= L) {  // whole tile
+          if (lane == 0) {
+            mbar_arrive_remote(lead(ctl->pv_full[s][(int)rank]));      // j = 0, g = r
+            mbar_arrive_remote(lead(ctl->pv_full[s][2 + (int)rank]));  // j = 1, g = r
+          }
+          const int g = 1 - (int)rank;
+          const int page = btb[2 * t + g];
+          for (int j = 0; j < 2; ++j) {
+            const int pr = 2 * j + g;
+            if (!wwait(ctl->qk_done[s][pr], ph)) {
+              ok = false;
+              break;
+            }
+            if (lane == 0) {
+              mbar_arrive_expect_tx_remote(lead(ctl->pv_full[s][pr]), 2 * kChunk);
+              tma_load_3d_pair(set_u32 + s * kSetBytes + 2 * pr * kChunk, &maps.pool2, lead(ctl->pv_full[s][pr]), 0,
+                               page * kPage, 4 * j + 2 * (int)rank);
+            }
+          }
+        } else {  // tail tile
+          for (int g = 0; ok && g < 2; ++g)
+            for (int j = 0; j < 2; ++j) {
+              const int pr = 2 * j + g;
+              if (!wwait(ctl->qk_done[s][pr], ph)) {
                 ok = false;
                 break;
               }
+              const int nv = max(0, min(kPage, L - kTile * t - kPage * g));  // valid rows of page g
+              const uint32_t slot = set_u32 + s * kSetBytes + 2 * pr * kChunk;
+              if (g != (int)rank && nv > 0) {
+                const int fb = s * 4 + pr;
+                if (lane == 0) {
+                  mbar_arrive_expect_tx(bar(ctl->fix_full[s][pr]), 2 * kChunk);
+                  tma_load_3d(slot, &maps.pool2, bar(ctl->fix_full[s][pr]), 0, btb[2 * t + g] * kPage,
+                              4 * j + 2 * (int)rank);
+                }
+                if (!wwait(ctl->fix_full[s][pr], (fix_par >> fb) & 1u)) {
+                  ok = false;
+                  break;
+                }
+                fix_par ^= 1u << fb;
+              }
+              uint8_t* sp = data + (slot - data_u32);
+              const int per = (kPage - nv) * 8;  // 16-byte units to clear per chunk
+              for (int e = lane; e < 2 * per; e += 32) {
+                const int ch = e / per, rem = e - ch * per;
+                *reinterpret_cast<uint4*>(sp + ch * kChunk + (nv + (rem >> 3)) * 128 + (rem & 7) * 16) =
+                    make_uint4(0, 0, 0, 0);
+              }
+              fence_proxy_async_cta();
+              __syncwarp();
+              if (lane == 0) mbar_arrive_remote(lead(ctl->pv_full[s][pr]));
+            }
+        }
+        c.advance(prefix);
+      }
+    } else if (warp == kMmaWarp) {
+      // ---------------------------------------------------------------- MMA issue (rank 0, one lane)
+      // Two cursors: S MMAs of tile qc (rope chunk, then the 8 latent chunks) and O MMAs of tile
+      // pc < qc (pairs in the order (g, j) = (0,0), (0,1), (1,0), (1,1)). Whichever step is ready
+      // is issued, the O step first, so that a tile's sets are freed as early as possible.
+      if (rank == 0 && lane == 0) {
+        const uint32_t idesc_qk = idesc_f16(128, kTile, kBf16, false, false);
+        const uint32_t idesc_pv = idesc_f16(128, 256, kBf16, false, true);
+        Cursor qc, pc;
+        qc.start(prefix, p.B, cluster, nclusters);
+        pc.start(prefix, p.B, cluster, nclusters);
+        int cq = 0, gq = 0;
+        uint64_t t_idle = globaltimer();
+        while (qc.valid || pc.valid) {
+          bool did = false;
+          if (pc.valid && (!qc.valid || pc.ti < qc.ti)) {
+            const int s = pc.ti & 1, g = gq >> 1, j = gq & 1, pr = 2 * j + g;
+            bool ready = mbar_test_cluster(bar(ctl->pv_full[s][pr]), (pc.ti >> 1) & 1);
+            if (ready && gq == 0)
+              ready = mbar_test_cluster(bar(ctl->p_full), pc.ti & 1) &&
+                      (!pc.first() || mbar_test_cluster(bar(ctl->o_free), (pc.ii & 1) ^ 1));
+            if (ready) {
               tc_fence_after();
-              for (int kc = 0; kc < 9; ++kc, ++slot_i) {
-                const int s = slot_i % kScoreSlots;
-                if (!wait(ctl->full[s], (slot_i / kScoreSlots) & 1)) {
-                  ok = false;
-                  break;
-                }
-                tc_fence_after();
-                const uint32_t sa = data_u32 + s * kPair;
+              const uint32_t pa = data_u32 + kPOff + g * kChunk;
+              const uint32_t vb = set_u32 + s * kSetBytes + 2 * pr * kChunk;
 #pragma unroll
-                for (int ks = 0; ks < 4; ++ks)
-                  mma_ts(tmem + kSCol, tmem + kQCol + kc * 32 + ks * 8, desc_sw128(sa + ks * 32, 16, 1024), idesc,
-                         (kc | ks) != 0);
-                mma_commit(bar(ctl->empty[s]));
+              for (int ks = 0; ks < 4; ++ks)
+                mma2_ss(tmem + kOCol + 128 * j, desc_sw128(pa + ks * 32, 16, 1024),
+                        desc_sw128(vb + ks * 2048, kChunk, 1024), idesc_pv, !(pc.first() && g == 0 && ks == 0));
+              if (++gq == 4) {
+                gq = 0;
+                mma_commit2(bar(ctl->p_free), 3);
+                mma_commit2(bar(ctl->set_free[s]), 3);
+                pc.advance(prefix);
               }
-              if (ok) mma_commit(bar(ctl->s_full));
-            }
-            ++item_i;
-          }
-        }
-        __syncwarp();
-      } else if (warp == 6) {  // ---------------- sender: staged P tiles -> value CTA, one bulk copy each
-        if (lane == 0) {
-          int tile = 0;
-          bool ok = true;
-          ItemIter it = item_iter(p.tile_prefix, p.B, cluster, nclusters);
-          Item item;
-          while (ok && next_item(it, p.tile_prefix, item)) {
-            for (int t = item.t0; t < item.t1; t += 2, ++tile) {
-              const int sb = tile % kStg, pb = tile % kPBufs;
-              if (!wait(ctl->stg_ready[sb], (tile / kStg) & 1) ||
-                  !wait_cl(ctl->p_empty[pb], ((tile / kPBufs) & 1) ^ 1)) {
-                ok = false;
-                break;
-              }
-              const uint32_t full_remote = mapa(bar(ctl->p_full[pb]), 1u);
-              mbar_arrive_expect_tx_remote(full_remote, kPBytes);
-              bulk_copy_to_peer(mapa(data_u32 + kPOff + pb * kPStride, 1u), data_u32 + kStageOff + sb * kPStride,
-                                kPBytes, full_remote);
-              bulk_commit_group();
-              bulk_wait_read<1>();  // the previous tile's staging buffer has been read: hand it back
-              if (tile > 0) mbar_arrive(bar(ctl->stg_free[(tile - 1) % kStg]));
+              did = true;
             }
           }
-          bulk_wait<0>();
-          // The value CTA's last commits arrive on p_empty asynchronously: let them land first.
-          if (ok)
-            for (int j = max(0, tile - kPBufs); j < tile; ++j)
-              if (!wait_cl(ctl->p_empty[j % kPBufs], (j / kPBufs) & 1)) break;
+          if (!did && qc.valid) {
+            const int s = qc.ti & 1, sb = qc.ti & 1;
+            bool ready = true;
+            if (cq == 0)
+              ready = mbar_test_cluster(bar(ctl->rope_full), qc.ti & 1) &&
+                      mbar_test_cluster(bar(ctl->s_free[sb]), ((qc.ti >> 1) & 1) ^ 1) &&
+                      (!qc.first() || mbar_test_cluster(bar(ctl->q_full), qc.ii & 1));
+            else if (cq == 1 || cq == 5)
+              ready = mbar_test_cluster(bar(ctl->qk_full[s][(cq - 1) >> 2]), (qc.ti >> 1) & 1);
+            if (ready) {
+              tc_fence_after();
+              const int kc = cq == 0 ? 8 : cq - 1;
+              const uint32_t bsl = cq == 0 ? data_u32 + kRopeOff : set_u32 + s * kSetBytes + kc * kChunk;
+#pragma unroll
+              for (int ks = 0; ks < 4; ++ks)
+                mma2_ss(tmem + kSCol + 64 * sb, desc_sw128(data_u32 + kQOff + kc * kChunk + ks * 32, 16, 1024),
+                        desc_sw128(bsl + ks * 32, 16, 1024), idesc_qk, (cq | ks) != 0);
+              if (cq == 0) mma_commit2(bar(ctl->rope_done), 3);
+              else if ((kc & 1) == 1) mma_commit2(bar(ctl->qk_done[s][kc >> 1]), 3);
+              if (++cq == 9) {
+                cq = 0;
+                mma_commit2(bar(ctl->s_full[sb]), 3);
+                if (qc.last()) mma_commit2(bar(ctl->q_free), 3);
+                qc.advance(prefix);
+              }
+              did = true;
+            }
+          }
+          if (did) {
+            t_idle = globaltimer();
+          } else if (*abort_flag) {
+            break;
+          } else if (globaltimer() - t_idle > kWaitLimitNs) {
+            record_error(MLA_ERR_TIMEOUT);
+            *abort_flag = 1;
+            st_cluster_u32(peer_abort, 1u);
+            break;
+          }
         }
+      }
+      __syncwarp();
+    } else if (warp < kSoftWarps) {
+      // ---------------------------------------------------------------- softmax, rescale, epilogue
+      // Thread: TMEM lane lt = 32 (warp % 4) + lane, head h = lt % 64 of this CTA, page g = lt / 64,
+      // column half ch = warp / 4: tokens [64g + 32ch, 64g + 32ch + 32) of the tile, and O
+      // columns [128ch, 128ch + 128) (latent columns 256ch + 128g + [0, 128)).
+      const int qd = warp & 3, ch = warp >> 2;
+      const int lt = 32 * qd + lane, h = lt & 63, g = lt >> 6;
+      const int head = 64 * (int)rank + h;
+      const uint32_t lane_base = (uint32_t)(qd * 32) << 16;
+      const uint32_t p_row = data_u32 + kPOff + g * kChunk + (h >> 3) * 1024 + (h & 7) * 128;
+      uint8_t* const p_row_ptr = data + (p_row - data_u32);
+      uint32_t xc = 0;  // exchanges so far (phase of xm_full / xm_free)
+      // Exchange one value among the four threads of a head; returns the four in a fixed order
+      // (page 0 half 0, page 0 half 1, page 1 half 0, page 1 half 1).
+      auto exchange = [&](float v, float (&out)[4]) {
+        if (xc > 0 && !wwait(ctl->xm_free, (xc - 1) & 1)) return false;
+        ctl->xm[ch][lt] = v;
         __syncwarp();
-      } else {  // ---------------- softmax warps 0-3: thread = head row = TMEM lane
-        const int h = warp * 32 + lane;
-        const uint32_t lane_base = (uint32_t)(warp * 32) << 16;
-        const uint32_t row_off = (uint32_t)((h >> 3) * 1024 + (h & 7) * 128);
-        int tile = 0, item_i = 0;
-        bool ok = true;
-        ItemIter it = item_iter(p.tile_prefix, p.B, cluster, nclusters);
-        Item item;
-        while (ok && next_item(it, p.tile_prefix, item)) {
-          // Q row h of sequence b into TMEM columns [kQCol, kQCol + 288): two elements per column,
-          // loaded in three batches of 24 x 16 bytes so that the loads overlap
-          const uint4* qrow = reinterpret_cast<const uint4*>(static_cast<const T*>(p.q) +
-                                                             ((long)item.b * p.n_h + (h < p.n_h ? h : 0)) * kD);
+        if (lane == 0) mbar_arrive(bar(ctl->xm_full));
+        if (!wwait(ctl->xm_full, xc & 1)) return false;
+        const int l0 = lt & 63;
+        out[0] = ctl->xm[0][l0];
+        out[1] = ctl->xm[1][l0];
+        out[2] = ctl->xm[0][l0 + 64];
+        out[3] = ctl->xm[1][l0 + 64];
+        __syncwarp();
+        if (lane == 0) mbar_arrive(bar(ctl->xm_free));
+        ++xc;
+        return true;
+      };
+      Cursor c;
+      c.start(prefix, p.B, cluster, nclusters);
+      float m_ref = -INFINITY, lsum = 0.f;
+      int L = 0;
+      bool ok = true;
+      while (ok && c.valid) {
+        const int ti = c.ti, sb = ti & 1, t = c.t;
+        if (c.first()) {
+          m_ref = -INFINITY;
+          lsum = 0.f;
+          L = p.seq_lens[c.item.b];
+        }
+        if (!wwait(ctl->s_full[sb], (ti >> 1) & 1)) break;
+        tc_fence_after();
+        uint32_t sr[32];
+        tmem_ld32(tmem + lane_base + kSCol + 64 * sb + 32 * ch, sr);
+        tmem_wait_ld();
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive_remote(lead(ctl->s_free[sb]));
+        // tokens past the sequence end become -inf (weight exactly 0), whatever the slot held
+        const int nv = max(0, min(32, L - (kTile * t + kPage * g + 32 * ch)));
+        if (nv < 32) {
+#pragma unroll
+          for (int k = 0; k < 32; ++k)
+            if (k >= nv) sr[k] = __float_as_uint(-INFINITY);
+        }
+        float mxs[8];
+#pragma unroll
+        for (int k = 0; k < 8; ++k) mxs[k] = u2f(sr[k]);
+#pragma unroll
+        for (int k = 8; k < 32; ++k) mxs[k & 7] = fmaxf(mxs[k & 7], u2f(sr[k]));
+        float four[4];
+        if (!exchange(fmaxf(fmaxf(fmaxf(mxs[0], mxs[1]), fmaxf(mxs[2], mxs[3])),
+                            fmaxf(fmaxf(mxs[4], mxs[5]), fmaxf(mxs[6], mxs[7]))),
+                      four))
+          break;
+        const float mx = fmaxf(fmaxf(four[0], four[1]), fmaxf(four[2], four[3])) * p.scale_log2;
+        float alpha = 1.f;
+        if (mx > m_ref + kLazy) {
+          alpha = ex2_approx(m_ref - mx);
+          lsum *= alpha;
+          m_ref = mx;
+        }
+        // the O MMAs of the previous tile are done: P may be overwritten and O rescaled
+        if (!wwait(ctl->p_free, (ti & 1) ^ 1)) break;
+        if (!c.first() && __any_sync(0xffffffffu, alpha != 1.f)) {
+          tc_fence_after();
 #pragma unroll 1
-          for (int c0 = 0; c0 < kD / 2; c0 += 96) {
-            uint4 x[24];
+          for (int c0 = 0; c0 < 128; c0 += 64) {  // two TMEM loads in flight per wait
+            uint32_t r[2][32];
 #pragma unroll
-            for (int v = 0; v < 24; ++v) x[v] = h < p.n_h ? __ldg(qrow + c0 / 4 + v) : make_uint4(0, 0, 0, 0);
+            for (int q2 = 0; q2 < 2; ++q2) tmem_ld32(tmem + lane_base + kOCol + 128 * ch + c0 + 32 * q2, r[q2]);
+            tmem_wait_ld();
 #pragma unroll
-            for (int part = 0; part < 3; ++part) {
-              uint32_t r[32];
+            for (int q2 = 0; q2 < 2; ++q2) {
 #pragma unroll
-              for (int v = 0; v < 8; ++v) {
-                r[4 * v] = x[part * 8 + v].x;
-                r[4 * v + 1] = x[part * 8 + v].y;
-                r[4 * v + 2] = x[part * 8 + v].z;
-                r[4 * v + 3] = x[part * 8 + v].w;
-              }
-              tmem_st32(tmem + lane_base + kQCol + c0 + part * 32, r);
+              for (int k = 0; k < 32; ++k) r[q2][k] = __float_as_uint(u2f(r[q2][k]) * alpha);
+              tmem_st32(tmem + lane_base + kOCol + 128 * ch + c0 + 32 * q2, r[q2]);
             }
           }
           tmem_wait_st();
-          tc_fence_before();
-          mbar_arrive(bar(ctl->q_ready));
-
-          const int L = p.seq_lens[item.b];
-          float m_ref = -INFINITY, l = 0.f;
-          for (int t = item.t0; t < item.t1; t += 2, ++tile) {
-            if (!wwait(ctl->s_full, tile & 1)) {
-              ok = false;
-              break;
-            }
-            tc_fence_after();
-            // S row h: four TMEM loads in flight, one wait
-            uint32_t sr[4][32];
-#pragma unroll
-            for (int c4 = 0; c4 < 4; ++c4) tmem_ld32(tmem + lane_base + kSCol + c4 * 32, sr[c4]);
-            tmem_wait_ld();
-            tc_fence_before();
-            mbar_arrive(bar(ctl->s_empty));
-
-            // tokens of this tile: page t (0..63) and, if it belongs to this item, page t+1 (64..127);
-            // masked tokens become -inf and get weight exactly 0
-            const int nv = min(t + 1 < item.t1 ? kTile : kPage, L - t * kPage);
-            if (nv < kTile) {
-#pragma unroll
-              for (int k = 0; k < kTile; ++k)
-                if (k >= nv) sr[k >> 5][k & 31] = __float_as_uint(-INFINITY);
-            }
-            // running maximum on the raw scores (the scale is positive, so the order is the same),
-            // eight independent chains
-            float mxs[8];
-#pragma unroll
-            for (int j = 0; j < 8; ++j) mxs[j] = u2f(sr[0][j]);
-#pragma unroll
-            for (int k = 8; k < kTile; ++k) mxs[k & 7] = fmaxf(mxs[k & 7], u2f(sr[k >> 5][k & 31]));
-            const float mx = fmaxf(fmaxf(fmaxf(mxs[0], mxs[1]), fmaxf(mxs[2], mxs[3])),
-                                   fmaxf(fmaxf(mxs[4], mxs[5]), fmaxf(mxs[6], mxs[7]))) * p.scale_log2;
-            float alpha = 1.f;
-            if (mx > m_ref + kLazy) {
-              alpha = ex2_approx(m_ref - mx);
-              l *= alpha;
-              m_ref = mx;
-            }
-            const int sb = tile % kStg;
-            if (!wwait(ctl->stg_free[sb], ((tile / kStg) & 1) ^ 1)) {
-              ok = false;
-              break;
-            }
-            // P row h in the 128-byte-swizzled K-major layout (two 64-token halves):
-            // p = 2^(s * scale - m_ref), one FFMA and one ex2 per token. The sum of the rounded
-            // weights is the denominator (it matches what the MMA accumulates); four chains.
-            uint8_t* stage = data + kStageOff + sb * kPStride;
-            float sums[4] = {0.f, 0.f, 0.f, 0.f};
-#pragma unroll
-            for (int c = 0; c < 16; ++c) {
-              uint32_t w[4];
-#pragma unroll
-              for (int j = 0; j < 4; ++j) {
-                const int k = 8 * c + 2 * j;
-                const typename Pack<T>::T2 pr =
-                    Pack<T>::make(ex2_approx(fmaf(u2f(sr[k >> 5][k & 31]), p.scale_log2, -m_ref)),
-                                  ex2_approx(fmaf(u2f(sr[(k + 1) >> 5][(k + 1) & 31]), p.scale_log2, -m_ref)));
-                const float2 back = Pack<T>::f2(pr);
-                sums[j] += back.x + back.y;
-                w[j] = *reinterpret_cast<const uint32_t*>(&pr);
-              }
-              *reinterpret_cast<uint4*>(stage + (c >> 3) * 16384 + row_off + (((c & 7) ^ (h & 7)) << 4)) =
-                  make_uint4(w[0], w[1], w[2], w[3]);
-            }
-            const float sum = (sums[0] + sums[1]) + (sums[2] + sums[3]);
-            l += sum;
-            reinterpret_cast<float*>(stage + kPTile)[h] = alpha;
-            fence_proxy_async_cta();
-            mbar_arrive(bar(ctl->stg_ready[sb]));
-          }
-          if (!ok) break;
-          if (!wwait_cl(ctl->stats_empty, (item_i & 1) ^ 1)) break;
-          st_cluster_f32(mapa(smem_u32(&ctl->stats[h][0]), 1u), m_ref);
-          st_cluster_f32(mapa(smem_u32(&ctl->stats[h][1]), 1u), l);
-          mbar_arrive_remote(mapa(bar(ctl->stats_full), 1u));
-          ++item_i;
         }
-      }
-    } else {
-      // =========================================================== value CTA
-      if (warp == 4) {  // ---------------- TMA producer: half the latent of one page per slot
-        if (lane == 0) {
-          tma_prefetch_map(&pool_map);
-          int vslot = 0;
-          bool ok = true;
-          ItemIter it = item_iter(p.tile_prefix, p.B, cluster, nclusters);
-          Item item;
-          while (ok && next_item(it, p.tile_prefix, item)) {
-            const int* btb = p.bt + (long)item.b * p.max_pages;
-            for (int t = item.t0; ok && t < item.t1; t += 2) {
-              const int np = t + 1 < item.t1 ? 2 : 1;
-              const int pages[2] = {btb[t], np == 2 ? btb[t + 1] : 0};
-              for (int hf = 0; ok && hf < 2; ++hf)
-                for (int g = 0; g < np; ++g, ++vslot) {
-                  const int s = vslot % kValSlots;
-                  if (!wait(ctl->empty[s], ((vslot / kValSlots) & 1) ^ 1)) {
-                    ok = false;
-                    break;
-                  }
-                  mbar_arrive_expect_tx(bar(ctl->full[s]), 4 * kChunk);
+        // P row h, tokens [32ch, 32ch + 32) of page g: p = 2^(s * scale - m_ref), one FFMA and one
+        // ex2 per token. The sum of the rounded weights is the denominator (it matches what the
+        // MMA accumulates).
+        float sums[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
-                  for (int q4 = 0; q4 < 4; ++q4)
-                    tma_load_2d(data_u32 + (s * 4 + q4) * kChunk, &pool_map, bar(ctl->full[s]), (hf * 4 + q4) * 64,
-                                pages[g] * kPage);
-                }
-            }
+        for (int u4 = 0; u4 < 4; ++u4) {
+          uint32_t w[4];
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            const int k = 8 * u4 + 2 * e;
+            const typename Pack<T>::T2 pr2 = Pack<T>::make(ex2_approx(fmaf(u2f(sr[k]), p.scale_log2, -m_ref)),
+                                                           ex2_approx(fmaf(u2f(sr[k + 1]), p.scale_log2, -m_ref)));
+            const float2 back = Pack<T>::f2(pr2);
+            sums[e] += back.x + back.y;
+            w[e] = *reinterpret_cast<const uint32_t*>(&pr2);
           }
-          if (!ok)
-            for (int i = max(0, vslot - kValSlots); i < vslot; ++i)
-              mbar_wait_slow<false>(bar(ctl->full[i % kValSlots]), (i / kValSlots) & 1, nullptr);
+          *reinterpret_cast<uint4*>(p_row_ptr + ((((4 * ch + u4) ^ (h & 7))) << 4)) = make_uint4(w[0], w[1], w[2], w[3]);
         }
+        lsum += (sums[0] + sums[1]) + (sums[2] + sums[3]);
+        fence_proxy_async_cta();
+        tc_fence_before();
         __syncwarp();
-      } else if (warp == 5) {  // ---------------- MMA issue: O += P C_lat (whole warp waits; lane 0 issues)
-        const uint32_t idesc = idesc_f16(128, 256, kBf16, false, true);
-        int vslot = 0, tile = 0, item_i = 0;
-        bool ok = true;
-        ItemIter it = item_iter(p.tile_prefix, p.B, cluster, nclusters);
-        Item item;
-        while (ok && next_item(it, p.tile_prefix, item)) {
-          if (!wwait(ctl->o_free, (item_i & 1) ^ 1)) break;
+        if (lane == 0) mbar_arrive_remote(lead(ctl->p_full));
+
+        if (c.last()) {  // ---- epilogue of the item: O / l for this thread's head and columns
+          if (!wwait(ctl->p_free, ti & 1)) break;  // the last O MMAs are done
           tc_fence_after();
-          const int L = p.seq_lens[item.b];
-          for (int t = item.t0; ok && t < item.t1; t += 2, ++tile) {
-            const int pb = tile % kPBufs;
-            if (!wwait(ctl->p_ready[pb], (tile / kPBufs) & 1)) {
-              ok = false;
-              break;
-            }
-            tc_fence_after();
-            const uint32_t pa = data_u32 + kPOff + pb * kPStride;
-            const int np = t + 1 < item.t1 ? 2 : 1;
-            for (int hf = 0; ok && hf < 2; ++hf)
-              for (int g = 0; g < np; ++g, ++vslot) {
-                const int s = vslot % kValSlots;
-                if (!wwait(ctl->full[s], (vslot / kValSlots) & 1)) {
-                  ok = false;
-                  break;
-                }
-                const int nv = min(kPage, L - (t + g) * kPage);
-                if (nv < kPage) {  // rows past the sequence end may hold anything (even NaN): zero them
-                  uint8_t* slot = data + s * 4 * kChunk;
-                  const int per_chunk = (kPage - nv) * 8;
-                  for (int e = lane; e < 4 * per_chunk; e += 32) {
-                    const int q4 = e / per_chunk, rem = e % per_chunk;
-                    *reinterpret_cast<uint4*>(slot + q4 * kChunk + (nv + rem / 8) * 128 + (rem % 8) * 16) =
-                        make_uint4(0, 0, 0, 0);
-                  }
-                  fence_proxy_async_cta();
-                  __syncwarp();
-                }
-                tc_fence_after();
-                if (lane == 0) {
-                  const uint32_t sb = data_u32 + s * 4 * kChunk;
-#pragma unroll
-                  for (int ks = 0; ks < 4; ++ks)
-                    mma_ss(tmem + kOCol + hf * 256, desc_sw128(pa + g * 16384 + ks * 32, 16, 1024),
-                           desc_sw128(sb + ks * 2048, 4 * 2048, 1024), idesc, !(t == item.t0 && g == 0 && ks == 0));
-                  mma_commit(bar(ctl->empty[s]));
-                }
-                __syncwarp();
-              }
-            if (ok && lane == 0) {
-              mma_commit_mc(bar(ctl->p_empty[pb]), (uint16_t)1u);  // P buffer free: tell the score CTA
-              mma_commit(bar(ctl->o_done[pb]));
-            }
-            __syncwarp();
-          }
-          ++item_i;
-        }
-      } else if (warp < 4) {  // ---------------- correction + epilogue warps 0-3: thread = head row
-        const int h = warp * 32 + lane;
-        const uint32_t lane_base = (uint32_t)(warp * 32) << 16;
-        const uint32_t stats_empty_remote = mapa(bar(ctl->stats_empty), 0u);
-        int tile = 0, item_i = 0;
-        bool ok = true;
-        ItemIter it = item_iter(p.tile_prefix, p.B, cluster, nclusters);
-        Item item;
-        while (ok && next_item(it, p.tile_prefix, item)) {
-          for (int t = item.t0; t < item.t1; t += 2, ++tile) {
-            const int pb = tile % kPBufs;
-            if (!wwait_cl(ctl->p_full[pb], (tile / kPBufs) & 1)) {
-              ok = false;
-              break;
-            }
-            const float alpha = reinterpret_cast<const float*>(data + kPOff + pb * kPStride + kPTile)[h];
-            if (t != item.t0 && __any_sync(0xffffffffu, alpha != 1.f)) {
-              if (!wwait(ctl->o_done[(tile - 1) % kPBufs], ((tile - 1) / kPBufs) & 1)) {
-                ok = false;
-                break;
-              }
-              tc_fence_after();
-#pragma unroll 1
-              for (int c0 = 0; c0 < kDc; c0 += 128) {  // four TMEM loads in flight per wait
-                uint32_t r[4][32];
-#pragma unroll
-                for (int q4 = 0; q4 < 4; ++q4) tmem_ld32(tmem + lane_base + kOCol + c0 + 32 * q4, r[q4]);
-                tmem_wait_ld();
-#pragma unroll
-                for (int q4 = 0; q4 < 4; ++q4) {
-#pragma unroll
-                  for (int j = 0; j < 32; ++j) r[q4][j] = __float_as_uint(u2f(r[q4][j]) * alpha);
-                  tmem_st32(tmem + lane_base + kOCol + c0 + 32 * q4, r[q4]);
-                }
-              }
-              tmem_wait_st();
-            }
-            tc_fence_before();
-            mbar_arrive(bar(ctl->p_ready[pb]));
-          }
-          if (!ok) break;
-          if (!wwait_cl(ctl->stats_full, item_i & 1)) break;
-          const float m_ref = ctl->stats[h][0], l = ctl->stats[h][1];
-          mbar_arrive_remote(stats_empty_remote);
-          // O holds every tile of the item once the last one is done; the other buffer's last
-          // arrival is waited for as well so that none is still in flight when the CTA exits
-          if (!wwait(ctl->o_done[(tile - 1) % kPBufs], ((tile - 1) / kPBufs) & 1)) break;
-          if (tile >= 2 && !wwait(ctl->o_done[(tile - 2) % kPBufs], ((tile - 2) / kPBufs) & 1)) break;
-          tc_fence_after();
+          if (!exchange(lsum, four)) break;
+          const float l = (four[0] + four[1]) + (four[2] + four[3]);
           const float inv = l > 0.f ? 1.f / l : 0.f;
           const float lse = l > 0.f ? (m_ref + log2f(l)) * 0.6931471805599453f : -INFINITY;
-          const bool whole = item.t0 == 0 && item.t1 == item.n_b;
-          const long slot = (long)item.b + cluster;
+          const Item& it = c.item;
+          const bool whole = it.t0 == 0 && it.t1 == it.n_b;
+          const long slot = (long)it.b + cluster;
+          const int col0 = 256 * ch + 128 * g;  // latent columns [col0, col0 + 128)
 #pragma unroll 1
-          for (int c0 = 0; c0 < kDc; c0 += 128) {  // four TMEM loads in flight per wait
-            uint32_t r[4][32];
+          for (int c0 = 0; c0 < 128; c0 += 64) {  // two TMEM loads in flight per wait
+            uint32_t r[2][32];
 #pragma unroll
-            for (int q4 = 0; q4 < 4; ++q4) tmem_ld32(tmem + lane_base + kOCol + c0 + 32 * q4, r[q4]);
+            for (int q2 = 0; q2 < 2; ++q2) tmem_ld32(tmem + lane_base + kOCol + 128 * ch + c0 + 32 * q2, r[q2]);
             tmem_wait_ld();
-            if (h < p.n_h) {
+            if (head < p.n_h) {
               if (whole) {
-                uint4* dst = reinterpret_cast<uint4*>(static_cast<T*>(p.o_lat) + ((long)item.b * p.n_h + h) * kDc + c0);
+                uint4* dst = reinterpret_cast<uint4*>(static_cast<T*>(p.o_lat) + ((long)it.b * p.n_h + head) * kDc +
+                                                      col0 + c0);
 #pragma unroll
-                for (int j = 0; j < 16; ++j) {
+                for (int q = 0; q < 8; ++q) {
                   uint32_t w[4];
 #pragma unroll
                   for (int e = 0; e < 4; ++e) {
-                    const int k = 8 * j + 2 * e;
+                    const int k = 8 * q + 2 * e;
                     const typename Pack<T>::T2 v =
                         Pack<T>::make(u2f(r[k >> 5][k & 31]) * inv, u2f(r[(k + 1) >> 5][(k + 1) & 31]) * inv);
                     w[e] = *reinterpret_cast<const uint32_t*>(&v);
                   }
-                  dst[j] = make_uint4(w[0], w[1], w[2], w[3]);
+                  dst[q] = make_uint4(w[0], w[1], w[2], w[3]);
                 }
               } else {
-                float4* dst = reinterpret_cast<float4*>(p.o_part + (slot * p.n_h + h) * kDc + c0);
+                float4* dst = reinterpret_cast<float4*>(p.o_part + (slot * p.n_h + head) * kDc + col0 + c0);
 #pragma unroll
-                for (int j = 0; j < 32; ++j) {
-                  const int k = 4 * j;
-                  dst[j] = make_float4(u2f(r[k >> 5][k & 31]) * inv, u2f(r[k >> 5][(k & 31) + 1]) * inv,
+                for (int q = 0; q < 16; ++q) {
+                  const int k = 4 * q;
+                  dst[q] = make_float4(u2f(r[k >> 5][k & 31]) * inv, u2f(r[k >> 5][(k & 31) + 1]) * inv,
                                        u2f(r[k >> 5][(k & 31) + 2]) * inv, u2f(r[k >> 5][(k & 31) + 3]) * inv);
                 }
               }
             }
           }
-          if (h < p.n_h) {
+          if (head < p.n_h && g == 0 && ch == 0) {
             if (whole) {
-              if (p.lse_out != nullptr) p.lse_out[(long)item.b * p.n_h + h] = lse;
+              if (p.lse_out != nullptr) p.lse_out[(long)it.b * p.n_h + head] = lse;
             } else {
-              p.lse_part[slot * p.n_h + h] = lse;
+              p.lse_part[slot * p.n_h + head] = lse;
             }
           }
           tc_fence_before();
-          mbar_arrive(bar(ctl->o_free));
-          ++item_i;
+          __syncwarp();
+          if (lane == 0) mbar_arrive_remote(lead(ctl->o_free));
         }
+        c.advance(prefix);
       }
     }
   }
 
   // ---------------------------------------------------------------- teardown
-  if (has_work && warp == 5) {
-    if (lane == 0) {  // every MMA this thread issued has completed before TMEM is released
-      mma_commit(bar(ctl->drain));
+  if (has_work && warp == kMmaWarp && rank == 0) {
+    if (lane == 0) {  // every pair MMA has completed before either CTA releases its tensor memory
+      mma_commit2(bar(ctl->drain), 1);
       mbar_wait_slow<false>(bar(ctl->drain), 0, nullptr);
     }
     __syncwarp();
   }
+  if (*abort_flag && threadIdx.x == 0) {
+    // A wait gave up: loads already issued (to this CTA's slots, signalling rank 0's barriers)
+    // land within microseconds; give them 200 us before either CTA of the pair exits.
+    const uint64_t t0 = globaltimer();
+    while (globaltimer() - t0 < 200000ull) {
+    }
+  }
   tc_fence_before();
   __syncthreads();
-  if (warp == 5) {
-    tc_fence_after();
-    tmem_dealloc(tmem, kTmemCols);
-  }
   cluster_arrive();  // neither CTA leaves while its peer may still touch its shared memory
   cluster_wait();
+  if (warp == kMmaWarp) {
+    tc_fence_after();
+    tmem_dealloc2(tmem, kTmemCols);
+  }
 }
 
-// Pages per sequence (0 for a sequence whose length or pages are invalid) and their exclusive
+// Tiles per sequence (0 for a sequence whose length or pages are invalid) and their exclusive
 // prefix sum, in one block of 1024 threads: a warp checks a sequence's pages (lanes stride over
-// its block-table row), then a block-wide scan turns the counts into offsets in place.
+// its block-table row), then a block-wide scan turns the counts into offsets in place. The host
+// keeps the total (B x tiles of max_seq_len) within int32.
 __global__ void __launch_bounds__(1024) k_decode_plan(const int* __restrict__ seq_lens, const int* __restrict__ bt,
                                                       int B, int max_pages, int num_pages, int max_seq_len,
                                                       int* __restrict__ tile_prefix) {
@@ -639,7 +677,7 @@ __global__ void __launch_bounds__(1024) k_decode_plan(const int* __restrict__ se
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   for (int b = warp; b < B; b += 32) {
     const int L = seq_lens[b];
-    const int n = (L + dec::kPage - 1) / dec::kPage;
+    const int n = (int)(((long)L + dec::kPage - 1) / dec::kPage);
     bool ok = L >= 1 && L <= max_seq_len && n <= max_pages;
     if (!ok && lane == 0) record_error(MLA_ERR_BAD_SEQ_LEN);
     if (ok) {
@@ -653,7 +691,7 @@ __global__ void __launch_bounds__(1024) k_decode_plan(const int* __restrict__ se
         if (lane == 0) record_error(MLA_ERR_BAD_PAGE);
       }
     }
-    if (lane == 0) tile_prefix[b] = ok ? n : 0;
+    if (lane == 0) tile_prefix[b] = ok ? (int)(((long)L + dec::kTile - 1) / dec::kTile) : 0;
   }
   __syncthreads();
   const int per = (B + 1023) / 1024;
@@ -677,9 +715,9 @@ __global__ void __launch_bounds__(1024) k_decode_plan(const int* __restrict__ se
   if (tid == 1023) tile_prefix[B] = part[1023];
 }
 
-// Merge of the partials of sequences that span clusters, in cluster order; zero output for
-// rejected sequences. grid (B, ceil(n_h / 8)), 256 threads: one warp per head, each lane 16 of
-// the 512 latent values (four 16-byte loads per contributing cluster, all in flight together).
+// Merge of the partials of sequences that span pairs, in pair order; zero output for rejected
+// sequences. grid (B, ceil(n_h / 8)), 256 threads: one warp per head, each lane 16 of the 512
+// latent values (four 16-byte loads per contributing pair, all in flight together).
 template <typename T>
 __global__ void __launch_bounds__(256) k_decode_tc_merge(const float* __restrict__ o_part,
                                                           const float* __restrict__ lse_part,
@@ -699,9 +737,9 @@ __global__ void __launch_bounds__(256) k_decode_tc_merge(const float* __restrict
     return;
   }
   const int c0 = cluster_of(g0, T_, C), c1 = cluster_of(g1 - 1, T_, C);
-  if (c0 == c1) return;  // written whole by its cluster
-  // clusters between c0 and c1 own consecutive pages of this sequence, except those whose range
-  // is empty (fewer pages than clusters): they wrote nothing and are skipped
+  if (c0 == c1) return;  // written whole by its pair
+  // pairs between c0 and c1 own consecutive tiles of this sequence, except those whose range is
+  // empty (fewer tiles than pairs): they wrote nothing and are skipped
   auto owns = [&](int c) { return T_ * (c + 1) / C > T_ * c / C; };
   const float* lp = lse_part + (long)b * n_h + h;  // slot b + c is at lp[c * n_h]
   float mx = -INFINITY;

@@ -43,6 +43,7 @@ struct EpiParams {
   // RoPE (append, query): rows m >= rope_lo rotate in pairs (m, m ^ 1)
   int rope_lo, d_rope;
   double rope_base;
+  const double* rope_table;  // [d_rope/2] theta_k supplied by the caller, or null (base^(-2k/d_rope))
   const int* pos;       // [N]
   float2* cs_glob;      // [N][d_rope/2] cos/sin for split tiles' reduction (or null)
   int cs_ready;         // 1: cs_glob was filled by an earlier kernel (read it, do not compute it)
@@ -139,10 +140,10 @@ struct RowDest {
 // loop that may call it is unrolled and runs with cold instruction fetch, so an inlined
 // double-precision pow and sincos in its branch would slow every pass through it.
 __device__ __noinline__ float2 rope_cs_out_of_line(const float2* tab, const int* pos, int n, int k, int d_rope,
-                                                   double base) {
+                                                   double base, const double* table) {
   if (tab != nullptr) return tab[(long)n * (d_rope / 2) + k];
   float2 q;
-  rope_cos_sin(pos[n], k, d_rope, base, q.x, q.y);
+  rope_cos_sin(pos[n], k, d_rope, base, table, q.x, q.y);
   return q;
 }
 
@@ -340,7 +341,8 @@ __global__ void __launch_bounds__(192, 2)
     if (fill != nullptr)
       for (int e = cta * 128 + ml; e < p.N * half_rope; e += G * 128) {
         float c, sn;
-        rope_cos_sin(p.epi.pos[e / half_rope], e % half_rope, p.epi.d_rope, p.epi.rope_base, c, sn);
+        rope_cos_sin(p.epi.pos[e / half_rope], e % half_rope, p.epi.d_rope, p.epi.rope_base, p.epi.rope_table, c,
+                     sn);
         fill[e] = make_float2(c, sn);
       }
     if (tab_cs && p.epi.cs_ready) {
@@ -352,7 +354,7 @@ __global__ void __launch_bounds__(192, 2)
       for (int e = ml; e < BN * half_rope; e += 128) {
         const int n = e / half_rope, k = e % half_rope;
         if (k != theta_k) {  // with half_rope dividing 128 this runs once per thread
-          theta = rope_inv_freq(k, p.epi.d_rope, p.epi.rope_base);
+          theta = rope_inv_freq(k, p.epi.d_rope, p.epi.rope_base, p.epi.rope_table);
           theta_k = k;
         }
         float c = 1.f, sn = 0.f;
@@ -418,7 +420,7 @@ __global__ void __launch_bounds__(192, 2)
                 float2 q;
                 if (tab_cs) q = cs_tab[nl * half_rope + k];
                 else q = rope_cs_out_of_line(p.epi.cs_ready ? p.epi.cs_glob : nullptr, p.epi.pos, n0 + nl, k,
-                                             p.epi.d_rope, p.epi.rope_base);
+                                             p.epi.d_rope, p.epi.rope_base, p.epi.rope_table);
                 v = (m & 1) ? fmaf(w, q.y, v * q.x) : fmaf(v, q.x, -w * q.y);
               }
             }
@@ -497,7 +499,7 @@ __global__ void __launch_bounds__(256) k_sk_reduce(const SkParams p, int G) {
       cs = t.x;
       sn = t.y;
     } else {
-      rope_cos_sin(p.epi.pos[n], k, p.epi.d_rope, p.epi.rope_base, cs, sn);
+      rope_cos_sin(p.epi.pos[n], k, p.epi.d_rope, p.epi.rope_base, p.epi.rope_table, cs, sn);
     }
     const float ra = fmaf(a, cs, -b * sn), rb2 = fmaf(b, cs, a * sn);
     a = ra;

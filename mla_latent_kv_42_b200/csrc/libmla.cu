@@ -3,6 +3,8 @@
 // Host code here validates arguments (before anything is queued), carves the caller's
 // workspace, picks kernels and launches them on the caller's stream. It allocates nothing.
 #include "mla_debug.h"
+#include <nvtx3/nvToolsExt.h>
+
 #include <atomic>
 #include <cmath>
 #include <cstring>
@@ -17,6 +19,15 @@
 using namespace mla;
 
 namespace {
+
+// NVTX range around each entry point (host side: the argument checks and the launches), named
+// after the call, for timelines taken with a profiler; without one attached it costs a few ns.
+struct NvtxRange {
+  explicit NvtxRange(const char* name) { nvtxRangePushA(name); }
+  ~NvtxRange() { nvtxRangePop(); }
+  NvtxRange(const NvtxRange&) = delete;
+  NvtxRange& operator=(const NvtxRange&) = delete;
+};
 
 thread_local int32_t t_launches[5] = {0, 0, 0, 0, 0};
 // Profiling hook: events recorded around the attention kernel of this thread's decode calls.
@@ -71,6 +82,7 @@ int check_dims_impl(const mla_dims* d) {
     if (v <= 0) return MLA_ERR_INVALID_ARG;
   if (d->d_model % 8 || d->d_head % 8 || d->d_c % 8 || d->d_cq % 8 || d->d_rope % 8) return MLA_ERR_UNSUPPORTED_DIMS;
   if (d->n_heads > 128 || d->d_c > 512 || d->d_c + d->d_rope > 576) return MLA_ERR_UNSUPPORTED_DIMS;
+  if ((reinterpret_cast<uintptr_t>(d->rope_inv_freq) & 7u) != 0) return MLA_ERR_ALIGNMENT;
   return MLA_OK;
 }
 
@@ -127,13 +139,10 @@ int absorb_impl(const mla_dims* d, const void* h, const void* w_dq, const void* 
 
 // ---------------------------------------------------------------- tensor-core decode
 // The tcgen05 path serves DeepSeek-V2-shaped caches (d_c = 512, d_h^R = 64, 64-token pages,
-// 65..128 heads); MLA_DECODE_IMPL=simt selects the CUDA-core kernel instead.
+// 65..128 heads: one pair of SMs holds the heads' 512-column accumulators); other shapes, the
+// running model's eight heads among them, take the CUDA-core kernel.
 bool decode_tc_eligible(const mla_dims* d) {
-  static const bool forced_simt = [] {
-    const char* e = std::getenv("MLA_DECODE_IMPL");
-    return e != nullptr && std::strcmp(e, "simt") == 0;
-  }();
-  return !forced_simt && d->n_heads > 64 && d->n_heads <= 128 && d->d_c == tc::dec::kDc &&
+  return d->n_heads > 64 && d->n_heads <= 128 && d->d_c == tc::dec::kDc &&
          d->d_c + d->d_rope == tc::dec::kD && d->page_size == tc::dec::kPage;
 }
 
@@ -207,15 +216,18 @@ int decode_tc_impl(const mla_dims* d, const void* q, const void* pool, int32_t n
   int* prefix = c.take<int>((size_t)B + 1);
   float* o_part = c.take<float>(((size_t)B + C) * d->n_heads * tc::dec::kDc);
   float* lse_part = c.take<float>(((size_t)B + C) * d->n_heads);
-  CUtensorMap map;
-  if (!host::encode_2d(&map, pool, tc::IsBf16<T>::value, tc::dec::kD, (uint64_t)num_pages * tc::dec::kPage,
-                       tc::dec::kD * 2, 64, 64))
+  constexpr bool bf16 = tc::IsBf16<T>::value;
+  const uint64_t pool_rows = (uint64_t)num_pages * tc::dec::kPage;
+  tc::DecodeTcMaps maps;
+  if (!host::encode_2d(&maps.pool1, pool, bf16, tc::dec::kD, pool_rows, tc::dec::kD * 2, 64, 64) ||
+      !host::encode_chunks(&maps.pool2, pool, bf16, pool_rows, tc::dec::kD * 2, 2) ||
+      !host::encode_chunks(&maps.pool4, pool, bf16, pool_rows, tc::dec::kD * 2, 4) ||
+      !host::encode_chunks(&maps.q9, q, bf16, (uint64_t)B * d->n_heads, tc::dec::kD * 2, 9))
     return MLA_ERR_CUDA;
   if (launch_pdl(tc::k_decode_plan, dim3(1), dim3(1024), 0, st, seq_lens, bt, (int)B, (int)max_pages, (int)num_pages,
                  (int)max_seq_len, prefix) != cudaSuccess)
     return MLA_ERR_CUDA;
   tc::DecodeTcParams p;
-  p.q = q;
   p.bt = bt;
   p.max_pages = max_pages;
   p.seq_lens = seq_lens;
@@ -228,7 +240,7 @@ int decode_tc_impl(const mla_dims* d, const void* q, const void* pool, int32_t n
   p.o_part = o_part;
   p.lse_part = lse_part;
   mark_before(st);
-  if (launch_pdl(tc::k_decode_tc<T>, dim3(2 * C), dim3(tc::dec::kThreads), tc::dec::kSmem, st, map, p) != cudaSuccess)
+  if (launch_pdl(tc::k_decode_tc<T>, dim3(2 * C), dim3(tc::dec::kThreads), tc::dec::kSmem, st, maps, p) != cudaSuccess)
     return MLA_ERR_CUDA;
   mark_after(st);
   if (launch_pdl(tc::k_decode_tc_merge<T>, dim3(B, (d->n_heads + 7) / 8), dim3(256), 0, st,
@@ -382,6 +394,7 @@ size_t mla_workspace_size(const mla_dims* dims, int32_t call, int32_t B, int32_t
 int mla_append_kv(const mla_dims* dims, const void* h, const void* w_dkv_kr, const int32_t* seq_idx,
                   const int32_t* pos, const int32_t* block_table, int32_t num_seqs, int32_t max_pages, void* pool,
                   int32_t num_pages, int32_t T, void* ws, size_t ws_bytes, mla_stream_t stream) {
+  NvtxRange nvtx_range("mla_append_kv");
   int r = check_dims_impl(dims);
   if (r != MLA_OK) return r;
   if (T < 0 || num_seqs <= 0 || max_pages <= 0 || num_pages <= 0) return MLA_ERR_INVALID_ARG;
@@ -403,6 +416,7 @@ int mla_append_kv(const mla_dims* dims, const void* h, const void* w_dkv_kr, con
 
 int mla_absorb_query(const mla_dims* dims, const void* h, const void* w_dq, const void* w_uq_qr, const void* w_uk,
                      const int32_t* pos, void* q_out, int32_t B, void* ws, size_t ws_bytes, mla_stream_t stream) {
+  NvtxRange nvtx_range("mla_absorb_query");
   int r = check_dims_impl(dims);
   if (r != MLA_OK) return r;
   if (B < 0 || B > 65535) return MLA_ERR_INVALID_ARG;
@@ -425,6 +439,7 @@ int mla_decode_attention(const mla_dims* dims, const void* q, const void* pool, 
                          const int32_t* block_table, int32_t max_pages, const int32_t* seq_lens, int32_t B,
                          int32_t max_seq_len, void* o_lat, float* lse_out, void* ws, size_t ws_bytes,
                          mla_stream_t stream) {
+  NvtxRange nvtx_range("mla_decode_attention");
   int r = check_dims_impl(dims);
   if (r != MLA_OK) return r;
   if (B < 0 || B > 65535 || max_seq_len < 1 || max_seq_len > kMaxSeqLen || max_pages <= 0 || num_pages <= 0)
@@ -456,6 +471,7 @@ int mla_prefill_attention(const mla_dims* dims, const void* q, const void* pool,
                           const int32_t* block_table, int32_t num_seqs, int32_t max_pages, const int32_t* seq_idx,
                           const int32_t* pos, int32_t T, int32_t max_seq_len, void* o_lat, float* lse_out, void* ws,
                           size_t ws_bytes, mla_stream_t stream) {
+  NvtxRange nvtx_range("mla_prefill_attention");
   const int r = check_dims_impl(dims);
   if (r != MLA_OK) return r;
   if (T < 0 || max_seq_len < 1 || max_seq_len > kMaxSeqLen || num_seqs <= 0 || max_pages <= 0 || num_pages <= 0)
@@ -479,6 +495,7 @@ int mla_prefill_attention(const mla_dims* dims, const void* q, const void* pool,
 
 int mla_out_proj(const mla_dims* dims, const void* o_lat, const void* w_uv, const void* w_o, void* u, int32_t B,
                  void* ws, size_t ws_bytes, mla_stream_t stream) {
+  NvtxRange nvtx_range("mla_out_proj");
   int r = check_dims_impl(dims);
   if (r != MLA_OK) return r;
   if (B < 0 || B > 65535) return MLA_ERR_INVALID_ARG;
@@ -533,6 +550,16 @@ int mla_debug_gemm_plan(int32_t M, int32_t N, int32_t K, int32_t batch, int32_t 
   return MLA_OK;
 }
 
+int mla_debug_inject_missing_load(int32_t tile) {
+#ifdef MLA_FAULT_INJECT
+  if (tile < -1) return MLA_ERR_INVALID_ARG;
+  return cudaMemcpyToSymbol(tc::g_inject_missing_tile, &tile, sizeof(int)) == cudaSuccess ? MLA_OK : MLA_ERR_CUDA;
+#else
+  (void)tile;
+  return MLA_ERR_INVALID_ARG;
+#endif
+}
+
 int mla_set_decode_timing_events(mla_event_t before, mla_event_t after) {
   if ((before == nullptr) != (after == nullptr)) return MLA_ERR_INVALID_ARG;
   t_ev_before = reinterpret_cast<cudaEvent_t>(before);
@@ -572,6 +599,7 @@ extern "C" {
 int mla_decode_attention_noalloc(const mla_dims* dims, const void* q, const void* pool, int32_t num_pages,
                                  const int32_t* block_table, int32_t max_pages, const int32_t* seq_lens, int32_t B,
                                  int32_t max_seq_len, void* o_lat, float* lse_out, mla_stream_t stream) {
+  NvtxRange nvtx_range("mla_decode_attention_noalloc");
   const int r = check_dims_impl(dims);
   if (r != MLA_OK) return r;
   // the argument checks of mla_decode_attention come first, so that the size below is defined

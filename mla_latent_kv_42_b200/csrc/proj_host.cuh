@@ -1,7 +1,8 @@
 // Host side of the three projection calls (mla_append_kv, mla_absorb_query, mla_out_proj):
 // GEMM planning, TMA tensor maps, workspace layout and launches. Every product runs on the
-// tcgen05 GEMM; the CUDA-core kernels remain as a second implementation, selected by setting
-// MLA_PROJ_IMPL=simt in the environment (used to cross-check the two in tests).
+// tcgen05 GEMM, except the two per-head products when the head's slice is not a whole number of
+// 64-wide blocks (d_h % 64 for (W^UK_i)^T q^C_i, d_c % 64 for W^UV_i o_lat_i): the GEMM batches
+// heads by whole blocks, so those shapes take the CUDA-core kernels of proj_simt.cuh.
 // Included once, from libmla.cu.
 #pragma once
 
@@ -48,14 +49,6 @@ struct Carver {
   }
 };
 
-inline bool proj_uses_simt() {
-  static const bool v = [] {
-    const char* e = std::getenv("MLA_PROJ_IMPL");
-    return e != nullptr && std::strcmp(e, "simt") == 0;
-  }();
-  return v;
-}
-
 // ------------------------------------------------------------------ TMA tensor maps
 inline PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder() {
   static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
@@ -81,6 +74,22 @@ inline bool encode_2d(CUtensorMap* map, const void* base, bool bf16, uint64_t in
   cuuint32_t box[2] = {box_inner, box_outer};
   cuuint32_t es[2] = {1, 1};
   return fn(map, bf16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, const_cast<void*>(base),
+            dims, strides, box, es, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+            CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+// 3-D view of a row-major [rows][9 * 64] tensor of 16-bit elements, rows `row_bytes` apart, as
+// (64 columns, rows, 9 column chunks): one box of (64, 64, depth) lands in shared memory as
+// `depth` consecutive 64 x 64 chunks, each in the 128-byte-swizzled layout of a 2-D 64 x 64 box.
+inline bool encode_chunks(CUtensorMap* map, const void* base, bool bf16, uint64_t rows, uint64_t row_bytes,
+                          uint32_t depth) {
+  auto fn = tensor_map_encoder();
+  if (fn == nullptr) return false;
+  cuuint64_t dims[3] = {64, rows, 9};
+  cuuint64_t strides[2] = {row_bytes, 128};
+  cuuint32_t box[3] = {64, 64, depth};
+  cuuint32_t es[3] = {1, 1, 1};
+  return fn(map, bf16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 3, const_cast<void*>(base),
             dims, strides, box, es, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
@@ -252,8 +261,7 @@ void launch_rowdot(const T* W, const T* X, OutT* Y, int M, int K, int Tn, long l
 // ------------------------------------------------------------------ mla_append_kv
 struct AppendLayout {
   SkPlan g;
-  float* Y;     // CUDA-core route: fp32 [T, D]
-  float* part;  // tensor-core route: stream-K partials
+  float* part;  // stream-K partials
   float2* cs;   // RoPE cos/sin per token for the reduction of split tiles
   size_t bytes;
 };
@@ -262,9 +270,8 @@ inline AppendLayout append_layout(const mla_dims* d, int T_, void* ws) {
   const int D = d->d_c + d->d_rope;
   L.g = plan_sk(D, T_, d->d_model, 1, true, d->d_rope);
   Carver c{static_cast<char*>(ws)};
-  L.Y = proj_uses_simt() ? c.take<float>((size_t)T_ * D) : nullptr;
-  L.part = (!proj_uses_simt() && L.g.split) ? c.take<float>(L.g.part_bytes / sizeof(float)) : nullptr;
-  L.cs = (!proj_uses_simt() && L.g.split && L.g.n_tiles == 1) ? c.take<float2>((size_t)T_ * (d->d_rope / 2)) : nullptr;
+  L.part = L.g.split ? c.take<float>(L.g.part_bytes / sizeof(float)) : nullptr;
+  L.cs = (L.g.split && L.g.n_tiles == 1) ? c.take<float2>((size_t)T_ * (d->d_rope / 2)) : nullptr;
   L.bytes = c.off;
   return L;
 }
@@ -275,15 +282,6 @@ int append_run(const mla_dims* d, const void* h, const void* w, const int32_t* s
                void* ws, cudaStream_t st, int32_t& n) {
   const int D = d->d_c + d->d_rope;
   const AppendLayout L = append_layout(d, T_, ws);
-  if (proj_uses_simt()) {
-    launch_rowdot<T, float>(static_cast<const T*>(w), static_cast<const T*>(h), L.Y, D, d->d_model, T_, d->d_model,
-                            D, 1, 0, 0, 0, st, n);
-    k_append_epilogue<T><<<T_, 128, (d->d_rope / 2) * sizeof(float2), st>>>(
-        L.Y, 1, (long)T_ * D, seq_idx, pos, bt, num_seqs, max_pages, static_cast<T*>(pool), num_pages,
-        d->page_size, d->d_c, d->d_rope, d->rope_base);
-    ++n;
-    return MLA_OK;
-  }
   // [c^KV ; k^R] = W^{DKV,KR} h, RoPE on k^R, written to each token's cache slot
   tc::EpiParams e{};
   e.mode = tc::kEpiAppend;
@@ -291,6 +289,7 @@ int append_run(const mla_dims* d, const void* h, const void* w, const int32_t* s
   e.rope_lo = d->d_c;
   e.d_rope = d->d_rope;
   e.rope_base = d->rope_base;
+  e.rope_table = d->rope_inv_freq;
   e.pos = pos;
   e.seq_idx = seq_idx;
   e.bt = bt;
@@ -308,7 +307,6 @@ struct AbsorbLayout {
   SkPlan g1, g2, g3;
   void* cq;     // c^Q, element type [B, d_cq]
   void* qc;     // q^C, element type [B, n_h*d_h]
-  float* Y2;    // CUDA-core route: [q^C ; q^R before RoPE] fp32 [B, nq]
   float* part;  // stream-K partials, shared by the three products (they run one after another)
   float2* cs;   // RoPE cos/sin per token, filled by the W^DQ product for the query product
   size_t bytes;
@@ -317,19 +315,16 @@ struct AbsorbLayout {
 inline AbsorbLayout absorb_layout(const mla_dims* d, int B, void* ws) {
   AbsorbLayout L;
   const int nq = d->n_heads * (d->d_head + d->d_rope);
-  const bool simt = proj_uses_simt();
   L.g1 = plan_sk(d->d_cq, B, d->d_model, 1, false, d->d_rope);
   L.g2 = plan_sk(nq, B, d->d_cq, 1, true, d->d_rope);
   L.g3 = plan_sk(d->d_c, B, d->d_head, d->n_heads, false, d->d_rope);
-  L.tc_uk = !simt && d->d_head % 64 == 0;
+  L.tc_uk = d->d_head % 64 == 0;
   Carver c{static_cast<char*>(ws)};
   L.cq = c.take<uint16_t>((size_t)B * d->d_cq);
   L.qc = c.take<uint16_t>((size_t)B * d->n_heads * d->d_head);
-  L.Y2 = simt ? c.take<float>((size_t)B * nq) : nullptr;
-  size_t part = 0;
-  if (!simt) part = std::max(L.g1.part_bytes, std::max(L.g2.part_bytes, L.tc_uk ? L.g3.part_bytes : 0));
+  const size_t part = std::max(L.g1.part_bytes, std::max(L.g2.part_bytes, L.tc_uk ? L.g3.part_bytes : 0));
   L.part = part ? c.take<float>(part / sizeof(float)) : nullptr;
-  L.cs = !simt ? c.take<float2>((size_t)B * (d->d_rope / 2)) : nullptr;
+  L.cs = c.take<float2>((size_t)B * (d->d_rope / 2));
   L.bytes = c.off;
   return L;
 }
@@ -343,21 +338,14 @@ int absorb_run(const mla_dims* d, const void* h, const void* w_dq, const void* w
   const AbsorbLayout L = absorb_layout(d, B, ws);
   T* cq = static_cast<T*>(L.cq);
   T* qc = static_cast<T*>(L.qc);
-  if (proj_uses_simt()) {
-    launch_rowdot<T, T>(static_cast<const T*>(w_dq), static_cast<const T*>(h), cq, d->d_cq, d->d_model, B,
-                        d->d_model, d->d_cq, 1, 0, 0, 0, st, n);
-    launch_rowdot<T, float>(static_cast<const T*>(w_uq_qr), cq, L.Y2, nq, d->d_cq, B, d->d_cq, nq, 1, 0, 0, 0, st, n);
-    k_query_epilogue<T><<<B, 256, (d->d_rope / 2) * sizeof(float2), st>>>(
-        L.Y2, 1, (long)B * nq, pos, qc, static_cast<T*>(q_out), d->n_heads, d->d_head, d->d_rope, d->d_c,
-        d->rope_base);
-    ++n;
-  } else {
+  {
     // c^Q = W^DQ h; its CTAs also tabulate the query's RoPE cos/sin for the next product
     tc::EpiParams e1 = epi_plain(cq, d->d_cq, 0);
     e1.cs_prefill = L.cs;
     e1.pos = pos;
     e1.d_rope = d->d_rope;
     e1.rope_base = d->rope_base;
+    e1.rope_table = d->rope_inv_freq;
     int r = gemm_sk<T>({w_dq, d->d_cq, d->d_model, 0}, false, {h, B, d->d_model, 0}, d->d_cq, B, d->d_model, L.g1, e1,
                        L.part, st, n);
     if (r != MLA_OK) return r;
@@ -368,6 +356,7 @@ int absorb_run(const mla_dims* d, const void* h, const void* w_dq, const void* w
     e.rope_lo = nhd;
     e.d_rope = d->d_rope;
     e.rope_base = d->rope_base;
+    e.rope_table = d->rope_inv_freq;
     e.pos = pos;
     e.qc = qc;
     e.n_h = d->n_heads;
@@ -407,14 +396,12 @@ struct OutLayout {
 inline OutLayout out_layout(const mla_dims* d, int B, void* ws) {
   OutLayout L;
   const int nhd = d->n_heads * d->d_head;
-  const bool simt = proj_uses_simt();
   L.g_o = plan_sk(d->d_head, B, d->d_c, d->n_heads, false, d->d_rope);
   L.g_u = plan_sk(d->d_model, B, nhd, 1, false, d->d_rope);
-  L.tc_o = !simt && d->d_c % 64 == 0;
+  L.tc_o = d->d_c % 64 == 0;
   Carver c{static_cast<char*>(ws)};
   L.o = c.take<uint16_t>((size_t)B * nhd);
-  size_t part = 0;
-  if (!simt) part = std::max(L.tc_o ? L.g_o.part_bytes : 0, L.g_u.part_bytes);
+  const size_t part = std::max(L.tc_o ? L.g_o.part_bytes : 0, L.g_u.part_bytes);
   L.part = part ? c.take<float>(part / sizeof(float)) : nullptr;
   L.bytes = c.off;
   return L;
@@ -436,11 +423,6 @@ int out_run(const mla_dims* d, const void* o_lat, const void* w_uv, const void* 
                         (long)d->n_heads * d->d_c, nhd, d->n_heads, (long)d->d_head * d->d_c, d->d_c, d->d_head, st, n);
   }
   // u = W^O [o_1; ...; o_n_h]
-  if (proj_uses_simt()) {
-    launch_rowdot<T, T>(static_cast<const T*>(w_o), o, static_cast<T*>(u), d->d_model, nhd, B, nhd, d->d_model, 1, 0,
-                        0, 0, st, n);
-    return MLA_OK;
-  }
   return gemm_sk<T>({w_o, d->d_model, nhd, 0}, false, {o, B, nhd, 0}, d->d_model, B, nhd, L.g_u,
                     epi_plain(u, d->d_model, 0), L.part, st, n);
 }

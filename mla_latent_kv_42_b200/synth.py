@@ -29,7 +29,7 @@ import torch
 __all__ = [
     "Dims", "RUNNING", "PRODUCTION", "Workload", "WORKLOADS", "workload",
     "WEIGHT_ORDER", "weights", "hidden", "cached_lengths", "page_table", "prefix_rows",
-    "paged_pool", "synthetic_query", "to_storage", "storage_dtype",
+    "paged_pool", "synthetic_query", "to_storage", "storage_dtype", "yarn_inv_freq",
 ]
 
 
@@ -44,6 +44,7 @@ class Dims:
     page_size: int = 64
     dtype: str = "bf16"          # "bf16" or "fp16"
     rope_base: float = 10000.0
+    rope_inv_freq: tuple | None = None   # caller-supplied RoPE frequencies theta_k (d_h^R/2 of them)
 
     @property
     def D(self) -> int:
@@ -221,3 +222,19 @@ def synthetic_query(w: Workload, batch: int, scale: float = 1.0, seed_tag: int =
     q[..., :d.d_c] *= np.float32(s_qt * scale)
     q[..., d.d_c:] *= np.float32(s_qc * scale)
     return to_storage(q, d)
+
+
+def yarn_inv_freq(d_rope: int, base: float, factor: float = 40.0, original_ctx: int = 4096, beta_fast: float = 32.0,
+                  beta_slow: float = 1.0) -> tuple:
+    """An example caller-supplied RoPE frequency table (an input to the library, not part of its
+    arithmetic): YaRN's "NTK-by-parts" interpolation of theta_k = base^(-2k/d_rope) for a context
+    `factor` times `original_ctx`. Pair k makes r_k = original_ctx * theta_k / (2 pi) turns over the
+    original context; pairs with r_k >= beta_fast keep theta_k, pairs with r_k <= beta_slow take
+    theta_k / factor, and the ramp between is linear in r_k. The constants are illustrative."""
+    out = []
+    for k in range(d_rope // 2):
+        theta = base ** (-2.0 * k / d_rope)
+        r = original_ctx * theta / (2.0 * math.pi)
+        gamma = min(1.0, max(0.0, (r - beta_slow) / (beta_fast - beta_slow)))
+        out.append((1.0 - gamma) * theta / factor + gamma * theta)
+    return tuple(out)

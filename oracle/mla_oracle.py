@@ -41,6 +41,9 @@ Readings where the pages are silent:
      without its format): e4m3 bytes with two float32 scales per token, max|part| / 448 for c and for k^R,
      values divided by their scale in float32 and rounded to the nearest e4m3 value, ties to
      even. Attention over it is the attention over the rows it stands for.
+  R9 The RoPE frequencies may come from the caller ([S2] §4.1 applies YaRN to the decoupled key
+     to reach a 128K context; its constants are not on the pages): theta_k is then the table's
+     k-th entry, for the query and the key alike; positions and pairing are unchanged.
 
 Every function has pins in ``tests/test_oracle_pins.py``; none is "parity unpinned".
 """
@@ -97,14 +100,17 @@ def rope_frequencies(d_rope: int, base: float) -> np.ndarray:
     return np.power(float(base), -2.0 * k / d_rope)
 
 
-def rope(x, pos, base: float) -> np.ndarray:
+def rope(x, pos, base: float, inv_freq=None) -> np.ndarray:
     """RoPE(x, t): rotate each pair (x_2k, x_2k+1) by the angle t * theta_k ([S1] §3.1; R1, R2).
 
-    ``x`` has shape [..., d_R]; ``pos`` broadcasts against ``x.shape[:-1]``.
+    ``x`` has shape [..., d_R]; ``pos`` broadcasts against ``x.shape[:-1]``. ``inv_freq`` (d_R/2
+    values) replaces the base formula for theta_k when given: a caller-supplied table such as
+    YaRN's interpolated frequencies ([S2] §4.1; R9).
     """
     x = np.asarray(x, dtype=np.float64)
     pos = np.asarray(pos, dtype=np.float64)
-    phi = pos[..., None] * rope_frequencies(x.shape[-1], base)
+    theta = rope_frequencies(x.shape[-1], base) if inv_freq is None else np.asarray(inv_freq, dtype=np.float64)
+    phi = pos[..., None] * theta
     c, s = np.cos(phi), np.sin(phi)
     x0, x1 = x[..., 0::2], x[..., 1::2]
     y = np.empty(np.broadcast_shapes(x.shape, phi.shape[:-1] + (x.shape[-1],)), dtype=np.float64)
@@ -144,7 +150,7 @@ def kv_rows(w_dkv_kr, h, pos, dims) -> np.ndarray:
     w = as64(w_dkv_kr)
     h = as64(h)
     c = h @ w[:dims.d_c].T
-    k_r = rope(h @ w[dims.d_c:].T, np.asarray(pos), dims.rope_base)
+    k_r = rope(h @ w[dims.d_c:].T, np.asarray(pos), dims.rope_base, getattr(dims, "rope_inv_freq", None))
     return np.concatenate([c, k_r], axis=-1)
 
 
@@ -161,7 +167,7 @@ def query_path(w_dq, w_uq_qr, h, pos, dims):
     c_q = h @ as64(w_dq).T
     q_c = (c_q @ w_uq_qr[:n_h * d_h].T).reshape(-1, n_h, d_h)
     q_r_hat = (c_q @ w_uq_qr[n_h * d_h:].T).reshape(-1, n_h, d_r)
-    q_r = rope(q_r_hat, np.asarray(pos)[:, None], dims.rope_base)
+    q_r = rope(q_r_hat, np.asarray(pos)[:, None], dims.rope_base, getattr(dims, "rope_inv_freq", None))
     return c_q, q_c, q_r
 
 

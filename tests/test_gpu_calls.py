@@ -321,3 +321,62 @@ def test_layer_step_running_model_fp16():
     assert_parity(to64(q)[..., d.d_c:], absd["q"][..., d.d_c:], "q^R")
     assert_parity(to64(o_lat), absd["o_lat"], "o_lat")
     assert_parity(to64(u), naive["u"], "u")
+
+
+def test_layer_step_head_widths_off_the_gemm_blocks():
+    """Dims whose per-head slices are not whole 64-wide blocks (d_h = 40, d_c = 96): the two
+    per-head products take the CUDA-core kernels (k_absorb_uk for (W^UK_i)^T q^C_i, k_rowdot for
+    W^UV_i o_lat_i), the rest the tensor-core GEMM, attention the CUDA-core kernel with 16-token
+    pages; a whole layer step through the C ABI against the naive and absorbed oracle."""
+    d = synth.Dims(d_model=256, n_heads=4, d_head=40, d_c=96, d_cq=72, d_rope=16, page_size=16)
+    w = synth.Workload("odd_dims_b3", d, 3, 0, 1, 0.05, "shuffled")
+    cached = np.array([0, 17, 300])
+    L = harness.make_layer(w, cached)
+    ix = harness.step_index(cached)
+    h = synth.hidden(w)
+    u, q, o_lat, lse = M.layer_step(L.state, h.cuda(), ix.pos, ix.seq_idx, ix.seq_lens, ix.max_seq_len)
+    assert M.read_device_status() == 0
+    W64 = {k: O.as64(v) for k, v in L.W_host.items()}
+    prefix = [O.as64(L.prefix(b)) for b in range(w.batch)]
+    naive = O.layer_step_naive(W64, O.as64(h), prefix, d)
+    absd = O.layer_step_absorbed(W64, O.as64(h), prefix, d)
+    assert_parity(to64(q)[..., :d.d_c], absd["q"][..., :d.d_c], "q~")
+    assert_parity(to64(q)[..., d.d_c:], absd["q"][..., d.d_c:], "q^R")
+    assert_parity(to64(o_lat), absd["o_lat"], "o_lat")
+    assert_parity(to64(u), naive["u"], "u")
+
+
+@pytest.mark.parametrize("fam", ["running_bf16", "production_bf16"])
+def test_caller_rope_table_in_append_and_absorb(fam):
+    """A caller-supplied RoPE frequency table (mla_dims.rope_inv_freq; here a YaRN-style
+    interpolation for a 40x longer context) replaces base^(-2k/d_R) in the k^R the append writes
+    and in the q^R the query path produces, at positions up to 131072 (one n tile and, with 300
+    tokens, several)."""
+    w0 = FAMILIES[fam]
+    d = w0.dims.with_(rope_inv_freq=synth.yarn_inv_freq(w0.dims.d_rope, w0.dims.rope_base))
+    W, W64 = weights64(w0)
+    for T in (19, 300):
+        pos = ((np.arange(T, dtype=np.int64) * 7919) % 131073).astype(np.int32)
+        seq_idx = np.arange(T, dtype=np.int32)
+        # one physical page per token, at its logical page pos // P (the other entries unused)
+        max_pages = int(pos.max()) // d.page_size + 1
+        bt = np.full((T, max_pages), -1, dtype=np.int32)
+        bt[np.arange(T), pos // d.page_size] = np.random.default_rng(T).permutation(T)
+        num_pages = T
+        h = synth.hidden(w0, step=3, batch=T)
+        pool = torch.zeros((num_pages, d.page_size, d.D), dtype=synth.storage_dtype(d), device="cuda")
+        M.append_kv(d, h.cuda(), W["w_dkv_kr"].cuda(), torch.from_numpy(seq_idx).cuda(), torch.from_numpy(pos).cuda(),
+                    torch.from_numpy(bt).cuda(), pool)
+        q = M.absorb_query(d, h.cuda(), W["w_dq"].cuda(), W["w_uq_qr"].cuda(), W["w_uk"].cuda(),
+                           torch.from_numpy(pos).cuda())
+        assert M.read_device_status() == 0
+        slots = np.array([O.page_slot(bt, s_, p_, d.page_size) for s_, p_ in zip(seq_idx, pos)])
+        got = to64(pool.view(-1, d.D)[torch.from_numpy(slots).cuda()])
+        ref = O.kv_rows(W64["w_dkv_kr"], O.as64(h), pos, d)
+        assert_parity(got[:, d.d_c:], ref[:, d.d_c:], f"k^R with the table, T={T}")
+        # the table matters: the base formula's k^R is far from what was written
+        plain = O.kv_rows(W64["w_dkv_kr"], O.as64(h), pos, w0.dims)
+        assert np.abs(plain[:, d.d_c:] - got[:, d.d_c:]).max() > 10 * np.abs(ref[:, d.d_c:] - got[:, d.d_c:]).max()
+        refq = O.absorb_query(W64["w_dq"], W64["w_uq_qr"], W64["w_uk"], O.as64(h), pos, d)
+        assert_parity(to64(q)[..., d.d_c:], refq[..., d.d_c:], f"q^R with the table, T={T}")
+        assert_parity(to64(q)[..., :d.d_c], refq[..., :d.d_c], f"q~, T={T}")

@@ -13,6 +13,7 @@ import torch
 
 import oracle as O
 from conftest import read_golden
+from mla_latent_kv_42_b200 import synth
 from mla_latent_kv_42_b200.synth import RUNNING, PRODUCTION, Dims
 
 TINY = Dims(d_model=12, n_heads=3, d_head=4, d_c=6, d_cq=5, d_rope=4, page_size=4, rope_base=100.0)
@@ -135,6 +136,40 @@ def test_rope_frequency_closed_forms():
     e[0] = 1.0
     y = O.rope(e, 1, 10000.0)
     assert y[0] == pytest.approx(math.cos(1.0)) and y[1] == pytest.approx(math.sin(1.0))
+
+
+def test_rope_with_a_caller_table():
+    """A caller-supplied frequency table (reading R9): the default table reproduces the base formula
+    exactly; any table is still a rotation whose scores depend only on t - j; pair k turns by
+    t * table[k] (checked on unit vectors); and a table that differs changes k^R and q^R."""
+    rng = np.random.default_rng(6)
+    x = rng.standard_normal((7, 64))
+    pos = np.array([0, 1, 63, 4096, 40000, 131071, 131072])
+    np.testing.assert_array_equal(O.rope(x, pos, 10000.0, O.rope_frequencies(64, 10000.0)), O.rope(x, pos, 10000.0))
+    table = np.asarray(synth.yarn_inv_freq(64, 10000.0))
+    y = O.rope(x, pos, 10000.0, table)
+    np.testing.assert_allclose(np.linalg.norm(y, axis=1), np.linalg.norm(x, axis=1), rtol=1e-13)
+    q, k = rng.standard_normal((2, 64))
+    ref = O.rope(q, 4100, 10000.0, table) @ O.rope(k, 17, 10000.0, table)
+    assert O.rope(q, 4100 + 90000, 10000.0, table) @ O.rope(k, 17 + 90000, 10000.0, table) == pytest.approx(ref,
+                                                                                                             abs=1e-9)
+    for kk in (0, 13, 31):
+        e = np.zeros(64)
+        e[2 * kk] = 1.0
+        yy = O.rope(e, 1000, 10000.0, table)
+        assert yy[2 * kk] == pytest.approx(math.cos(1000 * table[kk]), abs=1e-12)
+        assert yy[2 * kk + 1] == pytest.approx(math.sin(1000 * table[kk]), abs=1e-12)
+    assert np.abs(y - O.rope(x, pos, 10000.0)).max() > 0.1
+    # the example table keeps the fastest pairs and divides the slowest by the factor
+    base = O.rope_frequencies(64, 10000.0)
+    assert table[0] == base[0] and table[-1] == pytest.approx(base[-1] / 40.0, rel=1e-15)
+    # the projections read the table from the dims
+    d = synth.RUNNING.with_(rope_inv_freq=tuple(synth.yarn_inv_freq(32, 10000.0)))
+    w = rng.standard_normal((d.D, d.d_model)) * 0.02
+    h = rng.standard_normal((2, d.d_model))
+    rows = O.kv_rows(w, h, [5000, 7], d)
+    np.testing.assert_allclose(rows[:, d.d_c:], O.rope(h @ w[d.d_c:].T, np.array([5000, 7]), 10000.0,
+                                                       d.rope_inv_freq), atol=1e-12)
 
 
 # ----------------------------------------------------------------------------- attention
