@@ -97,28 +97,47 @@ __global__ void __launch_bounds__(256) k_decode_simt(
 }
 
 // Merge of split-KV partials: o = sum_s w_s o_s / sum_s w_s with w_s = e^{lse_s - max lse},
-// summed in split order. One block per (b, head); o_part [BH][S][d_c], lse_part [BH][S].
+// summed in split order. One warp per (b, head), lanes over the latent columns (d_c <= 512, a
+// multiple of 8), every split's loads in flight together; grid ceil(B n_h / 8), 256 threads.
+// o_part [BH][S][d_c], lse_part [BH][S].
 template <typename T>
-__global__ void k_lse_merge(const float* __restrict__ o_part, const float* __restrict__ lse_part, int n_splits,
-                            int d_c, T* __restrict__ o_lat, float* __restrict__ lse_out) {
-  const long bh = blockIdx.x;
+__global__ void __launch_bounds__(256) k_lse_merge_warp(const float* __restrict__ o_part,
+                                                         const float* __restrict__ lse_part, int n_splits, int d_c,
+                                                         long BH, T* __restrict__ o_lat, float* __restrict__ lse_out) {
+  griddep_wait();
+  if (threadIdx.x == 0) griddep_launch();
+  const long bh = (long)blockIdx.x * 8 + (threadIdx.x >> 5);
+  const int lane = threadIdx.x & 31;
+  if (bh >= BH) return;
   const float* lp = lse_part + bh * n_splits;
   float mx = -INFINITY;
-  for (int s = 0; s < n_splits; ++s) mx = fmaxf(mx, lp[s]);
+  for (int s = lane; s < n_splits; s += 32) mx = fmaxf(mx, lp[s]);
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+  float acc[16];
+#pragma unroll
+  for (int j = 0; j < 16; ++j) acc[j] = 0.f;
   float z = 0.f;
-  if (mx != -INFINITY)
-    for (int s = 0; s < n_splits; ++s) z += exp2f((lp[s] - mx) * kLog2e);
-  const float inv = z > 0.f ? 1.f / z : 0.f;
-  for (int e = threadIdx.x; e < d_c; e += blockDim.x) {
-    float acc = 0.f;
-    if (z > 0.f)
-      for (int s = 0; s < n_splits; ++s) {
-        const float w = exp2f((lp[s] - mx) * kLog2e);
-        acc = fmaf(w, o_part[(bh * n_splits + s) * d_c + e], acc);
+  if (mx != -INFINITY) {
+#pragma unroll 4
+    for (int s = 0; s < n_splits; ++s) {
+      const float w = exp2f((lp[s] - mx) * kLog2e);  // -inf partials (no tokens) weigh 0
+      z += w;
+      const float* src = o_part + (bh * n_splits + s) * d_c;
+#pragma unroll
+      for (int j = 0; j < 16; ++j) {
+        const int e = lane + 32 * j;
+        if (e < d_c) acc[j] = fmaf(w, src[e], acc[j]);
       }
-    Out<T>::put(o_lat + bh * d_c + e, acc * inv);
+    }
   }
-  if (lse_out != nullptr && threadIdx.x == 0) lse_out[bh] = z > 0.f ? mx + logf(z) : -INFINITY;
+  const float inv = z > 0.f ? 1.f / z : 0.f;
+#pragma unroll
+  for (int j = 0; j < 16; ++j) {
+    const int e = lane + 32 * j;
+    if (e < d_c) Out<T>::put(o_lat + bh * d_c + e, acc[j] * inv);
+  }
+  if (lse_out != nullptr && lane == 0) lse_out[bh] = z > 0.f ? mx + logf(z) : -INFINITY;
 }
 
 }  // namespace mla

@@ -53,6 +53,7 @@ constexpr int kSetOff = kRopeOff + kChunk;    // two sets of 8 latent chunks
 constexpr int kSetBytes = 8 * kChunk;
 constexpr int kDataBytes = kSetOff + 2 * kSetBytes;  // 229376
 constexpr float kLazy = 8.f;       // rescale threshold in log2 units
+constexpr int kAhead = 3;          // tiles between a page's L2 prefetch and its shared-memory load
 constexpr int kSoftWarps = 8;      // warps 0-7: softmax, rescale, epilogue
 constexpr int kLoadWarp = 8;       // Q, rope and own-page latent loads
 constexpr int kMmaWarp = 9;        // TMEM allocation; rank 0: MMA issue
@@ -73,7 +74,7 @@ struct Ctrl {
   uint64_t o_free;         // O read out by all 16 softmax warps (end of a sequence's item)
   // Barriers arrived by rank 0's MMA commits, multicast to both CTAs.
   uint64_t qk_done[2][4];  // set s, the S MMAs of pair p are complete (its slots may be reused)
-  uint64_t set_free[2];    // the O MMAs of the tile using set s are complete
+  uint64_t set_free[2][2];  // the O MMAs of the tile using set s are done with its chunks [4h, 4h + 4)
   uint64_t rope_done, q_free;
   uint64_t s_full[2], p_free;
   // Local barriers.
@@ -102,10 +103,11 @@ struct DecodeTcParams {
 };
 
 // Tensor maps of the attention kernel: the paged pool viewed as [pages * 64 rows, 576] with one
-// 64 x 64 box (rope), and as (64 columns, rows, 9 column chunks) with boxes of 2 and 4 chunks;
-// the queries viewed as (64 columns, B * n_h rows, 9 chunks) with a box of 9 chunks.
+// 64 x 64 box (rope), and as (64 columns, rows, 9 column chunks) with boxes of 2, 4 and 9 chunks
+// (the last for L2 prefetches of whole pages); the queries viewed as (64 columns, B * n_h rows,
+// 9 chunks) with a box of 9 chunks.
 struct DecodeTcMaps {
-  CUtensorMap pool1, pool2, pool4, q9;
+  CUtensorMap pool1, pool2, pool4, pool9, q9;
 };
 
 // Tiles [t0, t1) of sequence b handled by this pair (n_b = tiles of the sequence).
@@ -179,6 +181,13 @@ __device__ __forceinline__ void tma_load_3d(uint32_t dst, const CUtensorMap* map
       "l"(reinterpret_cast<uint64_t>(map)), "r"(bar), "r"(x), "r"(y), "r"(z)
       : "memory");
 }
+// Prefetch a 3-D box into L2 (no shared memory, no barrier).
+__device__ __forceinline__ void tma_prefetch_3d(const CUtensorMap* map, int x, int y, int z) {
+  asm volatile("cp.async.bulk.prefetch.tensor.3d.L2.global.tile [%0, {%1, %2, %3}];" ::"l"(
+                   reinterpret_cast<uint64_t>(map)),
+               "r"(x), "r"(y), "r"(z)
+               : "memory");
+}
 __device__ __forceinline__ void tma_load_3d_pair(uint32_t dst, const CUtensorMap* map, uint32_t cluster_bar, int x,
                                                  int y, int z) {
   asm volatile(
@@ -213,7 +222,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(dec::kThreads, 1)
         mbar_init(bar(ctl->fix_full[s][q]), 1);
       }
       mbar_init(bar(ctl->s_free[s]), 2 * kSoftWarps);
-      mbar_init(bar(ctl->set_free[s]), 1);
+      mbar_init(bar(ctl->set_free[s][0]), 1);
+      mbar_init(bar(ctl->set_free[s][1]), 1);
       mbar_init(bar(ctl->s_full[s]), 1);
     }
     mbar_init(bar(ctl->rope_full), 2);
@@ -269,42 +279,67 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(dec::kThreads, 1)
         tma_prefetch_map(&maps.pool1);
         tma_prefetch_map(&maps.pool2);
         tma_prefetch_map(&maps.pool4);
+        tma_prefetch_map(&maps.pool9);
         tma_prefetch_map(&maps.q9);
         Cursor c;
         c.start(prefix, p.B, cluster, nclusters);
+        int L = 0;
+        // A second cursor runs kAhead tiles ahead and prefetches its own page into L2, so that the
+        // shared-memory loads of that tile, issued once its set is free, read from L2.
+        Cursor ahead;
+        ahead.start(prefix, p.B, cluster, nclusters);
+        int L_ahead = ahead.valid ? p.seq_lens[ahead.item.b] : 0;
+        auto prefetch_ahead = [&]() {
+          const int pi = 2 * ahead.t + (int)rank;
+          if (kPage * pi < L_ahead) tma_prefetch_3d(&maps.pool9, 0, p.bt[(long)ahead.item.b * p.max_pages + pi] * kPage, 0);
+          const int ii = ahead.ii;
+          ahead.advance(prefix);
+          if (ahead.valid && ahead.ii != ii) L_ahead = p.seq_lens[ahead.item.b];
+        };
+        for (int k = 0; k < kAhead && ahead.valid; ++k) prefetch_ahead();
         while (c.valid) {
           const int s = c.ti & 1, b = c.item.b, t = c.t;
-          const int L = p.seq_lens[b];
+          // global reads first: their latency overlaps the waits below
+          if (c.first()) L = p.seq_lens[b];
+          const int* btb = p.bt + (long)b * p.max_pages;
+          const int page_idx = 2 * t + (int)rank;
+          const bool own = kPage * page_idx < L;  // page r of the tile holds tokens
+          const int page = own ? btb[page_idx] : 0;
           if (c.first()) {  // this CTA's 64 heads of the sequence's queries, after the last S MMA of the item before
             if (!wait(ctl->q_free, (c.ii & 1) ^ 1)) break;
-            mbar_arrive_expect_tx_remote(lead(ctl->q_full), 9 * kChunk);
+            mbar_arrive_expect_tx_cl(lead(ctl->q_full), 9 * kChunk);
             tma_load_3d_pair(data_u32 + kQOff, &maps.q9, lead(ctl->q_full), 0, b * p.n_h + 64 * (int)rank, 0);
           }
-          const bool own = kTile * t + kPage * (int)rank < L;  // page r of the tile holds tokens
-          const int page = own ? p.bt[(long)b * p.max_pages + 2 * t + (int)rank] : 0;
           if (!wait(ctl->rope_done, (c.ti & 1) ^ 1)) break;
           if (own) {
-            mbar_arrive_expect_tx_remote(lead(ctl->rope_full), kChunk);
+            mbar_arrive_expect_tx_cl(lead(ctl->rope_full), kChunk);
             tma_load_2d_pair(data_u32 + kRopeOff, &maps.pool1, lead(ctl->rope_full), kDc, page * kPage);
           } else {
-            mbar_arrive_remote(lead(ctl->rope_full));
+            mbar_arrive_cl(lead(ctl->rope_full));
           }
-          if (!wait(ctl->set_free[s], ((c.ti >> 1) & 1) ^ 1)) break;  // the O MMAs of tile ti - 2 are done
+          bool ok = true;
           for (int h = 0; h < 2; ++h) {
+            // the O MMAs of tile ti - 2 are done with chunks [4h, 4h + 4) of set s
+            if (!wait(ctl->set_free[s][h], ((c.ti >> 1) & 1) ^ 1)) {
+              ok = false;
+              break;
+            }
 #ifdef MLA_FAULT_INJECT
             if (own && h == 0 && rank == 0 && prefix[b] + t == g_inject_missing_tile) {
-              mbar_arrive_expect_tx_remote(lead(ctl->qk_full[s][h]), 4 * kChunk);
+              mbar_arrive_expect_tx_cl(lead(ctl->qk_full[s][h]), 4 * kChunk);
               continue;
             }
 #endif
             if (own) {
-              mbar_arrive_expect_tx_remote(lead(ctl->qk_full[s][h]), 4 * kChunk);
+              mbar_arrive_expect_tx_cl(lead(ctl->qk_full[s][h]), 4 * kChunk);
               tma_load_3d_pair(set_u32 + s * kSetBytes + 4 * h * kChunk, &maps.pool4, lead(ctl->qk_full[s][h]), 0,
                                page * kPage, 4 * h);
             } else {
-              mbar_arrive_remote(lead(ctl->qk_full[s][h]));
+              mbar_arrive_cl(lead(ctl->qk_full[s][h]));
             }
           }
+          if (!ok) break;
+          if (ahead.valid) prefetch_ahead();
           c.advance(prefix);
         }
       }
@@ -320,20 +355,24 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(dec::kThreads, 1)
       c.start(prefix, p.B, cluster, nclusters);
       uint32_t fix_par = 0;
       bool ok = true;
+      int L = 0;
       while (ok && c.valid) {
         const int s = c.ti & 1, b = c.item.b, t = c.t;
-        const int L = p.seq_lens[b];
+        if (c.first()) L = p.seq_lens[b];
         const uint32_t ph = (c.ti >> 1) & 1;
         const int* btb = p.bt + (long)b * p.max_pages;
+        const int g_other = 1 - (int)rank;
+        const bool whole_tile = kTile * (t + 1) <= L;
+        const int page_other = whole_tile ? btb[2 * t + g_other] : 0;  // read ahead of the wait below
         // the O MMAs of tile ti - 2 are complete, so every barrier of set s is in this tile's phase
-        if (!wwait(ctl->set_free[s], ph ^ 1)) break;
-        if (kTile * (t + 1) <= L) {  // whole tile
+        if (!wwait(ctl->set_free[s][1], ph ^ 1)) break;
+        if (whole_tile) {
           if (lane == 0) {
-            mbar_arrive_remote(lead(ctl->pv_full[s][(int)rank]));      // j = 0, g = r
-            mbar_arrive_remote(lead(ctl->pv_full[s][2 + (int)rank]));  // j = 1, g = r
+            mbar_arrive_cl(lead(ctl->pv_full[s][(int)rank]));      // j = 0, g = r
+            mbar_arrive_cl(lead(ctl->pv_full[s][2 + (int)rank]));  // j = 1, g = r
           }
-          const int g = 1 - (int)rank;
-          const int page = btb[2 * t + g];
+          const int g = g_other;
+          const int page = page_other;
           for (int j = 0; j < 2; ++j) {
             const int pr = 2 * j + g;
             if (!wwait(ctl->qk_done[s][pr], ph)) {
@@ -341,7 +380,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(dec::kThreads, 1)
               break;
             }
             if (lane == 0) {
-              mbar_arrive_expect_tx_remote(lead(ctl->pv_full[s][pr]), 2 * kChunk);
+              mbar_arrive_expect_tx_cl(lead(ctl->pv_full[s][pr]), 2 * kChunk);
               tma_load_3d_pair(set_u32 + s * kSetBytes + 2 * pr * kChunk, &maps.pool2, lead(ctl->pv_full[s][pr]), 0,
                                page * kPage, 4 * j + 2 * (int)rank);
             }
@@ -378,88 +417,106 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(dec::kThreads, 1)
               }
               fence_proxy_async_cta();
               __syncwarp();
-              if (lane == 0) mbar_arrive_remote(lead(ctl->pv_full[s][pr]));
+              if (lane == 0) mbar_arrive_cl(lead(ctl->pv_full[s][pr]));
             }
         }
         c.advance(prefix);
       }
     } else if (warp == kMmaWarp) {
       // ---------------------------------------------------------------- MMA issue (rank 0, one lane)
-      // Two cursors: S MMAs of tile qc (rope chunk, then the 8 latent chunks) and O MMAs of tile
-      // pc < qc (pairs in the order (g, j) = (0,0), (0,1), (1,0), (1,1)). Whichever step is ready
-      // is issued, the O step first, so that a tile's sets are freed as early as possible.
+      // Tiles in order, each as its S step followed by the O step of the tile before it: S(i),
+      // O(i - 1), S(i + 1), O(i), ... The softmax of tile i - 1 runs while S(i) executes, and the
+      // set of tile i - 1 is released as soon as O(i - 1) completes. One thread issues all MMAs
+      // of the pair, and a single thread runs dependent instructions and branches at a few cycles
+      // each, so the issue path is straight-line code: per step a fixed sequence of waits, MMAs
+      // with compile-time operand offsets, and commits. Each descriptor is a fixed high word and
+      // a low word stepped by 32-bit adds (16-byte units: a K-step of 16 elements is +2 along a
+      // K-major row and +128, i.e. 16 rows, down an MN-major operand).
       if (rank == 0 && lane == 0) {
-        const uint32_t idesc_qk = idesc_f16(128, kTile, kBf16, false, false);
-        const uint32_t idesc_pv = idesc_f16(128, 256, kBf16, false, true);
-        Cursor qc, pc;
-        qc.start(prefix, p.B, cluster, nclusters);
-        pc.start(prefix, p.B, cluster, nclusters);
-        int cq = 0, gq = 0;
-        uint64_t t_idle = globaltimer();
-        while (qc.valid || pc.valid) {
-          bool did = false;
-          if (pc.valid && (!qc.valid || pc.ti < qc.ti)) {
-            const int s = pc.ti & 1, g = gq >> 1, j = gq & 1, pr = 2 * j + g;
-            bool ready = mbar_test_cluster(bar(ctl->pv_full[s][pr]), (pc.ti >> 1) & 1);
-            if (ready && gq == 0)
-              ready = mbar_test_cluster(bar(ctl->p_full), pc.ti & 1) &&
-                      (!pc.first() || mbar_test_cluster(bar(ctl->o_free), (pc.ii & 1) ^ 1));
-            if (ready) {
-              tc_fence_after();
-              const uint32_t pa = data_u32 + kPOff + g * kChunk;
-              const uint32_t vb = set_u32 + s * kSetBytes + 2 * pr * kChunk;
+        constexpr uint32_t idesc_qk = idesc_f16(128, kTile, kBf16, false, false);
+        constexpr uint32_t idesc_pv = idesc_f16(128, 256, kBf16, false, true);
+        constexpr uint32_t hi = desc_sw128_hi(1024);
+        constexpr uint32_t kChunkD = kChunk >> 4, kSetD = kSetBytes >> 4;
+        const uint32_t q_lo = desc_sw128_lo(data_u32 + kQOff, 16);
+        const uint32_t p_lo = desc_sw128_lo(data_u32 + kPOff, 16);
+        const uint32_t rope_lo = desc_sw128_lo(data_u32 + kRopeOff, 16);
+        const uint32_t k_lo = desc_sw128_lo(set_u32, 16);      // latent chunks as K-major B of S
+        const uint32_t v_lo = desc_sw128_lo(set_u32, kChunk);  // chunk pairs as MN-major B of O
+        const uint32_t b_qk_full = bar(ctl->qk_full[0][0]), b_pv_full = bar(ctl->pv_full[0][0]);
+        const uint32_t b_qk_done = bar(ctl->qk_done[0][0]), b_set_free = bar(ctl->set_free[0][0]);
+        const uint32_t b_s_free = bar(ctl->s_free[0]), b_s_full = bar(ctl->s_full[0]);
+        auto mwait = [&](uint32_t b, uint32_t parity) {
+          if (mbar_wait(b, parity, abort_flag)) return true;
+          st_cluster_u32(peer_abort, 1u);
+          return false;
+        };
+        // S(ti) = Q C^T into S buffer ti & 1: the rope chunk, then latent chunks 0-7.
+        auto s_step = [&](int ti, bool first, bool last, int ii) {
+          const int s = ti & 1;
+          const uint32_t ph = (ti >> 1) & 1;
+          if (!mwait(b_s_free + 8 * s, ph ^ 1)) return false;  // softmax has read S(ti - 2)
+          if (first && !mwait(bar(ctl->q_full), ii & 1)) return false;
+          if (!mwait(bar(ctl->rope_full), ti & 1)) return false;
+          tc_fence_after();
+          const uint32_t d = tmem + kSCol + 64 * s;
+#pragma unroll
+          for (int ks = 0; ks < 4; ++ks)
+            mma2_ss_lohi(d, q_lo + 8 * kChunkD + 2 * ks, rope_lo + 2 * ks, hi, idesc_qk, ks != 0);
+          mma_commit2(bar(ctl->rope_done), 3);
+          const uint32_t kb = k_lo + s * kSetD;
+#pragma unroll
+          for (int hh = 0; hh < 2; ++hh) {
+            if (!mwait(b_qk_full + 8 * (2 * s + hh), ph)) return false;
+            tc_fence_after();
+#pragma unroll
+            for (int kc = 4 * hh; kc < 4 * hh + 4; ++kc) {
 #pragma unroll
               for (int ks = 0; ks < 4; ++ks)
-                mma2_ss(tmem + kOCol + 128 * j, desc_sw128(pa + ks * 32, 16, 1024),
-                        desc_sw128(vb + ks * 2048, kChunk, 1024), idesc_pv, !(pc.first() && g == 0 && ks == 0));
-              if (++gq == 4) {
-                gq = 0;
-                mma_commit2(bar(ctl->p_free), 3);
-                mma_commit2(bar(ctl->set_free[s]), 3);
-                pc.advance(prefix);
-              }
-              did = true;
+                mma2_ss_lohi(d, q_lo + kc * kChunkD + 2 * ks, kb + kc * kChunkD + 2 * ks, hi, idesc_qk, 1);
+              if (kc & 1) mma_commit2(b_qk_done + 8 * (4 * s + (kc >> 1)), 3);
             }
           }
-          if (!did && qc.valid) {
-            const int s = qc.ti & 1, sb = qc.ti & 1;
-            bool ready = true;
-            if (cq == 0)
-              ready = mbar_test_cluster(bar(ctl->rope_full), qc.ti & 1) &&
-                      mbar_test_cluster(bar(ctl->s_free[sb]), ((qc.ti >> 1) & 1) ^ 1) &&
-                      (!qc.first() || mbar_test_cluster(bar(ctl->q_full), qc.ii & 1));
-            else if (cq == 1 || cq == 5)
-              ready = mbar_test_cluster(bar(ctl->qk_full[s][(cq - 1) >> 2]), (qc.ti >> 1) & 1);
-            if (ready) {
-              tc_fence_after();
-              const int kc = cq == 0 ? 8 : cq - 1;
-              const uint32_t bsl = cq == 0 ? data_u32 + kRopeOff : set_u32 + s * kSetBytes + kc * kChunk;
+          mma_commit2(b_s_full + 8 * s, 3);
+          if (last) mma_commit2(bar(ctl->q_free), 3);
+          return true;
+        };
+        // O += P C_lat for tile ti: pairs (g, j) = (0,0), (1,0), (0,1), (1,1); chunks 0-3 of the
+        // set are released after the first two.
+        auto o_step = [&](int ti, bool first, int ii) {
+          const int s = ti & 1;
+          const uint32_t ph = (ti >> 1) & 1;
+          if (!mwait(bar(ctl->p_full), ti & 1)) return false;  // P written, O rescaled
+          if (first && !mwait(bar(ctl->o_free), (ii & 1) ^ 1)) return false;  // O of the item before read out
+          const uint32_t vb = v_lo + s * kSetD;
 #pragma unroll
-              for (int ks = 0; ks < 4; ++ks)
-                mma2_ss(tmem + kSCol + 64 * sb, desc_sw128(data_u32 + kQOff + kc * kChunk + ks * 32, 16, 1024),
-                        desc_sw128(bsl + ks * 32, 16, 1024), idesc_qk, (cq | ks) != 0);
-              if (cq == 0) mma_commit2(bar(ctl->rope_done), 3);
-              else if ((kc & 1) == 1) mma_commit2(bar(ctl->qk_done[s][kc >> 1]), 3);
-              if (++cq == 9) {
-                cq = 0;
-                mma_commit2(bar(ctl->s_full[sb]), 3);
-                if (qc.last()) mma_commit2(bar(ctl->q_free), 3);
-                qc.advance(prefix);
-              }
-              did = true;
-            }
+          for (int gq = 0; gq < 4; ++gq) {
+            const int g = gq & 1, jh = gq >> 1, pr = 2 * jh + g;
+            if (!mwait(b_pv_full + 8 * (4 * s + pr), ph)) return false;
+            tc_fence_after();
+            const uint32_t d = tmem + kOCol + 128 * jh;
+            mma2_ss_lohi(d, p_lo + g * kChunkD, vb + 2 * pr * kChunkD, hi, idesc_pv, g != 0 || !first);
+#pragma unroll
+            for (int ks = 1; ks < 4; ++ks)
+              mma2_ss_lohi(d, p_lo + g * kChunkD + 2 * ks, vb + 2 * pr * kChunkD + 128 * ks, hi, idesc_pv, 1);
+            if (gq == 1) mma_commit2(b_set_free + 8 * (2 * s), 3);
           }
-          if (did) {
-            t_idle = globaltimer();
-          } else if (*abort_flag) {
-            break;
-          } else if (globaltimer() - t_idle > kWaitLimitNs) {
-            record_error(MLA_ERR_TIMEOUT);
-            *abort_flag = 1;
-            st_cluster_u32(peer_abort, 1u);
-            break;
-          }
+          mma_commit2(bar(ctl->p_free), 3);
+          mma_commit2(b_set_free + 8 * (2 * s + 1), 3);
+          return true;
+        };
+        Cursor c;
+        c.start(prefix, p.B, cluster, nclusters);
+        int prev_ti = -1, prev_ii = 0;
+        bool prev_first = false;
+        while (c.valid) {
+          if (!s_step(c.ti, c.first(), c.last(), c.ii)) break;
+          if (prev_ti >= 0 && !o_step(prev_ti, prev_first, prev_ii)) break;
+          prev_ti = c.ti;
+          prev_first = c.first();
+          prev_ii = c.ii;
+          c.advance(prefix);
         }
+        if (!c.valid && prev_ti >= 0) o_step(prev_ti, prev_first, prev_ii);
       }
       __syncwarp();
     } else if (warp < kSoftWarps) {
@@ -511,7 +568,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(dec::kThreads, 1)
         tmem_wait_ld();
         tc_fence_before();
         __syncwarp();
-        if (lane == 0) mbar_arrive_remote(lead(ctl->s_free[sb]));
+        if (lane == 0) mbar_arrive_cl(lead(ctl->s_free[sb]));
         // tokens past the sequence end become -inf (weight exactly 0), whatever the slot held
         const int nv = max(0, min(32, L - (kTile * t + kPage * g + 32 * ch)));
         if (nv < 32) {
@@ -577,7 +634,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(dec::kThreads, 1)
         fence_proxy_async_cta();
         tc_fence_before();
         __syncwarp();
-        if (lane == 0) mbar_arrive_remote(lead(ctl->p_full));
+        if (lane == 0) mbar_arrive_cl(lead(ctl->p_full));
 
         if (c.last()) {  // ---- epilogue of the item: O / l for this thread's head and columns
           if (!wwait(ctl->p_free, ti & 1)) break;  // the last O MMAs are done
@@ -632,7 +689,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(dec::kThreads, 1)
           }
           tc_fence_before();
           __syncwarp();
-          if (lane == 0) mbar_arrive_remote(lead(ctl->o_free));
+          if (lane == 0) mbar_arrive_cl(lead(ctl->o_free));
         }
         c.advance(prefix);
       }

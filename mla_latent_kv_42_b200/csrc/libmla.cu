@@ -11,6 +11,7 @@
 #include <mutex>
 
 #include "common.cuh"
+#include "decode_mma.cuh"
 #include "decode_simt.cuh"
 #include "decode_tc.cuh"
 #include "prefill.cuh"
@@ -93,7 +94,32 @@ struct DecodePlan {
   int head_groups;
 };
 
+// The warp-MMA kernel for small head counts (decode_mma.cuh): up to 16 heads of a row of at most
+// 192 columns, latent at most 128, everything in 16-column steps.
+bool decode_mma_eligible(const mla_dims* d) {
+  const int D = d->d_c + d->d_rope;
+  return d->n_heads <= 16 && D % 16 == 0 && D <= 16 * dmma::kMaxKD && d->d_c % 16 == 0 &&
+         d->d_c <= 8 * dmma::kMaxND && d->page_size % 16 == 0;
+}
+
+// Split-KV plan of the warp-MMA kernel: about three CTAs per SM in one wave, each a whole number
+// of 64-token stages.
+DecodePlan plan_decode_mma(int B, int max_seq_len) {
+  DecodePlan p;
+  p.head_groups = 1;
+  const long ctas_wanted = 3L * device_sm_count();
+  long s = (ctas_wanted + B - 1) / B;
+  const long stages = ((long)max_seq_len + dmma::kStageTokens - 1) / dmma::kStageTokens;
+  if (s > stages) s = stages;
+  if (s < 1) s = 1;
+  const long per = (stages + s - 1) / s;  // stages per split
+  p.split_len = (int)(per * dmma::kStageTokens);
+  p.n_splits = (int)(((long)max_seq_len + p.split_len - 1) / p.split_len);
+  return p;
+}
+
 DecodePlan plan_decode(const mla_dims* d, int B, int max_seq_len) {
+  if (decode_mma_eligible(d)) return plan_decode_mma(B, max_seq_len);
   DecodePlan p;
   p.head_groups = (d->n_heads + 7) / 8;
   const long blocks_wanted = 4L * device_sm_count();
@@ -222,6 +248,7 @@ int decode_tc_impl(const mla_dims* d, const void* q, const void* pool, int32_t n
   if (!host::encode_2d(&maps.pool1, pool, bf16, tc::dec::kD, pool_rows, tc::dec::kD * 2, 64, 64) ||
       !host::encode_chunks(&maps.pool2, pool, bf16, pool_rows, tc::dec::kD * 2, 2) ||
       !host::encode_chunks(&maps.pool4, pool, bf16, pool_rows, tc::dec::kD * 2, 4) ||
+      !host::encode_chunks(&maps.pool9, pool, bf16, pool_rows, tc::dec::kD * 2, 9) ||
       !host::encode_chunks(&maps.q9, q, bf16, (uint64_t)B * d->n_heads, tc::dec::kD * 2, 9))
     return MLA_ERR_CUDA;
   if (launch_pdl(tc::k_decode_plan, dim3(1), dim3(1024), 0, st, seq_lens, bt, (int)B, (int)max_pages, (int)num_pages,
@@ -250,6 +277,21 @@ int decode_tc_impl(const mla_dims* d, const void* q, const void* pool, int32_t n
     return MLA_ERR_CUDA;
   launches += 3;
   return MLA_OK;
+}
+
+template <typename T>
+bool decode_mma_set_smem(size_t smem) {
+  static std::atomic<bool> done[kMaxDevices];
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return false;
+  if (!done[dev].load(std::memory_order_acquire)) {
+    // the largest row the kernel takes, so that one setting serves every eligible shape
+    if (cudaFuncSetAttribute(k_decode_mma<T>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             (int)dmma::smem_bytes(16 * dmma::kMaxKD)) != cudaSuccess)
+      return false;
+    done[dev].store(true, std::memory_order_release);
+  }
+  return smem <= dmma::smem_bytes(16 * dmma::kMaxKD);
 }
 
 template <typename T, int NPAIR>
@@ -284,19 +326,34 @@ int decode_impl(const mla_dims* d, const void* q, const void* pool, int32_t num_
   }
   const int D = d->d_c + d->d_rope;
   int32_t& n = launches;
-  if (D <= 192)
-    launch_decode_simt<T, 3>(d, p, q, pool, num_pages, bt, max_pages, seq_lens, B, max_seq_len, o_lat, lse_out,
-                             o_part, lse_part, st);
-  else if (D <= 384)
-    launch_decode_simt<T, 6>(d, p, q, pool, num_pages, bt, max_pages, seq_lens, B, max_seq_len, o_lat, lse_out,
-                             o_part, lse_part, st);
-  else
-    launch_decode_simt<T, 9>(d, p, q, pool, num_pages, bt, max_pages, seq_lens, B, max_seq_len, o_lat, lse_out,
-                             o_part, lse_part, st);
-  ++n;
+  if (decode_mma_eligible(d)) {
+    const float scale_log2 = (float)(1.0 / std::sqrt((double)(d->d_head + d->d_rope)) * 1.4426950408889634);
+    const size_t smem = dmma::smem_bytes(D);
+    if (!decode_mma_set_smem<T>(smem)) return MLA_ERR_CUDA;
+    mark_before(st);
+    const MmaAttnArgs a{q, pool, bt, (int)max_pages, seq_lens, (int)max_seq_len, (int)num_pages, (int)d->n_heads,
+                        (int)d->d_c, D, (int)d->page_size, scale_log2, p.split_len, p.n_splits, o_lat, lse_out,
+                        o_part, lse_part};
+    if (launch_pdl(k_decode_mma<T>, dim3(p.n_splits, B), dim3(128), smem, st, a) != cudaSuccess) return MLA_ERR_CUDA;
+    mark_after(st);
+    ++n;
+  } else {
+    if (D <= 192)
+      launch_decode_simt<T, 3>(d, p, q, pool, num_pages, bt, max_pages, seq_lens, B, max_seq_len, o_lat, lse_out,
+                               o_part, lse_part, st);
+    else if (D <= 384)
+      launch_decode_simt<T, 6>(d, p, q, pool, num_pages, bt, max_pages, seq_lens, B, max_seq_len, o_lat, lse_out,
+                               o_part, lse_part, st);
+    else
+      launch_decode_simt<T, 9>(d, p, q, pool, num_pages, bt, max_pages, seq_lens, B, max_seq_len, o_lat, lse_out,
+                               o_part, lse_part, st);
+    ++n;
+  }
   if (p.n_splits > 1) {
-    k_lse_merge<T><<<(unsigned)bh, 128, 0, st>>>(o_part, lse_part, p.n_splits, d->d_c, static_cast<T*>(o_lat),
-                                                 lse_out);
+    if (launch_pdl(k_lse_merge_warp<T>, dim3((unsigned)((bh + 7) / 8)), dim3(256), 0, st,
+                   static_cast<const float*>(o_part), static_cast<const float*>(lse_part), p.n_splits, (int)d->d_c,
+                   (long)bh, static_cast<T*>(o_lat), lse_out) != cudaSuccess)
+      return MLA_ERR_CUDA;
     ++n;
   }
   return cudaGetLastError() == cudaSuccess ? MLA_OK : MLA_ERR_CUDA;

@@ -132,6 +132,16 @@ __device__ __forceinline__ void st_cluster_u32(uint32_t caddr, uint32_t v) {
 // reads of it (bulk copies, tcgen05.mma operands).
 __device__ __forceinline__ void fence_proxy_async_cta() { asm volatile("fence.proxy.async.shared::cta;" ::: "memory"); }
 
+// Arrive on a barrier of either CTA of the pair given by its shared::cluster address, with the
+// instruction's default ordering (release at CTA scope: no cluster-wide fence on the way, which
+// a release.cluster arrive was measured to cost on every call).
+__device__ __forceinline__ void mbar_arrive_cl(uint32_t cluster_bar) {
+  asm volatile("mbarrier.arrive.shared::cluster.b64 _, [%0];" ::"r"(cluster_bar) : "memory");
+}
+__device__ __forceinline__ void mbar_arrive_expect_tx_cl(uint32_t cluster_bar, uint32_t bytes) {
+  asm volatile("mbarrier.arrive.expect_tx.shared::cluster.b64 _, [%0], %1;" ::"r"(cluster_bar), "r"(bytes)
+               : "memory");
+}
 // Arrive on a peer CTA's barrier and add `bytes` to the transaction count its current phase
 // waits for (releasing this thread's prior writes at cluster scope).
 __device__ __forceinline__ void mbar_arrive_expect_tx_remote(uint32_t cluster_bar, uint32_t bytes) {
@@ -244,6 +254,16 @@ __device__ __forceinline__ void mma2_ss(uint32_t d_tmem, uint64_t a_desc, uint64
       "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate)
       : "memory");
 }
+// Same with each descriptor given as its two 32-bit words (see desc_sw128_lo / desc_sw128_hi):
+// the issuing thread then steps an operand through K or through its buffers with one 32-bit add.
+__device__ __forceinline__ void mma2_ss_lohi(uint32_t d_tmem, uint32_t a_lo, uint32_t b_lo, uint32_t hi, uint32_t idesc,
+                                             uint32_t accumulate) {
+  asm volatile(
+      "{\n .reg .pred p;\n .reg .b64 da, db;\n setp.ne.b32 p, %5, 0;\n mov.b64 da, {%1, %3};\n"
+      " mov.b64 db, {%2, %3};\n tcgen05.mma.cta_group::2.kind::f16 [%0], da, db, %4, p;\n}\n" ::"r"(d_tmem),
+      "r"(a_lo), "r"(b_lo), "r"(hi), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
 // Arrive (once) on the barrier at offset `bar` in every CTA of `cta_mask` when all pair MMAs
 // this thread issued so far are complete.
 __device__ __forceinline__ void mma_commit2(uint32_t bar, uint16_t cta_mask) {
@@ -302,6 +322,17 @@ __device__ __forceinline__ void tmem_wait_st() { asm volatile("tcgen05.wait::st.
 __device__ __forceinline__ uint64_t desc_sw128(uint32_t saddr, uint32_t lbo, uint32_t sbo) {
   return (uint64_t)((saddr >> 4) & 0x3FFFu) | ((uint64_t)((lbo >> 4) & 0x3FFFu) << 16) |
          ((uint64_t)((sbo >> 4) & 0x3FFFu) << 32) | (1ull << 46) | (2ull << 61);
+}
+
+// The two words of desc_sw128: the low word holds the start address (bits 0-13, in 16-byte
+// units) and the leading byte offset, the high word the stride byte offset and the layout bits.
+// Shared-memory addresses stay below 2^18, so adding a 16-byte-unit offset to the low word never
+// carries into the leading-offset field.
+__device__ __forceinline__ uint32_t desc_sw128_lo(uint32_t saddr, uint32_t lbo) {
+  return ((saddr >> 4) & 0x3FFFu) | (((lbo >> 4) & 0x3FFFu) << 16);
+}
+__host__ __device__ constexpr uint32_t desc_sw128_hi(uint32_t sbo) {
+  return ((sbo >> 4) & 0x3FFFu) | (1u << 14) | (2u << 29);
 }
 
 // Instruction descriptor of tcgen05.mma kind::f16 with fp32 accumulation.

@@ -323,12 +323,22 @@ def test_layer_step_running_model_fp16():
     assert_parity(to64(u), naive["u"], "u")
 
 
-def test_layer_step_head_widths_off_the_gemm_blocks():
-    """Dims whose per-head slices are not whole 64-wide blocks (d_h = 40, d_c = 96): the two
-    per-head products take the CUDA-core kernels (k_absorb_uk for (W^UK_i)^T q^C_i, k_rowdot for
-    W^UV_i o_lat_i), the rest the tensor-core GEMM, attention the CUDA-core kernel with 16-token
-    pages; a whole layer step through the C ABI against the naive and absorbed oracle."""
-    d = synth.Dims(d_model=256, n_heads=4, d_head=40, d_c=96, d_cq=72, d_rope=16, page_size=16)
+ODD_DIMS = {
+    # 4 heads, 112-wide rows, 16-token pages: attention on the warp-MMA kernel
+    "h4_dh40_dc96": synth.Dims(d_model=256, n_heads=4, d_head=40, d_c=96, d_cq=72, d_rope=16, page_size=16),
+    # 32 heads, 80-wide rows, 8-token pages: attention on the CUDA-core kernel
+    "h32_dh24_dc72": synth.Dims(d_model=256, n_heads=32, d_head=24, d_c=72, d_cq=48, d_rope=8, page_size=8),
+}
+
+
+@pytest.mark.parametrize("name", list(ODD_DIMS))
+def test_layer_step_head_widths_off_the_gemm_blocks(name):
+    """Dims whose per-head slices are not whole 64-wide blocks (d_h = 40 or 24, d_c = 96 or 72): the
+    two per-head products take the CUDA-core kernels (k_absorb_uk for (W^UK_i)^T q^C_i, k_rowdot for
+    W^UV_i o_lat_i), the rest the tensor-core GEMM; attention runs on the warp-MMA kernel (4 heads)
+    or the CUDA-core kernel (32 heads, rows not a multiple of 16); a whole layer step through the
+    C ABI against the naive and absorbed oracle."""
+    d = ODD_DIMS[name]
     w = synth.Workload("odd_dims_b3", d, 3, 0, 1, 0.05, "shuffled")
     cached = np.array([0, 17, 300])
     L = harness.make_layer(w, cached)
