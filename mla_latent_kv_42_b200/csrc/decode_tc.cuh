@@ -57,7 +57,7 @@ constexpr int kAhead = 3;          // tiles between a page's L2 prefetch and its
 constexpr int kSoftWarps = 8;      // warps 0-7: softmax, rescale, epilogue
 constexpr int kLoadWarp = 8;       // Q, rope and own-page latent loads
 constexpr int kMmaWarp = 9;        // TMEM allocation; rank 0: MMA issue
-constexpr int kPairWarp = 10;      // the other page's latent half; tail tiles' row clearing
+constexpr int kPairWarp = 10;      // the other page's latent half
 constexpr int kThreads = 11 * 32;
 // TMEM columns
 constexpr uint32_t kOCol = 0;      // O: n-half j in columns [128j, 128j + 128)
@@ -78,7 +78,6 @@ struct Ctrl {
   uint64_t rope_done, q_free;
   uint64_t s_full[2], p_free;
   // Local barriers.
-  uint64_t fix_full[2][4];  // tail tiles: this CTA's own load of pair p
   uint64_t xm_full, xm_free;  // exchange of per-thread partial maxima / sums among the softmax warps
   uint64_t drain;
   float xm[2][128];          // [column half][TMEM lane]
@@ -102,12 +101,17 @@ struct DecodeTcParams {
   float* lse_part;        // [B + C][n_h]
 };
 
-// Tensor maps of the attention kernel: the paged pool viewed as [pages * 64 rows, 576] with one
-// 64 x 64 box (rope), and as (64 columns, rows, 9 column chunks) with boxes of 2, 4 and 9 chunks
-// (the last for L2 prefetches of whole pages); the queries viewed as (64 columns, B * n_h rows,
-// 9 chunks) with a box of 9 chunks.
+// Tensor maps of the attention kernel: the paged pool viewed as (64 columns, 64 rows of a page,
+// pages, 9 column chunks) with boxes of 1, 2 and 4 chunks of one page, and as (64 columns, rows,
+// 9 chunks) with a box of a whole page (L2 prefetches); the queries viewed as (64 columns,
+// B * n_h rows, 9 chunks) with a box of 9 chunks.
+//
+// A page that holds nv < 64 tokens of its sequence (the last one) is loaded from row nv - 64:
+// its tokens land in slot rows [64 - nv, 64) and the rows before are the tensor map's zero fill,
+// so whatever the pool holds past the end of a sequence never reaches shared memory, and a page
+// wholly past the end (nv = 0) loads as zeros. Softmax masks slot rows r < 64 - nv.
 struct DecodeTcMaps {
-  CUtensorMap pool1, pool2, pool4, pool9, q9;
+  CUtensorMap page1, page2, page4, pool9, q9;
 };
 
 // Tiles [t0, t1) of sequence b handled by this pair (n_b = tiles of the sequence).
@@ -197,6 +201,17 @@ __device__ __forceinline__ void tma_load_3d_pair(uint32_t dst, const CUtensorMap
       : "memory");
 }
 
+// Box of page `page` of a paged map, rows from `row0` (negative: zero fill before the page's
+// first row), chunks from `chunk`.
+__device__ __forceinline__ void tma_load_page_pair(uint32_t dst, const CUtensorMap* map, uint32_t cluster_bar, int row0,
+                                                   int page, int chunk) {
+  asm volatile(
+      "cp.async.bulk.tensor.4d.cta_group::2.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%3, %4, "
+      "%5, %6}], [%2];" ::"r"(dst),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(cluster_bar), "r"(0), "r"(row0), "r"(page), "r"(chunk)
+      : "memory");
+}
+
 template <typename T>
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(dec::kThreads, 1)
     k_decode_tc(const __grid_constant__ DecodeTcMaps maps, const DecodeTcParams p) {
@@ -219,7 +234,6 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(dec::kThreads, 1)
       for (int q = 0; q < 4; ++q) {
         mbar_init(bar(ctl->pv_full[s][q]), 2);
         mbar_init(bar(ctl->qk_done[s][q]), 1);
-        mbar_init(bar(ctl->fix_full[s][q]), 1);
       }
       mbar_init(bar(ctl->s_free[s]), 2 * kSoftWarps);
       mbar_init(bar(ctl->set_free[s][0]), 1);
@@ -276,9 +290,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(dec::kThreads, 1)
     if (warp == kLoadWarp) {
       // ---------------------------------------------------------------- Q, rope and own-page loads
       if (lane == 0) {
-        tma_prefetch_map(&maps.pool1);
-        tma_prefetch_map(&maps.pool2);
-        tma_prefetch_map(&maps.pool4);
+        tma_prefetch_map(&maps.page1);
+        tma_prefetch_map(&maps.page2);
+        tma_prefetch_map(&maps.page4);
         tma_prefetch_map(&maps.pool9);
         tma_prefetch_map(&maps.q9);
         Cursor c;
@@ -303,20 +317,16 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(dec::kThreads, 1)
           if (c.first()) L = p.seq_lens[b];
           const int* btb = p.bt + (long)b * p.max_pages;
           const int page_idx = 2 * t + (int)rank;
-          const bool own = kPage * page_idx < L;  // page r of the tile holds tokens
-          const int page = own ? btb[page_idx] : 0;
+          const int nv = min(kPage, max(0, L - kPage * page_idx));  // tokens in page r of the tile
+          const int page = nv > 0 ? btb[page_idx] : 0;
           if (c.first()) {  // this CTA's 64 heads of the sequence's queries, after the last S MMA of the item before
             if (!wait(ctl->q_free, (c.ii & 1) ^ 1)) break;
             mbar_arrive_expect_tx_cl(lead(ctl->q_full), 9 * kChunk);
             tma_load_3d_pair(data_u32 + kQOff, &maps.q9, lead(ctl->q_full), 0, b * p.n_h + 64 * (int)rank, 0);
           }
           if (!wait(ctl->rope_done, (c.ti & 1) ^ 1)) break;
-          if (own) {
-            mbar_arrive_expect_tx_cl(lead(ctl->rope_full), kChunk);
-            tma_load_2d_pair(data_u32 + kRopeOff, &maps.pool1, lead(ctl->rope_full), kDc, page * kPage);
-          } else {
-            mbar_arrive_cl(lead(ctl->rope_full));
-          }
+          mbar_arrive_expect_tx_cl(lead(ctl->rope_full), kChunk);
+          tma_load_page_pair(data_u32 + kRopeOff, &maps.page1, lead(ctl->rope_full), nv - kPage, page, 8);
           bool ok = true;
           for (int h = 0; h < 2; ++h) {
             // the O MMAs of tile ti - 2 are done with chunks [4h, 4h + 4) of set s
@@ -325,18 +335,14 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(dec::kThreads, 1)
               break;
             }
 #ifdef MLA_FAULT_INJECT
-            if (own && h == 0 && rank == 0 && prefix[b] + t == g_inject_missing_tile) {
+            if (h == 0 && rank == 0 && prefix[b] + t == g_inject_missing_tile) {
               mbar_arrive_expect_tx_cl(lead(ctl->qk_full[s][h]), 4 * kChunk);
               continue;
             }
 #endif
-            if (own) {
-              mbar_arrive_expect_tx_cl(lead(ctl->qk_full[s][h]), 4 * kChunk);
-              tma_load_3d_pair(set_u32 + s * kSetBytes + 4 * h * kChunk, &maps.pool4, lead(ctl->qk_full[s][h]), 0,
-                               page * kPage, 4 * h);
-            } else {
-              mbar_arrive_cl(lead(ctl->qk_full[s][h]));
-            }
+            mbar_arrive_expect_tx_cl(lead(ctl->qk_full[s][h]), 4 * kChunk);
+            tma_load_page_pair(set_u32 + s * kSetBytes + 4 * h * kChunk, &maps.page4, lead(ctl->qk_full[s][h]),
+                               nv - kPage, page, 4 * h);
           }
           if (!ok) break;
           if (ahead.valid) prefetch_ahead();
@@ -347,81 +353,39 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(dec::kThreads, 1)
     } else if (warp == kPairWarp) {
       // ---------------------------------------------------------------- the other page's latent half
       // Pair p = 2j + g of set s holds, for O, the columns this CTA supplies for n-half j of page
-      // g. Page g = r is already there (loaded for S); page 1 - r is loaded once S is done with
-      // the own page's columns in those slots. In a tail tile (the sequence ends inside it) rows
-      // past the end may hold anything (even NaN): this warp zeroes them in both pages, loading
-      // the other page's half to a local barrier first.
-      Cursor c;
-      c.start(prefix, p.B, cluster, nclusters);
-      uint32_t fix_par = 0;
-      bool ok = true;
-      int L = 0;
-      while (ok && c.valid) {
-        const int s = c.ti & 1, b = c.item.b, t = c.t;
-        if (c.first()) L = p.seq_lens[b];
-        const uint32_t ph = (c.ti >> 1) & 1;
-        const int* btb = p.bt + (long)b * p.max_pages;
-        const int g_other = 1 - (int)rank;
-        const bool whole_tile = kTile * (t + 1) <= L;
-        const int page_other = whole_tile ? btb[2 * t + g_other] : 0;  // read ahead of the wait below
-        // the O MMAs of tile ti - 2 are complete, so every barrier of set s is in this tile's phase
-        if (!wwait(ctl->set_free[s][1], ph ^ 1)) break;
-        if (whole_tile) {
-          if (lane == 0) {
-            mbar_arrive_cl(lead(ctl->pv_full[s][(int)rank]));      // j = 0, g = r
-            mbar_arrive_cl(lead(ctl->pv_full[s][2 + (int)rank]));  // j = 1, g = r
-          }
-          const int g = g_other;
-          const int page = page_other;
+      // g. Page g = r is already there (loaded for S); page 1 - r is loaded once the S MMAs are
+      // done with the own page's columns in those slots (a tail page with its zero-filled rows).
+      if (lane == 0) {
+        Cursor c;
+        c.start(prefix, p.B, cluster, nclusters);
+        int L = 0;
+        const int g = 1 - (int)rank;
+        while (c.valid) {
+          const int s = c.ti & 1, b = c.item.b, t = c.t;
+          if (c.first()) L = p.seq_lens[b];
+          const uint32_t ph = (c.ti >> 1) & 1;
+          const int nv = min(kPage, max(0, L - kTile * t - kPage * g));  // tokens in page g of the tile
+          const int page = nv > 0 ? p.bt[(long)b * p.max_pages + 2 * t + g] : 0;  // read ahead of the waits
+          // the O MMAs of tile ti - 2 are complete, so every barrier of set s is in this tile's phase
+          if (!wait(ctl->set_free[s][1], ph ^ 1)) break;
+          mbar_arrive_cl(lead(ctl->pv_full[s][(int)rank]));      // j = 0, g = r
+          mbar_arrive_cl(lead(ctl->pv_full[s][2 + (int)rank]));  // j = 1, g = r
+          bool ok = true;
           for (int j = 0; j < 2; ++j) {
             const int pr = 2 * j + g;
-            if (!wwait(ctl->qk_done[s][pr], ph)) {
+            if (!wait(ctl->qk_done[s][pr], ph)) {
               ok = false;
               break;
             }
-            if (lane == 0) {
-              mbar_arrive_expect_tx_cl(lead(ctl->pv_full[s][pr]), 2 * kChunk);
-              tma_load_3d_pair(set_u32 + s * kSetBytes + 2 * pr * kChunk, &maps.pool2, lead(ctl->pv_full[s][pr]), 0,
-                               page * kPage, 4 * j + 2 * (int)rank);
-            }
+            mbar_arrive_expect_tx_cl(lead(ctl->pv_full[s][pr]), 2 * kChunk);
+            tma_load_page_pair(set_u32 + s * kSetBytes + 2 * pr * kChunk, &maps.page2, lead(ctl->pv_full[s][pr]),
+                               nv - kPage, page, 4 * j + 2 * (int)rank);
           }
-        } else {  // tail tile
-          for (int g = 0; ok && g < 2; ++g)
-            for (int j = 0; j < 2; ++j) {
-              const int pr = 2 * j + g;
-              if (!wwait(ctl->qk_done[s][pr], ph)) {
-                ok = false;
-                break;
-              }
-              const int nv = max(0, min(kPage, L - kTile * t - kPage * g));  // valid rows of page g
-              const uint32_t slot = set_u32 + s * kSetBytes + 2 * pr * kChunk;
-              if (g != (int)rank && nv > 0) {
-                const int fb = s * 4 + pr;
-                if (lane == 0) {
-                  mbar_arrive_expect_tx(bar(ctl->fix_full[s][pr]), 2 * kChunk);
-                  tma_load_3d(slot, &maps.pool2, bar(ctl->fix_full[s][pr]), 0, btb[2 * t + g] * kPage,
-                              4 * j + 2 * (int)rank);
-                }
-                if (!wwait(ctl->fix_full[s][pr], (fix_par >> fb) & 1u)) {
-                  ok = false;
-                  break;
-                }
-                fix_par ^= 1u << fb;
-              }
-              uint8_t* sp = data + (slot - data_u32);
-              const int per = (kPage - nv) * 8;  // 16-byte units to clear per chunk
-              for (int e = lane; e < 2 * per; e += 32) {
-                const int ch = e / per, rem = e - ch * per;
-                *reinterpret_cast<uint4*>(sp + ch * kChunk + (nv + (rem >> 3)) * 128 + (rem & 7) * 16) =
-                    make_uint4(0, 0, 0, 0);
-              }
-              fence_proxy_async_cta();
-              __syncwarp();
-              if (lane == 0) mbar_arrive_cl(lead(ctl->pv_full[s][pr]));
-            }
+          if (!ok) break;
+          c.advance(prefix);
         }
-        c.advance(prefix);
       }
+      __syncwarp();
     } else if (warp == kMmaWarp) {
       // ---------------------------------------------------------------- MMA issue (rank 0, one lane)
       // Tiles in order, each as its S step followed by the O step of the tile before it: S(i),
@@ -569,12 +533,12 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(dec::kThreads, 1)
         tc_fence_before();
         __syncwarp();
         if (lane == 0) mbar_arrive_cl(lead(ctl->s_free[sb]));
-        // tokens past the sequence end become -inf (weight exactly 0), whatever the slot held
-        const int nv = max(0, min(32, L - (kTile * t + kPage * g + 32 * ch)));
-        if (nv < 32) {
+        // Slot rows before 64 - nv of a tail page (nv tokens) are zero fill: -inf, weight exactly 0.
+        const int lo = kPage - min(kPage, max(0, L - kTile * t - kPage * g)) - 32 * ch;  // first valid k
+        if (lo > 0) {
 #pragma unroll
           for (int k = 0; k < 32; ++k)
-            if (k >= nv) sr[k] = __float_as_uint(-INFINITY);
+            if (k < lo) sr[k] = __float_as_uint(-INFINITY);
         }
         float mxs[8];
 #pragma unroll
@@ -647,36 +611,62 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(dec::kThreads, 1)
           const bool whole = it.t0 == 0 && it.t1 == it.n_b;
           const long slot = (long)it.b + cluster;
           const int col0 = 256 * ch + 128 * g;  // latent columns [col0, col0 + 128)
+          // The warp writes its 32 heads x 128 columns in rounds of 64 bytes per head through its
+          // own 2 KB of the P buffer (free: the last O MMAs are done). Each lane puts its head's
+          // segment in row `lane` (16-byte chunks swizzled by row, conflict-free both ways), and
+          // each store instruction then writes 8 heads x 64 contiguous bytes.
+          uint8_t* const stage = data + kPOff + warp * 2048;
+          const uint32_t wsw = (lane >> 1) & 3;
+          const int rq = lane >> 2, cq = lane & 3;
+          auto stage_put = [&](const uint32_t (&w)[16]) {
+#pragma unroll
+            for (int i2 = 0; i2 < 4; ++i2)
+              *reinterpret_cast<uint4*>(stage + lane * 64 + ((i2 ^ wsw) << 4)) =
+                  make_uint4(w[4 * i2], w[4 * i2 + 1], w[4 * i2 + 2], w[4 * i2 + 3]);
+            __syncwarp();
+          };
+          // row 8k + rq of the round: its head and its chunk cq
+          auto stage_get = [&](int k, int& hd) {
+            const int row = 8 * k + rq;
+            hd = 64 * (int)rank + ((32 * qd + row) & 63);
+            return *reinterpret_cast<const uint4*>(stage + row * 64 + ((cq ^ ((row >> 1) & 3)) << 4));
+          };
 #pragma unroll 1
-          for (int c0 = 0; c0 < 128; c0 += 64) {  // two TMEM loads in flight per wait
-            uint32_t r[2][32];
-#pragma unroll
-            for (int q2 = 0; q2 < 2; ++q2) tmem_ld32(tmem + lane_base + kOCol + 128 * ch + c0 + 32 * q2, r[q2]);
+          for (int c0 = 0; c0 < 128; c0 += 32) {
+            uint32_t r[32];
+            tmem_ld32(tmem + lane_base + kOCol + 128 * ch + c0, r);
             tmem_wait_ld();
-            if (head < p.n_h) {
-              if (whole) {
-                uint4* dst = reinterpret_cast<uint4*>(static_cast<T*>(p.o_lat) + ((long)it.b * p.n_h + head) * kDc +
-                                                      col0 + c0);
+            if (whole) {  // 32 columns of bf16 / fp16 per round
+              uint32_t w[16];
 #pragma unroll
-                for (int q = 0; q < 8; ++q) {
-                  uint32_t w[4];
+              for (int e = 0; e < 16; ++e) {
+                const typename Pack<T>::T2 v = Pack<T>::make(u2f(r[2 * e]) * inv, u2f(r[2 * e + 1]) * inv);
+                w[e] = *reinterpret_cast<const uint32_t*>(&v);
+              }
+              stage_put(w);
+              T* const ob = static_cast<T*>(p.o_lat) + (long)it.b * p.n_h * kDc + col0 + c0 + 8 * cq;
 #pragma unroll
-                  for (int e = 0; e < 4; ++e) {
-                    const int k = 8 * q + 2 * e;
-                    const typename Pack<T>::T2 v =
-                        Pack<T>::make(u2f(r[k >> 5][k & 31]) * inv, u2f(r[(k + 1) >> 5][(k + 1) & 31]) * inv);
-                    w[e] = *reinterpret_cast<const uint32_t*>(&v);
-                  }
-                  dst[q] = make_uint4(w[0], w[1], w[2], w[3]);
+              for (int k = 0; k < 4; ++k) {
+                int hd;
+                const uint4 v = stage_get(k, hd);
+                if (hd < p.n_h) *reinterpret_cast<uint4*>(ob + (long)hd * kDc) = v;
+              }
+              __syncwarp();
+            } else {  // 16 columns of fp32 per round
+#pragma unroll
+              for (int half = 0; half < 2; ++half) {
+                uint32_t w[16];
+#pragma unroll
+                for (int e = 0; e < 16; ++e) w[e] = __float_as_uint(u2f(r[16 * half + e]) * inv);
+                stage_put(w);
+                float* const ob = p.o_part + slot * p.n_h * kDc + col0 + c0 + 16 * half + 4 * cq;
+#pragma unroll
+                for (int k = 0; k < 4; ++k) {
+                  int hd;
+                  const uint4 v = stage_get(k, hd);
+                  if (hd < p.n_h) *reinterpret_cast<uint4*>(ob + (long)hd * kDc) = v;
                 }
-              } else {
-                float4* dst = reinterpret_cast<float4*>(p.o_part + (slot * p.n_h + head) * kDc + col0 + c0);
-#pragma unroll
-                for (int q = 0; q < 16; ++q) {
-                  const int k = 4 * q;
-                  dst[q] = make_float4(u2f(r[k >> 5][k & 31]) * inv, u2f(r[k >> 5][(k & 31) + 1]) * inv,
-                                       u2f(r[k >> 5][(k & 31) + 2]) * inv, u2f(r[k >> 5][(k & 31) + 3]) * inv);
-                }
+                __syncwarp();
               }
             }
           }

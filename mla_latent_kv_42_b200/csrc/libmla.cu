@@ -245,9 +245,9 @@ int decode_tc_impl(const mla_dims* d, const void* q, const void* pool, int32_t n
   constexpr bool bf16 = tc::IsBf16<T>::value;
   const uint64_t pool_rows = (uint64_t)num_pages * tc::dec::kPage;
   tc::DecodeTcMaps maps;
-  if (!host::encode_2d(&maps.pool1, pool, bf16, tc::dec::kD, pool_rows, tc::dec::kD * 2, 64, 64) ||
-      !host::encode_chunks(&maps.pool2, pool, bf16, pool_rows, tc::dec::kD * 2, 2) ||
-      !host::encode_chunks(&maps.pool4, pool, bf16, pool_rows, tc::dec::kD * 2, 4) ||
+  if (!host::encode_pages(&maps.page1, pool, bf16, (uint64_t)num_pages, tc::dec::kD * 2, 1) ||
+      !host::encode_pages(&maps.page2, pool, bf16, (uint64_t)num_pages, tc::dec::kD * 2, 2) ||
+      !host::encode_pages(&maps.page4, pool, bf16, (uint64_t)num_pages, tc::dec::kD * 2, 4) ||
       !host::encode_chunks(&maps.pool9, pool, bf16, pool_rows, tc::dec::kD * 2, 9) ||
       !host::encode_chunks(&maps.q9, q, bf16, (uint64_t)B * d->n_heads, tc::dec::kD * 2, 9))
     return MLA_ERR_CUDA;

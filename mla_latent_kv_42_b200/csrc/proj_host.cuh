@@ -94,6 +94,23 @@ inline bool encode_chunks(CUtensorMap* map, const void* base, bool bf16, uint64_
             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+// 4-D view of a paged cache [pages][64 rows][9 * 64] of 16-bit elements, rows `row_bytes` apart, as
+// (64 columns, 64 rows of a page, pages, 9 column chunks) with boxes of (64, 64, 1, depth). A box
+// started at row nv - 64 (nv = rows of the page that hold tokens) lands with the page's rows
+// [0, nv) in the box's last nv rows and zeros (the fill outside the tensor) in the rows before.
+inline bool encode_pages(CUtensorMap* map, const void* base, bool bf16, uint64_t pages, uint64_t row_bytes,
+                         uint32_t depth) {
+  auto fn = tensor_map_encoder();
+  if (fn == nullptr) return false;
+  cuuint64_t dims[4] = {64, 64, pages, 9};
+  cuuint64_t strides[3] = {row_bytes, 64 * row_bytes, 128};
+  cuuint32_t box[4] = {64, 64, 1, depth};
+  cuuint32_t es[4] = {1, 1, 1, 1};
+  return fn(map, bf16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 4, const_cast<void*>(base),
+            dims, strides, box, es, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+            CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 // ------------------------------------------------------------------ GEMM planning
 // One stream-K GEMM launch (see gemm_sk.cuh): tile sizes, CTA count, ring depth, and whether
 // any tile is shared by several CTAs (then fp32 partials and a reduction launch are needed).
