@@ -53,7 +53,6 @@ constexpr int kSetOff = kRopeOff + kChunk;    // two sets of 8 latent chunks
 constexpr int kSetBytes = 8 * kChunk;
 constexpr int kDataBytes = kSetOff + 2 * kSetBytes;  // 229376
 constexpr float kLazy = 8.f;       // rescale threshold in log2 units
-constexpr int kAhead = 3;          // tiles between a page's L2 prefetch and its shared-memory load
 constexpr int kSoftWarps = 8;      // warps 0-7: softmax, rescale, epilogue
 constexpr int kLoadWarp = 8;       // Q, rope and own-page latent loads
 constexpr int kMmaWarp = 9;        // TMEM allocation; rank 0: MMA issue
@@ -102,16 +101,16 @@ struct DecodeTcParams {
 };
 
 // Tensor maps of the attention kernel: the paged pool viewed as (64 columns, 64 rows of a page,
-// pages, 9 column chunks) with boxes of 1, 2 and 4 chunks of one page, and as (64 columns, rows,
-// 9 chunks) with a box of a whole page (L2 prefetches); the queries viewed as (64 columns,
-// B * n_h rows, 9 chunks) with a box of 9 chunks.
+// pages, 9 column chunks) with boxes of 1, 2 and 4 chunks of one page; the queries viewed as
+// (64 columns, B * n_h rows, 9 chunks) with a box of 9 chunks. (Prefetching pages into L2 ahead
+// of their loads was measured slower: the prefetches take the same per-SM copy engine.)
 //
 // A page that holds nv < 64 tokens of its sequence (the last one) is loaded from row nv - 64:
 // its tokens land in slot rows [64 - nv, 64) and the rows before are the tensor map's zero fill,
 // so whatever the pool holds past the end of a sequence never reaches shared memory, and a page
 // wholly past the end (nv = 0) loads as zeros. Softmax masks slot rows r < 64 - nv.
 struct DecodeTcMaps {
-  CUtensorMap page1, page2, page4, pool9, q9;
+  CUtensorMap page1, page2, page4, q9;
 };
 
 // Tiles [t0, t1) of sequence b handled by this pair (n_b = tiles of the sequence).
@@ -184,13 +183,6 @@ __device__ __forceinline__ void tma_load_3d(uint32_t dst, const CUtensorMap* map
           dst),
       "l"(reinterpret_cast<uint64_t>(map)), "r"(bar), "r"(x), "r"(y), "r"(z)
       : "memory");
-}
-// Prefetch a 3-D box into L2 (no shared memory, no barrier).
-__device__ __forceinline__ void tma_prefetch_3d(const CUtensorMap* map, int x, int y, int z) {
-  asm volatile("cp.async.bulk.prefetch.tensor.3d.L2.global.tile [%0, {%1, %2, %3}];" ::"l"(
-                   reinterpret_cast<uint64_t>(map)),
-               "r"(x), "r"(y), "r"(z)
-               : "memory");
 }
 __device__ __forceinline__ void tma_load_3d_pair(uint32_t dst, const CUtensorMap* map, uint32_t cluster_bar, int x,
                                                  int y, int z) {
@@ -293,24 +285,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(dec::kThreads, 1)
         tma_prefetch_map(&maps.page1);
         tma_prefetch_map(&maps.page2);
         tma_prefetch_map(&maps.page4);
-        tma_prefetch_map(&maps.pool9);
         tma_prefetch_map(&maps.q9);
         Cursor c;
         c.start(prefix, p.B, cluster, nclusters);
         int L = 0;
-        // A second cursor runs kAhead tiles ahead and prefetches its own page into L2, so that the
-        // shared-memory loads of that tile, issued once its set is free, read from L2.
-        Cursor ahead;
-        ahead.start(prefix, p.B, cluster, nclusters);
-        int L_ahead = ahead.valid ? p.seq_lens[ahead.item.b] : 0;
-        auto prefetch_ahead = [&]() {
-          const int pi = 2 * ahead.t + (int)rank;
-          if (kPage * pi < L_ahead) tma_prefetch_3d(&maps.pool9, 0, p.bt[(long)ahead.item.b * p.max_pages + pi] * kPage, 0);
-          const int ii = ahead.ii;
-          ahead.advance(prefix);
-          if (ahead.valid && ahead.ii != ii) L_ahead = p.seq_lens[ahead.item.b];
-        };
-        for (int k = 0; k < kAhead && ahead.valid; ++k) prefetch_ahead();
         while (c.valid) {
           const int s = c.ti & 1, b = c.item.b, t = c.t;
           // global reads first: their latency overlaps the waits below
@@ -345,7 +323,6 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(dec::kThreads, 1)
                                nv - kPage, page, 4 * h);
           }
           if (!ok) break;
-          if (ahead.valid) prefetch_ahead();
           c.advance(prefix);
         }
       }
@@ -388,9 +365,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(dec::kThreads, 1)
       __syncwarp();
     } else if (warp == kMmaWarp) {
       // ---------------------------------------------------------------- MMA issue (rank 0, one lane)
-      // Tiles in order, each as its S step followed by the O step of the tile before it: S(i),
-      // O(i - 1), S(i + 1), O(i), ... The softmax of tile i - 1 runs while S(i) executes, and the
-      // set of tile i - 1 is released as soon as O(i - 1) completes. One thread issues all MMAs
+      // Tiles in order, the O step of the tile before each between its two S groups: S(i) rope
+      // and chunks 0-3, O(i - 1), S(i) chunks 4-7, S(i + 1) rope and chunks 0-3, O(i), ... The
+      // softmax of tile i - 1 runs while S(i) executes, O(i - 1) releases its set (and P) before
+      // S(i) ends, and the second box of tile i has time to land behind it. One thread issues all MMAs
       // of the pair, and a single thread runs dependent instructions and branches at a few cycles
       // each, so the issue path is straight-line code: per step a fixed sequence of waits, MMAs
       // with compile-time operand offsets, and commits. Each descriptor is a fixed high word and
@@ -414,34 +392,37 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(dec::kThreads, 1)
           st_cluster_u32(peer_abort, 1u);
           return false;
         };
-        // S(ti) = Q C^T into S buffer ti & 1: the rope chunk, then latent chunks 0-7.
-        auto s_step = [&](int ti, bool first, bool last, int ii) {
+        // S(ti) = Q C^T into S buffer ti & 1 in two groups: the rope chunk and latent chunks 0-3
+        // (the first box), then chunks 4-7 (the second).
+        auto s_group = [&](int ti, int grp, bool first, bool last, int ii) {
           const int s = ti & 1;
           const uint32_t ph = (ti >> 1) & 1;
-          if (!mwait(b_s_free + 8 * s, ph ^ 1)) return false;  // softmax has read S(ti - 2)
-          if (first && !mwait(bar(ctl->q_full), ii & 1)) return false;
-          if (!mwait(bar(ctl->rope_full), ti & 1)) return false;
-          tc_fence_after();
           const uint32_t d = tmem + kSCol + 64 * s;
-#pragma unroll
-          for (int ks = 0; ks < 4; ++ks)
-            mma2_ss_lohi(d, q_lo + 8 * kChunkD + 2 * ks, rope_lo + 2 * ks, hi, idesc_qk, ks != 0);
-          mma_commit2(bar(ctl->rope_done), 3);
           const uint32_t kb = k_lo + s * kSetD;
-#pragma unroll
-          for (int hh = 0; hh < 2; ++hh) {
-            if (!mwait(b_qk_full + 8 * (2 * s + hh), ph)) return false;
+          if (grp == 0) {
+            if (!mwait(b_s_free + 8 * s, ph ^ 1)) return false;  // softmax has read S(ti - 2)
+            if (first && !mwait(bar(ctl->q_full), ii & 1)) return false;
+            if (!mwait(bar(ctl->rope_full), ti & 1)) return false;
             tc_fence_after();
 #pragma unroll
-            for (int kc = 4 * hh; kc < 4 * hh + 4; ++kc) {
-#pragma unroll
-              for (int ks = 0; ks < 4; ++ks)
-                mma2_ss_lohi(d, q_lo + kc * kChunkD + 2 * ks, kb + kc * kChunkD + 2 * ks, hi, idesc_qk, 1);
-              if (kc & 1) mma_commit2(b_qk_done + 8 * (4 * s + (kc >> 1)), 3);
-            }
+            for (int ks = 0; ks < 4; ++ks)
+              mma2_ss_lohi(d, q_lo + 8 * kChunkD + 2 * ks, rope_lo + 2 * ks, hi, idesc_qk, ks != 0);
+            mma_commit2(bar(ctl->rope_done), 3);
           }
-          mma_commit2(b_s_full + 8 * s, 3);
-          if (last) mma_commit2(bar(ctl->q_free), 3);
+          if (!mwait(b_qk_full + 8 * (2 * s + grp), ph)) return false;
+          tc_fence_after();
+#pragma unroll
+          for (int k4 = 0; k4 < 4; ++k4) {
+            const int kc = 4 * grp + k4;
+#pragma unroll
+            for (int ks = 0; ks < 4; ++ks)
+              mma2_ss_lohi(d, q_lo + kc * kChunkD + 2 * ks, kb + kc * kChunkD + 2 * ks, hi, idesc_qk, 1);
+            if (k4 & 1) mma_commit2(b_qk_done + 8 * (4 * s + (kc >> 1)), 3);
+          }
+          if (grp == 1) {
+            mma_commit2(b_s_full + 8 * s, 3);
+            if (last) mma_commit2(bar(ctl->q_free), 3);
+          }
           return true;
         };
         // O += P C_lat for tile ti: pairs (g, j) = (0,0), (1,0), (0,1), (1,1); chunks 0-3 of the
@@ -473,8 +454,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(dec::kThreads, 1)
         int prev_ti = -1, prev_ii = 0;
         bool prev_first = false;
         while (c.valid) {
-          if (!s_step(c.ti, c.first(), c.last(), c.ii)) break;
+          if (!s_group(c.ti, 0, c.first(), c.last(), c.ii)) break;
           if (prev_ti >= 0 && !o_step(prev_ti, prev_first, prev_ii)) break;
+          if (!s_group(c.ti, 1, c.first(), c.last(), c.ii)) break;
           prev_ti = c.ti;
           prev_first = c.first();
           prev_ii = c.ii;

@@ -243,12 +243,10 @@ int decode_tc_impl(const mla_dims* d, const void* q, const void* pool, int32_t n
   float* o_part = c.take<float>(((size_t)B + C) * d->n_heads * tc::dec::kDc);
   float* lse_part = c.take<float>(((size_t)B + C) * d->n_heads);
   constexpr bool bf16 = tc::IsBf16<T>::value;
-  const uint64_t pool_rows = (uint64_t)num_pages * tc::dec::kPage;
   tc::DecodeTcMaps maps;
   if (!host::encode_pages(&maps.page1, pool, bf16, (uint64_t)num_pages, tc::dec::kD * 2, 1) ||
       !host::encode_pages(&maps.page2, pool, bf16, (uint64_t)num_pages, tc::dec::kD * 2, 2) ||
       !host::encode_pages(&maps.page4, pool, bf16, (uint64_t)num_pages, tc::dec::kD * 2, 4) ||
-      !host::encode_chunks(&maps.pool9, pool, bf16, pool_rows, tc::dec::kD * 2, 9) ||
       !host::encode_chunks(&maps.q9, q, bf16, (uint64_t)B * d->n_heads, tc::dec::kD * 2, 9))
     return MLA_ERR_CUDA;
   if (launch_pdl(tc::k_decode_plan, dim3(1), dim3(1024), 0, st, seq_lens, bt, (int)B, (int)max_pages, (int)num_pages,
