@@ -55,9 +55,10 @@ constexpr int kDataBytes = kSetOff + 2 * kSetBytes;  // 229376
 constexpr float kLazy = 8.f;       // rescale threshold in log2 units
 constexpr int kSoftWarps = 8;      // warps 0-7: softmax, rescale, epilogue
 constexpr int kLoadWarp = 8;       // Q, rope and own-page latent loads
-constexpr int kMmaWarp = 9;        // TMEM allocation; rank 0: MMA issue
+constexpr int kMmaWarp = 9;        // TMEM allocation; rank 0: S MMA issue
 constexpr int kPairWarp = 10;      // the other page's latent half
-constexpr int kThreads = 11 * 32;
+constexpr int kOWarp = 11;        // rank 0: O MMA issue
+constexpr int kThreads = 12 * 32;
 // TMEM columns
 constexpr uint32_t kOCol = 0;      // O: n-half j in columns [128j, 128j + 128)
 constexpr uint32_t kSCol = 256;    // S buffer b in columns [256 + 64b, 320 + 64b)
@@ -241,7 +242,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(dec::kThreads, 1)
     mbar_init(bar(ctl->p_free), 1);
     mbar_init(bar(ctl->xm_full), kSoftWarps);
     mbar_init(bar(ctl->xm_free), kSoftWarps);
-    mbar_init(bar(ctl->drain), 1);
+    mbar_init(bar(ctl->drain), 2);
     ctl->abort_flag = 0;
     fence_mbar_init();
   }
@@ -363,106 +364,106 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(dec::kThreads, 1)
         }
       }
       __syncwarp();
-    } else if (warp == kMmaWarp) {
-      // ---------------------------------------------------------------- MMA issue (rank 0, one lane)
-      // Tiles in order, the O step of the tile before each between its two S groups: S(i) rope
-      // and chunks 0-3, O(i - 1), S(i) chunks 4-7, S(i + 1) rope and chunks 0-3, O(i), ... The
-      // softmax of tile i - 1 runs while S(i) executes, O(i - 1) releases its set (and P) before
-      // S(i) ends, and the second box of tile i has time to land behind it. One thread issues all MMAs
-      // of the pair, and a single thread runs dependent instructions and branches at a few cycles
-      // each, so the issue path is straight-line code: per step a fixed sequence of waits, MMAs
-      // with compile-time operand offsets, and commits. Each descriptor is a fixed high word and
-      // a low word stepped by 32-bit adds (16-byte units: a K-step of 16 elements is +2 along a
-      // K-major row and +128, i.e. 16 rows, down an MN-major operand).
+    } else if (warp == kMmaWarp || warp == kOWarp) {
+      // ---------------------------------------------------------------- MMA issue (rank 0)
+      // Two issuing threads, one per stream of MMAs: warp kMmaWarp issues S(i) for the tiles in
+      // order (the rope chunk and latent chunks 0-3 once the first box lands, chunks 4-7 once the
+      // second does), warp kOWarp issues O(i) once P(i) is written and each pair's chunks are in
+      // place. The two streams touch disjoint tensor memory (S buffers, O) and are ordered through
+      // the softmax barriers, so neither waits behind the other's inputs. Each thread's commits
+      // track its own MMAs. A single thread runs dependent instructions and branches at a few
+      // cycles each, so each step is straight-line code: a wait, MMAs with compile-time operand
+      // offsets, commits. A descriptor is a fixed high word and a low word stepped by 32-bit adds
+      // (16-byte units: a K-step of 16 elements is +2 along a K-major row and +128, i.e. 16 rows,
+      // down an MN-major operand).
       if (rank == 0 && lane == 0) {
         constexpr uint32_t idesc_qk = idesc_f16(128, kTile, kBf16, false, false);
         constexpr uint32_t idesc_pv = idesc_f16(128, 256, kBf16, false, true);
         constexpr uint32_t hi = desc_sw128_hi(1024);
         constexpr uint32_t kChunkD = kChunk >> 4, kSetD = kSetBytes >> 4;
-        const uint32_t q_lo = desc_sw128_lo(data_u32 + kQOff, 16);
-        const uint32_t p_lo = desc_sw128_lo(data_u32 + kPOff, 16);
-        const uint32_t rope_lo = desc_sw128_lo(data_u32 + kRopeOff, 16);
-        const uint32_t k_lo = desc_sw128_lo(set_u32, 16);      // latent chunks as K-major B of S
-        const uint32_t v_lo = desc_sw128_lo(set_u32, kChunk);  // chunk pairs as MN-major B of O
         const uint32_t b_qk_full = bar(ctl->qk_full[0][0]), b_pv_full = bar(ctl->pv_full[0][0]);
         const uint32_t b_qk_done = bar(ctl->qk_done[0][0]), b_set_free = bar(ctl->set_free[0][0]);
         const uint32_t b_s_free = bar(ctl->s_free[0]), b_s_full = bar(ctl->s_full[0]);
-        auto mwait = [&](uint32_t b, uint32_t parity) {
+        auto wt = [&](uint32_t b, uint32_t parity) {
           if (mbar_wait(b, parity, abort_flag)) return true;
           st_cluster_u32(peer_abort, 1u);
           return false;
         };
-        // S(ti) = Q C^T into S buffer ti & 1 in two groups: the rope chunk and latent chunks 0-3
-        // (the first box), then chunks 4-7 (the second).
-        auto s_group = [&](int ti, int grp, bool first, bool last, int ii) {
-          const int s = ti & 1;
-          const uint32_t ph = (ti >> 1) & 1;
-          const uint32_t d = tmem + kSCol + 64 * s;
-          const uint32_t kb = k_lo + s * kSetD;
-          if (grp == 0) {
-            if (!mwait(b_s_free + 8 * s, ph ^ 1)) return false;  // softmax has read S(ti - 2)
-            if (first && !mwait(bar(ctl->q_full), ii & 1)) return false;
-            if (!mwait(bar(ctl->rope_full), ti & 1)) return false;
+        Cursor c;
+        c.start(prefix, p.B, cluster, nclusters);
+        if (warp == kMmaWarp) {
+          // S(i) = Q C^T into S buffer i & 1
+          const uint32_t q_lo = desc_sw128_lo(data_u32 + kQOff, 16);
+          const uint32_t rope_lo = desc_sw128_lo(data_u32 + kRopeOff, 16);
+          const uint32_t k_lo = desc_sw128_lo(set_u32, 16);  // latent chunks as K-major B
+          for (; c.valid; c.advance(prefix)) {
+            const int ti = c.ti, s = ti & 1;
+            const uint32_t ph = (ti >> 1) & 1;
+            const uint32_t d = tmem + kSCol + 64 * s;
+            const uint32_t kb = k_lo + s * kSetD;
+            if (!wt(b_s_free + 8 * s, ph ^ 1)) break;  // softmax has read S(i - 2)
+            if (c.first() && !wt(bar(ctl->q_full), c.ii & 1)) break;
+            if (!wt(bar(ctl->rope_full), ti & 1)) break;
             tc_fence_after();
 #pragma unroll
             for (int ks = 0; ks < 4; ++ks)
               mma2_ss_lohi(d, q_lo + 8 * kChunkD + 2 * ks, rope_lo + 2 * ks, hi, idesc_qk, ks != 0);
             mma_commit2(bar(ctl->rope_done), 3);
-          }
-          if (!mwait(b_qk_full + 8 * (2 * s + grp), ph)) return false;
-          tc_fence_after();
+            bool ok = true;
 #pragma unroll
-          for (int k4 = 0; k4 < 4; ++k4) {
-            const int kc = 4 * grp + k4;
+            for (int grp = 0; grp < 2; ++grp) {
+              if (!wt(b_qk_full + 8 * (2 * s + grp), ph)) {
+                ok = false;
+                break;
+              }
+              tc_fence_after();
 #pragma unroll
-            for (int ks = 0; ks < 4; ++ks)
-              mma2_ss_lohi(d, q_lo + kc * kChunkD + 2 * ks, kb + kc * kChunkD + 2 * ks, hi, idesc_qk, 1);
-            if (k4 & 1) mma_commit2(b_qk_done + 8 * (4 * s + (kc >> 1)), 3);
-          }
-          if (grp == 1) {
+              for (int k4 = 0; k4 < 4; ++k4) {
+                const int kc = 4 * grp + k4;
+#pragma unroll
+                for (int ks = 0; ks < 4; ++ks)
+                  mma2_ss_lohi(d, q_lo + kc * kChunkD + 2 * ks, kb + kc * kChunkD + 2 * ks, hi, idesc_qk, 1);
+                if (k4 & 1) mma_commit2(b_qk_done + 8 * (4 * s + (kc >> 1)), 3);
+              }
+            }
+            if (!ok) break;
             mma_commit2(b_s_full + 8 * s, 3);
-            if (last) mma_commit2(bar(ctl->q_free), 3);
+            if (c.last()) mma_commit2(bar(ctl->q_free), 3);
           }
-          return true;
-        };
-        // O += P C_lat for tile ti: pairs (g, j) = (0,0), (1,0), (0,1), (1,1); chunks 0-3 of the
-        // set are released after the first two.
-        auto o_step = [&](int ti, bool first, int ii) {
-          const int s = ti & 1;
-          const uint32_t ph = (ti >> 1) & 1;
-          if (!mwait(bar(ctl->p_full), ti & 1)) return false;  // P written, O rescaled
-          if (first && !mwait(bar(ctl->o_free), (ii & 1) ^ 1)) return false;  // O of the item before read out
-          const uint32_t vb = v_lo + s * kSetD;
+        } else {
+          // O += P C_lat, pairs (g, j) = (0,0), (1,0), (0,1), (1,1); chunks 0-3 of the set are
+          // released after the first two
+          const uint32_t p_lo = desc_sw128_lo(data_u32 + kPOff, 16);
+          const uint32_t v_lo = desc_sw128_lo(set_u32, kChunk);  // chunk pairs as MN-major B
+          for (; c.valid; c.advance(prefix)) {
+            const int ti = c.ti, s = ti & 1;
+            const uint32_t ph = (ti >> 1) & 1;
+            const bool first = c.first();
+            const uint32_t vb = v_lo + s * kSetD;
+            if (!wt(bar(ctl->p_full), ti & 1)) break;  // P written, O rescaled
+            if (first && !wt(bar(ctl->o_free), (c.ii & 1) ^ 1)) break;  // O of the item before read out
+            bool ok = true;
 #pragma unroll
-          for (int gq = 0; gq < 4; ++gq) {
-            const int g = gq & 1, jh = gq >> 1, pr = 2 * jh + g;
-            if (!mwait(b_pv_full + 8 * (4 * s + pr), ph)) return false;
-            tc_fence_after();
-            const uint32_t d = tmem + kOCol + 128 * jh;
-            mma2_ss_lohi(d, p_lo + g * kChunkD, vb + 2 * pr * kChunkD, hi, idesc_pv, g != 0 || !first);
+            for (int gq = 0; gq < 4; ++gq) {
+              const int g = gq & 1, jh = gq >> 1, pr = 2 * jh + g;
+              if (!wt(b_pv_full + 8 * (4 * s + pr), ph)) {
+                ok = false;
+                break;
+              }
+              tc_fence_after();
+              const uint32_t d = tmem + kOCol + 128 * jh;
+              mma2_ss_lohi(d, p_lo + g * kChunkD, vb + 2 * pr * kChunkD, hi, idesc_pv, g != 0 || !first);
 #pragma unroll
-            for (int ks = 1; ks < 4; ++ks)
-              mma2_ss_lohi(d, p_lo + g * kChunkD + 2 * ks, vb + 2 * pr * kChunkD + 128 * ks, hi, idesc_pv, 1);
-            if (gq == 1) mma_commit2(b_set_free + 8 * (2 * s), 3);
+              for (int ks = 1; ks < 4; ++ks)
+                mma2_ss_lohi(d, p_lo + g * kChunkD + 2 * ks, vb + 2 * pr * kChunkD + 128 * ks, hi, idesc_pv, 1);
+              if (gq == 1) mma_commit2(b_set_free + 8 * (2 * s), 3);
+            }
+            if (!ok) break;
+            mma_commit2(bar(ctl->p_free), 3);
+            mma_commit2(b_set_free + 8 * (2 * s + 1), 3);
           }
-          mma_commit2(bar(ctl->p_free), 3);
-          mma_commit2(b_set_free + 8 * (2 * s + 1), 3);
-          return true;
-        };
-        Cursor c;
-        c.start(prefix, p.B, cluster, nclusters);
-        int prev_ti = -1, prev_ii = 0;
-        bool prev_first = false;
-        while (c.valid) {
-          if (!s_group(c.ti, 0, c.first(), c.last(), c.ii)) break;
-          if (prev_ti >= 0 && !o_step(prev_ti, prev_first, prev_ii)) break;
-          if (!s_group(c.ti, 1, c.first(), c.last(), c.ii)) break;
-          prev_ti = c.ti;
-          prev_first = c.first();
-          prev_ii = c.ii;
-          c.advance(prefix);
         }
-        if (!c.valid && prev_ti >= 0) o_step(prev_ti, prev_first, prev_ii);
+        mma_commit2(bar(ctl->drain), 1);  // once all of this thread's MMAs are complete
       }
       __syncwarp();
     } else if (warp < kSoftWarps) {
@@ -670,10 +671,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(dec::kThreads, 1)
 
   // ---------------------------------------------------------------- teardown
   if (has_work && warp == kMmaWarp && rank == 0) {
-    if (lane == 0) {  // every pair MMA has completed before either CTA releases its tensor memory
-      mma_commit2(bar(ctl->drain), 1);
-      mbar_wait_slow<false>(bar(ctl->drain), 0, nullptr);
-    }
+    // every pair MMA (of both issuing threads) has completed before either CTA releases its
+    // tensor memory
+    if (lane == 0) mbar_wait_slow<false>(bar(ctl->drain), 0, nullptr);
     __syncwarp();
   }
   if (*abort_flag && threadIdx.x == 0) {
