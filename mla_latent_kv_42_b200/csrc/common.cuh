@@ -13,6 +13,9 @@
 
 namespace mla {
 
+constexpr float kLog2e = 1.4426950408889634f;
+constexpr float kLn2 = 0.6931471805599453f;
+
 // First device-side error since the last mla_read_device_status (0 = none). Kernels record
 // errors here instead of trapping; the first writer wins.
 __device__ int g_status;

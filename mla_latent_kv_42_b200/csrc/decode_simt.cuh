@@ -7,8 +7,6 @@
 
 namespace mla {
 
-constexpr float kLog2e = 1.4426950408889634f;
-constexpr float kLn2 = 0.6931471805599453f;
 
 // grid (n_splits, B, ceil(n_h / 8)), block 256 (warp w -> head blockIdx.z*8 + w).
 // NPAIR = ceil(D / 64): element pairs of one row held per lane.

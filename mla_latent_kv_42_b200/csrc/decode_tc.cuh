@@ -112,6 +112,7 @@ struct DecodeTcParams {
 // wholly past the end (nv = 0) loads as zeros. Softmax masks slot rows r < 64 - nv.
 struct DecodeTcMaps {
   CUtensorMap page1, page2, page4, q9;
+  CUtensorMap o_lat, o_part;  // outputs as (512 columns, n_h heads, rows), 64-byte x 32-head boxes
 };
 
 // Tiles [t0, t1) of sequence b handled by this pair (n_b = tiles of the sequence).
@@ -174,6 +175,13 @@ struct Cursor {
     }
   }
 };
+
+// Most SM pairs one call spreads its tiles over (the merge kernel lists a sequence's pairs).
+constexpr int kMaxDecodeClusters = 128;
+// A sequence whose tiles fall to pairs c0 < c1 is merged by the merge kernel from the pairs'
+// partials (fp32 o / l and lse in slot b + c). The planner gives each sequence
+// c0 | c1 << 16 | all << 28 (all: every pair has tiles, so the slots are b + c0 .. b + c1),
+// or -1 without tiles.
 
 // Pair that owns global tile g when T tiles are split over C pairs as [T c / C, T (c+1) / C).
 __device__ __forceinline__ int cluster_of(long g, long T, int C) { return (int)(((g + 1) * C - 1) / T); }
@@ -589,30 +597,34 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(dec::kThreads, 1)
           if (!exchange(lsum, four)) break;
           const float l = (four[0] + four[1]) + (four[2] + four[3]);
           const float inv = l > 0.f ? 1.f / l : 0.f;
-          const float lse = l > 0.f ? (m_ref + log2f(l)) * 0.6931471805599453f : -INFINITY;
+          const float lse = l > 0.f ? (m_ref + log2f(l)) * kLn2 : -INFINITY;
           const Item& it = c.item;
           const bool whole = it.t0 == 0 && it.t1 == it.n_b;
           const long slot = (long)it.b + cluster;
           const int col0 = 256 * ch + 128 * g;  // latent columns [col0, col0 + 128)
           // The warp writes its 32 heads x 128 columns in rounds of 64 bytes per head through its
-          // own 2 KB of the P buffer (free: the last O MMAs are done). Each lane puts its head's
-          // segment in row `lane` (16-byte chunks swizzled by row, conflict-free both ways), and
-          // each store instruction then writes 8 heads x 64 contiguous bytes.
+          // own 2 KB of the P buffer (free: the last O MMAs are done): each lane puts its head's
+          // segment in row `lane` in the 64-byte swizzle (16-byte chunk c of row r at c ^ (r/2 % 4),
+          // conflict-free), and lane 0 stores the 32 x 64-byte box with one TMA store, which heads
+          // past n_h fall outside of. The warp goes on while the copy engine reads the box.
           uint8_t* const stage = data + kPOff + warp * 2048;
+          const uint32_t stage_u32 = data_u32 + kPOff + warp * 2048;
           const uint32_t wsw = (lane >> 1) & 3;
-          const int rq = lane >> 2, cq = lane & 3;
-          auto stage_put = [&](const uint32_t (&w)[16]) {
+          const int head0 = 64 * (int)rank + 32 * (qd & 1);
+          auto stage_store = [&](const uint32_t (&w)[16], int col) {
+            if (lane == 0) bulk_wait_read<0>();  // the previous round's box has been read
+            __syncwarp();
 #pragma unroll
             for (int i2 = 0; i2 < 4; ++i2)
               *reinterpret_cast<uint4*>(stage + lane * 64 + ((i2 ^ wsw) << 4)) =
                   make_uint4(w[4 * i2], w[4 * i2 + 1], w[4 * i2 + 2], w[4 * i2 + 3]);
+            fence_proxy_async_cta();
             __syncwarp();
-          };
-          // row 8k + rq of the round: its head and its chunk cq
-          auto stage_get = [&](int k, int& hd) {
-            const int row = 8 * k + rq;
-            hd = 64 * (int)rank + ((32 * qd + row) & 63);
-            return *reinterpret_cast<const uint4*>(stage + row * 64 + ((cq ^ ((row >> 1) & 3)) << 4));
+            if (lane == 0) {
+              if (whole) tma_store_3d(&maps.o_lat, stage_u32, col, head0, it.b);
+              else tma_store_3d(&maps.o_part, stage_u32, col, head0, (int)slot);
+              bulk_commit_group();
+            }
           };
 #pragma unroll 1
           for (int c0 = 0; c0 < 128; c0 += 32) {
@@ -626,30 +638,14 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(dec::kThreads, 1)
                 const typename Pack<T>::T2 v = Pack<T>::make(u2f(r[2 * e]) * inv, u2f(r[2 * e + 1]) * inv);
                 w[e] = *reinterpret_cast<const uint32_t*>(&v);
               }
-              stage_put(w);
-              T* const ob = static_cast<T*>(p.o_lat) + (long)it.b * p.n_h * kDc + col0 + c0 + 8 * cq;
-#pragma unroll
-              for (int k = 0; k < 4; ++k) {
-                int hd;
-                const uint4 v = stage_get(k, hd);
-                if (hd < p.n_h) *reinterpret_cast<uint4*>(ob + (long)hd * kDc) = v;
-              }
-              __syncwarp();
+              stage_store(w, col0 + c0);
             } else {  // 16 columns of fp32 per round
 #pragma unroll
               for (int half = 0; half < 2; ++half) {
                 uint32_t w[16];
 #pragma unroll
                 for (int e = 0; e < 16; ++e) w[e] = __float_as_uint(u2f(r[16 * half + e]) * inv);
-                stage_put(w);
-                float* const ob = p.o_part + slot * p.n_h * kDc + col0 + c0 + 16 * half + 4 * cq;
-#pragma unroll
-                for (int k = 0; k < 4; ++k) {
-                  int hd;
-                  const uint4 v = stage_get(k, hd);
-                  if (hd < p.n_h) *reinterpret_cast<uint4*>(ob + (long)hd * kDc) = v;
-                }
-                __syncwarp();
+                stage_store(w, col0 + c0 + 16 * half);
               }
             }
           }
@@ -660,6 +656,13 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(dec::kThreads, 1)
               p.lse_part[slot * p.n_h + head] = lse;
             }
           }
+          // the boxes have left the P buffer before the next tile's softmax writes it; at the
+          // pair's last item they are also complete in global memory before the CTA exits
+          if (lane == 0) {
+            if (c.it.g >= c.it.g_end) bulk_wait<0>();
+            else bulk_wait_read<0>();
+          }
+          __syncwarp();
           tc_fence_before();
           __syncwarp();
           if (lane == 0) mbar_arrive_cl(lead(ctl->o_free));
@@ -698,113 +701,215 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(dec::kThreads, 1)
 // its block-table row), then a block-wide scan turns the counts into offsets in place. The host
 // keeps the total (B x tiles of max_seq_len) within int32.
 __global__ void __launch_bounds__(1024) k_decode_plan(const int* __restrict__ seq_lens, const int* __restrict__ bt,
-                                                      int B, int max_pages, int num_pages, int max_seq_len,
-                                                      int* __restrict__ tile_prefix) {
+                                                      int B, int max_pages, int num_pages, int max_seq_len, int C,
+                                                      int* __restrict__ tile_prefix, int* __restrict__ seq_pairs,
+                                                      int* __restrict__ pair_start) {
   griddep_wait();
   if (threadIdx.x == 0) griddep_launch();
-  __shared__ int part[1024];
+  __shared__ int warp_total[32];
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  for (int b = warp; b < B; b += 32) {
-    const int L = seq_lens[b];
-    const int n = (int)(((long)L + dec::kPage - 1) / dec::kPage);
-    bool ok = L >= 1 && L <= max_seq_len && n <= max_pages;
-    if (!ok && lane == 0) record_error(MLA_ERR_BAD_SEQ_LEN);
-    if (ok) {
-      bool bad = false;
-      for (int t = lane; t < n; t += 32) {
+  // Tiles of each sequence (0 for a rejected one), a half-warp per sequence, 64 sequences per
+  // pass; every lane runs every pass so the ballot below is warp-uniform.
+  const int grp = 2 * warp + (lane >> 4), sub = lane & 15;
+  const unsigned half = (lane >> 4) ? 0xffff0000u : 0x0000ffffu;
+  for (int b0 = 0; b0 < B; b0 += 64) {
+    const int b = b0 + grp;
+    int L = 0, n = 0;
+    bool ok = false;
+    if (b < B) {
+      L = seq_lens[b];
+      n = (int)(((long)L + dec::kPage - 1) / dec::kPage);
+      ok = L >= 1 && L <= max_seq_len && n <= max_pages;
+      if (!ok && sub == 0) record_error(MLA_ERR_BAD_SEQ_LEN);
+    }
+    bool bad = false;
+    if (ok)
+      for (int t = sub; t < n; t += 16) {
         const int pg = bt[(long)b * max_pages + t];
         bad |= pg < 0 || pg >= num_pages;
       }
-      if (__any_sync(0xffffffffu, bad)) {
-        ok = false;
-        if (lane == 0) record_error(MLA_ERR_BAD_PAGE);
-      }
+    const bool any_bad = (__ballot_sync(0xffffffffu, bad) & half) != 0;
+    if (ok && any_bad) {
+      ok = false;
+      if (sub == 0) record_error(MLA_ERR_BAD_PAGE);
     }
-    if (lane == 0) tile_prefix[b] = ok ? (int)(((long)L + dec::kTile - 1) / dec::kTile) : 0;
+    if (b < B && sub == 0) tile_prefix[b] = ok ? (int)(((long)L + dec::kTile - 1) / dec::kTile) : 0;
   }
   __syncthreads();
+  // exclusive scan: thread tid sums the counts of sequences [tid * per, tid * per + per), then a
+  // two-level warp-shuffle scan over the 1024 thread sums
   const int per = (B + 1023) / 1024;
   const int b0 = min(B, tid * per), b1 = min(B, b0 + per);
   int sum = 0;
   for (int b = b0; b < b1; ++b) sum += tile_prefix[b];
-  part[tid] = sum;
-  __syncthreads();
-  for (int off = 1; off < 1024; off <<= 1) {
-    const int v = tid >= off ? part[tid - off] : 0;
-    __syncthreads();
-    part[tid] += v;
-    __syncthreads();
+  int incl = sum;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const int v = __shfl_up_sync(0xffffffffu, incl, o);
+    if (lane >= o) incl += v;
   }
-  int run = tid > 0 ? part[tid - 1] : 0;
+  if (lane == 31) warp_total[warp] = incl;
+  __syncthreads();
+  if (warp == 0) {
+    int w = warp_total[lane];
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int v = __shfl_up_sync(0xffffffffu, w, o);
+      if (lane >= o) w += v;
+    }
+    warp_total[lane] = w;  // inclusive over warps
+  }
+  __syncthreads();
+  // Pair c takes tiles [T c / C, T (c+1) / C) (T = all tiles); each sequence gets the first and
+  // last pair its tiles fall to (c0 | c1 << 16, or -1 without tiles), for the merge.
+  const long T_ = warp_total[31];
+  int run = incl - sum + (warp > 0 ? warp_total[warp - 1] : 0);
   for (int b = b0; b < b1; ++b) {
     const int n = tile_prefix[b];
     tile_prefix[b] = run;
+    if (n > 0) {
+      const int c0 = cluster_of(run, T_, C), c1 = cluster_of(run + n - 1, T_, C);
+      seq_pairs[b] = c0 | (c1 << 16) | ((T_ >= C ? 1 : 0) << 28);
+    } else {
+      seq_pairs[b] = -1;
+    }
     run += n;
   }
-  if (tid == 1023) tile_prefix[B] = part[1023];
+  if (tid <= C) pair_start[tid] = (int)(T_ * tid / C);
+  if (tid == 1023) tile_prefix[B] = (int)T_;
 }
 
 // Merge of the partials of sequences that span pairs, in pair order; zero output for rejected
 // sequences. grid (B, ceil(n_h / 8)), 256 threads: one warp per head, each lane 16 of the 512
 // latent values (four 16-byte loads per contributing pair, all in flight together).
 template <typename T>
-__global__ void __launch_bounds__(256) k_decode_tc_merge(const float* __restrict__ o_part,
+__global__ void __launch_bounds__(512) k_decode_tc_merge(const float* __restrict__ o_part,
                                                           const float* __restrict__ lse_part,
-                                                          const int* __restrict__ tile_prefix, int B, int C, int n_h,
+                                                          const int* __restrict__ seq_pairs,
+                                                          const int* __restrict__ pair_start, int n_h,
                                                           T* __restrict__ o_lat, float* __restrict__ lse_out) {
   griddep_wait();
   if (threadIdx.x == 0) griddep_launch();
+  // grid (B, ceil(n_h / 32)), 16 warps of two heads each. Warp 0 lists the partial slots of
+  // sequence b (the pairs its tiles fall to, in pair order, skipping pairs without tiles): n = -1
+  // when one pair wrote it whole, 0 when it has no tiles (rejected: zero output).
+  __shared__ int s_slot[kMaxDecodeClusters];
+  __shared__ int s_n;
   const int b = blockIdx.x, warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int h = blockIdx.y * 8 + warp;
-  if (h >= n_h) return;
-  const long T_ = tile_prefix[B];
-  const int g0 = tile_prefix[b], g1 = tile_prefix[b + 1];
-  T* out = o_lat + ((long)b * n_h + h) * dec::kDc;
-  if (g1 == g0) {
-    for (int e = lane; e < dec::kDc; e += 32) Out<T>::put(out + e, 0.f);
-    if (lse_out != nullptr && lane == 0) lse_out[(long)b * n_h + h] = -INFINITY;
+  if (warp == 0) {
+    const int sp = seq_pairs[b];
+    int n = 0;
+    if (sp >= 0) {
+      const int c0 = sp & 0xffff, c1 = (sp >> 16) & 0xfff;
+      if (c0 == c1) {
+        n = -1;
+      } else if ((sp >> 28) & 1) {  // every pair has tiles
+        n = c1 - c0 + 1;
+        for (int k = lane; k < n; k += 32) s_slot[k] = b + c0 + k;
+      } else {
+        for (int cb = c0; cb <= c1; cb += 32) {
+          const int c = cb + lane;
+          const bool own = c <= c1 && pair_start[c + 1] > pair_start[c];
+          const unsigned m = __ballot_sync(0xffffffffu, own);
+          if (own) s_slot[n + __popc(m & ((1u << lane) - 1u))] = b + c;
+          n += __popc(m);
+        }
+      }
+    }
+    if (lane == 0) s_n = n;
+  }
+  __syncthreads();
+  const int n = s_n, h0 = blockIdx.y * 32 + 2 * warp;
+  if (n < 0 || h0 >= n_h) return;
+  const int nh = min(2, n_h - h0);
+  if (n == 0) {
+    for (int hh = 0; hh < nh; ++hh) {
+      T* out = o_lat + ((long)b * n_h + h0 + hh) * dec::kDc;
+      for (int e = lane; e < dec::kDc; e += 32) Out<T>::put(out + e, 0.f);
+      if (lse_out != nullptr && lane == 0) lse_out[(long)b * n_h + h0 + hh] = -INFINITY;
+    }
     return;
   }
-  const int c0 = cluster_of(g0, T_, C), c1 = cluster_of(g1 - 1, T_, C);
-  if (c0 == c1) return;  // written whole by its pair
-  // pairs between c0 and c1 own consecutive tiles of this sequence, except those whose range is
-  // empty (fewer tiles than pairs): they wrote nothing and are skipped
-  auto owns = [&](int c) { return T_ * (c + 1) / C > T_ * c / C; };
-  const float* lp = lse_part + (long)b * n_h + h;  // slot b + c is at lp[c * n_h]
-  float mx = -INFINITY;
-  for (int c = c0; c <= c1; ++c)
-    if (owns(c)) mx = fmaxf(mx, lp[(long)c * n_h]);
-  float z = 0.f;
-  for (int c = c0; c <= c1; ++c)
-    if (owns(c)) z += exp2f((lp[(long)c * n_h] - mx) * 1.4426950408889634f);
-  const float inv = 1.f / z;
-  float4 acc[4];
+  auto row = [&](int i, int hh) {
+    return reinterpret_cast<const float4*>(o_part + ((long)s_slot[i] * n_h + h0 + hh) * dec::kDc);
+  };
+  auto lse_of = [&](int i, int hh) { return lse_part[(long)s_slot[i] * n_h + h0 + hh]; };
+  // The first two partial rows of both heads are requested before the weights are formed, so
+  // that a sequence split over two pairs takes one round trip.
+  float4 pre[2][2][4];
 #pragma unroll
-  for (int j = 0; j < 4; ++j) acc[j] = make_float4(0.f, 0.f, 0.f, 0.f);
-#pragma unroll 2
-  for (int c = c0; c <= c1; ++c) {
-    if (!owns(c)) continue;
-    const float w = exp2f((lp[(long)c * n_h] - mx) * 1.4426950408889634f);
-    const float4* src = reinterpret_cast<const float4*>(o_part + (((long)b + c) * n_h + h) * dec::kDc);
-    float4 v[4];
+  for (int hh = 0; hh < 2; ++hh)
 #pragma unroll
-    for (int j = 0; j < 4; ++j) v[j] = src[lane + 32 * j];
+    for (int i = 0; i < 2; ++i)
+#pragma unroll
+      for (int j = 0; j < 4; ++j)
+        pre[hh][i][j] = hh < nh && i < n ? row(i, hh)[lane + 32 * j] : make_float4(0.f, 0.f, 0.f, 0.f);
+  // weights e^{lse_i - max}: lane i holds lse_i (i < 32); the sums run over lanes in a fixed order
+  float lp[2], mx[2], z[2];
+#pragma unroll
+  for (int hh = 0; hh < 2; ++hh) {
+    lp[hh] = hh < nh && lane < n ? lse_of(lane, hh) : -INFINITY;
+    float m = lp[hh];
+    for (int i = lane + 32; i < n; i += 32) m = fmaxf(m, hh < nh ? lse_of(i, hh) : -INFINITY);
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
+    mx[hh] = m;
+    float zz = lp[hh] > -INFINITY ? exp2f((lp[hh] - m) * kLog2e) : 0.f;
+    for (int i = lane + 32; i < n; i += 32) zz += hh < nh ? exp2f((lse_of(i, hh) - m) * kLog2e) : 0.f;
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) zz += __shfl_xor_sync(0xffffffffu, zz, o);
+    z[hh] = zz;
+  }
+  float4 acc[2][4];
+#pragma unroll
+  for (int hh = 0; hh < 2; ++hh) {
+#pragma unroll
+    for (int j = 0; j < 4; ++j) acc[hh][j] = make_float4(0.f, 0.f, 0.f, 0.f);
+  }
+  auto add = [&](int hh, float w, const float4 (&v)[4]) {
 #pragma unroll
     for (int j = 0; j < 4; ++j) {
-      acc[j].x = fmaf(w, v[j].x, acc[j].x);
-      acc[j].y = fmaf(w, v[j].y, acc[j].y);
-      acc[j].z = fmaf(w, v[j].z, acc[j].z);
-      acc[j].w = fmaf(w, v[j].w, acc[j].w);
+      acc[hh][j].x = fmaf(w, v[j].x, acc[hh][j].x);
+      acc[hh][j].y = fmaf(w, v[j].y, acc[hh][j].y);
+      acc[hh][j].z = fmaf(w, v[j].z, acc[hh][j].z);
+      acc[hh][j].w = fmaf(w, v[j].w, acc[hh][j].w);
+    }
+  };
+  auto weight = [&](int i, int hh) {
+    const float li = i < 32 ? __shfl_sync(0xffffffffu, lp[hh], i) : lse_of(i, hh);
+    return li > -INFINITY ? exp2f((li - mx[hh]) * kLog2e) : 0.f;
+  };
+#pragma unroll
+  for (int hh = 0; hh < 2; ++hh) {  // the prefetched rows (weight 0 past n or nh: zero rows)
+    const float w0 = weight(0, hh), w1 = weight(1, hh);
+    add(hh, hh < nh ? w0 : 0.f, pre[hh][0]);
+    add(hh, hh < nh && n > 1 ? w1 : 0.f, pre[hh][1]);
+  }
+  for (int i = 2; i < n; ++i) {
+#pragma unroll
+    for (int hh = 0; hh < 2; ++hh) {
+      const float w = weight(i, hh);
+      if (hh >= nh) continue;
+      float4 v[4];
+#pragma unroll
+      for (int j = 0; j < 4; ++j) v[j] = row(i, hh)[lane + 32 * j];
+      add(hh, w, v);
     }
   }
-  typename Pack<T>::T2* dst = reinterpret_cast<typename Pack<T>::T2*>(out);
 #pragma unroll
-  for (int j = 0; j < 4; ++j) {
-    const int e = 4 * (lane + 32 * j);
-    dst[e / 2] = Pack<T>::make(acc[j].x * inv, acc[j].y * inv);
-    dst[e / 2 + 1] = Pack<T>::make(acc[j].z * inv, acc[j].w * inv);
+  for (int hh = 0; hh < 2; ++hh) {
+    if (hh >= nh) continue;
+    const float inv = z[hh] > 0.f ? 1.f / z[hh] : 0.f;
+    typename Pack<T>::T2* dst = reinterpret_cast<typename Pack<T>::T2*>(o_lat + ((long)b * n_h + h0 + hh) * dec::kDc);
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      const int e = 4 * (lane + 32 * j);
+      dst[e / 2] = Pack<T>::make(acc[hh][j].x * inv, acc[hh][j].y * inv);
+      dst[e / 2 + 1] = Pack<T>::make(acc[hh][j].z * inv, acc[hh][j].w * inv);
+    }
+    if (lse_out != nullptr && lane == 0)
+      lse_out[(long)b * n_h + h0 + hh] = z[hh] > 0.f ? mx[hh] + logf(z[hh]) : -INFINITY;
   }
-  if (lse_out != nullptr && lane == 0) lse_out[(long)b * n_h + h] = mx + logf(z);
 }
 
 }  // namespace tc

@@ -5,6 +5,7 @@
 #include "mla_debug.h"
 #include <nvtx3/nvToolsExt.h>
 
+#include <algorithm>
 #include <atomic>
 #include <cmath>
 #include <cstring>
@@ -202,7 +203,7 @@ int decode_clusters() {
       if (cudaOccupancyMaxActiveClusters(&n, tc::k_decode_tc<__nv_bfloat16>, &cfg) != cudaSuccess) n = 0;
     }
     cudaGetLastError();
-    c = n > 0 ? n : device_sm_count() / 2;
+    c = std::min(n > 0 ? n : device_sm_count() / 2, tc::kMaxDecodeClusters);
     cache[dev].store(c, std::memory_order_relaxed);
   }
   return c;
@@ -210,8 +211,8 @@ int decode_clusters() {
 
 size_t ws_decode_tc(const mla_dims* d, int B) {
   const size_t slots = (size_t)B + decode_clusters();
-  return align256((size_t)(B + 1) * 4) + align256(slots * d->n_heads * tc::dec::kDc * 4) +
-         align256(slots * d->n_heads * 4);
+  return align256((size_t)(B + 1) * 4) + align256((size_t)B * 4) + align256((tc::kMaxDecodeClusters + 1) * 4) +
+         align256(slots * d->n_heads * tc::dec::kDc * 4) + align256(slots * d->n_heads * 4);
 }
 
 // Pages of the longest sequence; the planner's page counts, summed over a launch, must stay in
@@ -240,6 +241,8 @@ int decode_tc_impl(const mla_dims* d, const void* q, const void* pool, int32_t n
   if (!decode_tc_set_smem<T>()) return MLA_ERR_CUDA;
   Carve c{static_cast<char*>(ws)};
   int* prefix = c.take<int>((size_t)B + 1);
+  int* seq_pairs = c.take<int>((size_t)B);
+  int* pair_start = c.take<int>(tc::kMaxDecodeClusters + 1);
   float* o_part = c.take<float>(((size_t)B + C) * d->n_heads * tc::dec::kDc);
   float* lse_part = c.take<float>(((size_t)B + C) * d->n_heads);
   constexpr bool bf16 = tc::IsBf16<T>::value;
@@ -247,10 +250,14 @@ int decode_tc_impl(const mla_dims* d, const void* q, const void* pool, int32_t n
   if (!host::encode_pages(&maps.page1, pool, bf16, (uint64_t)num_pages, tc::dec::kD * 2, 1) ||
       !host::encode_pages(&maps.page2, pool, bf16, (uint64_t)num_pages, tc::dec::kD * 2, 2) ||
       !host::encode_pages(&maps.page4, pool, bf16, (uint64_t)num_pages, tc::dec::kD * 2, 4) ||
-      !host::encode_chunks(&maps.q9, q, bf16, (uint64_t)B * d->n_heads, tc::dec::kD * 2, 9))
+      !host::encode_chunks(&maps.q9, q, bf16, (uint64_t)B * d->n_heads, tc::dec::kD * 2, 9) ||
+      !host::encode_heads_out(&maps.o_lat, o_lat, bf16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT16,
+                              2, (uint64_t)d->n_heads, (uint64_t)B) ||
+      !host::encode_heads_out(&maps.o_part, o_part, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, (uint64_t)d->n_heads,
+                              (uint64_t)B + C))
     return MLA_ERR_CUDA;
   if (launch_pdl(tc::k_decode_plan, dim3(1), dim3(1024), 0, st, seq_lens, bt, (int)B, (int)max_pages, (int)num_pages,
-                 (int)max_seq_len, prefix) != cudaSuccess)
+                 (int)max_seq_len, C, prefix, seq_pairs, pair_start) != cudaSuccess)
     return MLA_ERR_CUDA;
   tc::DecodeTcParams p;
   p.bt = bt;
@@ -268,10 +275,10 @@ int decode_tc_impl(const mla_dims* d, const void* q, const void* pool, int32_t n
   if (launch_pdl(tc::k_decode_tc<T>, dim3(2 * C), dim3(tc::dec::kThreads), tc::dec::kSmem, st, maps, p) != cudaSuccess)
     return MLA_ERR_CUDA;
   mark_after(st);
-  if (launch_pdl(tc::k_decode_tc_merge<T>, dim3(B, (d->n_heads + 7) / 8), dim3(256), 0, st,
+  if (launch_pdl(tc::k_decode_tc_merge<T>, dim3(B, (d->n_heads + 31) / 32), dim3(512), 0, st,
                  static_cast<const float*>(o_part), static_cast<const float*>(lse_part),
-                 static_cast<const int*>(prefix), (int)B, C, (int)d->n_heads, static_cast<T*>(o_lat),
-                 lse_out) != cudaSuccess)
+                 static_cast<const int*>(seq_pairs), static_cast<const int*>(pair_start), (int)d->n_heads,
+                 static_cast<T*>(o_lat), lse_out) != cudaSuccess)
     return MLA_ERR_CUDA;
   launches += 3;
   return MLA_OK;
