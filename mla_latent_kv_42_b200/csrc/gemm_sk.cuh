@@ -232,22 +232,36 @@ __global__ void __launch_bounds__(192, 2)
                     kbi * C::BK + z * p.b_batch_off, nt * BN);
       };
       const int pre = min(S, n_it);
-      for (int j = 0; j < pre; ++j) {  // ring slots start empty: no wait
-        const long i = i0 + j;
-        int z, mt, nt;
-        tile_coords((int)(i / p.kb), z, mt, nt);
-        mbar_arrive_expect_tx(smem_u32(full + j), C::STAGE_BYTES);
-        load_a(j, z, mt, (int)(i % p.kb));
+      // (z, m tile, n tile, k block) of iteration i0, stepped with adds: one division per CTA
+      int z0, mt0, nt0;
+      const int tile0 = (int)(i0 / p.kb), kb0 = (int)(i0 - (long)tile0 * p.kb);
+      tile_coords(tile0, z0, mt0, nt0);
+      auto step = [&](int& z, int& mt, int& nt, int& kbi) {
+        if (++kbi == p.kb) {
+          kbi = 0;
+          if (++nt == p.n_tiles) {
+            nt = 0;
+            if (++mt == p.m_tiles) {
+              mt = 0;
+              ++z;
+            }
+          }
+        }
+      };
+      {
+        int z = z0, mt = mt0, nt = nt0, kbi = kb0;
+        for (int j = 0; j < pre; ++j) {  // ring slots start empty: no wait
+          mbar_arrive_expect_tx(smem_u32(full + j), C::STAGE_BYTES);
+          load_a(j, z, mt, kbi);
+          step(z, mt, nt, kbi);
+        }
       }
       griddep_wait();
+      int z = z0, mt = mt0, nt = nt0, kbi = kb0;
       for (int j = 0; j < pre; ++j) {
-        const long i = i0 + j;
-        int z, mt, nt;
-        tile_coords((int)(i / p.kb), z, mt, nt);
-        load_b(j, z, nt, (int)(i % p.kb));
+        load_b(j, z, nt, kbi);
+        step(z, mt, nt, kbi);
       }
-      int z, mt, nt, kbi = (int)((i0 + pre) % p.kb);
-      tile_coords((int)((i0 + pre) / p.kb), z, mt, nt);
       int s = pre % S, it = pre;
       uint32_t ph = pre == S ? 1u : 0u;
       for (; it < n_it; ++it) {
@@ -259,16 +273,7 @@ __global__ void __launch_bounds__(192, 2)
           s = 0;
           ph ^= 1;
         }
-        if (++kbi == p.kb) {
-          kbi = 0;
-          if (++nt == p.n_tiles) {
-            nt = 0;
-            if (++mt == p.m_tiles) {
-              mt = 0;
-              ++z;
-            }
-          }
-        }
+        step(z, mt, nt, kbi);
       }
       if (*abort_flag) {  // copies still in flight land before the CTA exits
         for (int j = max(0, it - S); j < it; ++j) mbar_wait_slow<false>(smem_u32(full + j % S), (j / S) & 1, nullptr);
@@ -321,13 +326,16 @@ __global__ void __launch_bounds__(192, 2)
     // n tiles the step computes them per element instead.
     // Shared-memory tables are built only by CTAs that finish a whole tile themselves: the cache
     // row offsets for any whole append tile, the RoPE cos/sin for a whole tile with rope rows.
+    // The CTA's segments: the first starts at k block kb0 of tile tile0 (one division per CTA),
+    // the others at tile starts.
+    const int tile0 = (int)(i0 / p.kb), kb0 = (int)(i0 - (long)tile0 * p.kb);
     bool tab_row = false, tab_cs = false;
     if (MODE != kEpiPlain && p.n_tiles == 1) {
-      for (long i = i0; i < i1;) {
-        const int tile = (int)(i / p.kb);
+      int tile = tile0, kbi0 = kb0;
+      for (long i = i0; i < i1; ++tile, kbi0 = 0) {
         const long tile_end = (long)(tile + 1) * p.kb, seg_end = min(i1, tile_end);
-        const bool rope_tile = ((tile / p.n_tiles) % p.m_tiles) * C::BM + C::BM > p.epi.rope_lo;
-        if (i % p.kb == 0 && seg_end == tile_end && !(p.epi.rope_in_reduce && rope_tile)) {
+        const bool rope_tile = (tile % p.m_tiles) * C::BM + C::BM > p.epi.rope_lo;  // n_tiles == 1
+        if (kbi0 == 0 && seg_end == tile_end && !(p.epi.rope_in_reduce && rope_tile)) {
           tab_row |= MODE == kEpiAppend;
           tab_cs |= rope_tile;
         }
@@ -372,10 +380,9 @@ __global__ void __launch_bounds__(192, 2)
         row_tab[e] = rb;
       }
     if (tab_cs || tab_row) named_bar_sync(1, 128);
-    int seg = 0;
+    int seg = 0, tile = tile0, kbi0 = kb0;
     long i = i0;
-    while (i < i1) {
-      const int tile = (int)(i / p.kb), kbi0 = (int)(i % p.kb);
+    for (; i < i1; ++tile, kbi0 = 0) {
       const long seg_end = min(i1, (long)(tile + 1) * p.kb);
       int z, mt, nt;
       tile_coords(tile, z, mt, nt);
