@@ -283,6 +283,9 @@ __global__ void __launch_bounds__(192, 2)
   } else if (warp == 5) {  // ----------------------------------------- MMA issue
     if (lane == 0) {
       const uint32_t idesc = idesc_f16(C::BM, BN, IsBf16<T>::value, A_MN, false);
+      constexpr uint32_t hi = desc_sw128_hi(1024);
+      const uint32_t a_lo0 = desc_sw128_lo(smem_u32(smem), A_MN ? 8192 : 16);
+      const uint32_t b_lo0 = desc_sw128_lo(smem_u32(smem) + C::A_BYTES, 16);
       const int n_it = (int)(i1 - i0);
       int kbi = (int)(i0 % p.kb), seg = 0, s = 0;
       uint32_t ph = 0, acc_col = 0;
@@ -297,13 +300,12 @@ __global__ void __launch_bounds__(192, 2)
         }
         if (!mbar_wait(smem_u32(full + s), ph, abort_flag)) break;
         tc_fence_after();
-        const uint32_t sa = smem_u32(smem + (size_t)s * C::STAGE_BYTES), sb = sa + C::A_BYTES;
+        // descriptor low words of stage s (16-byte units); a K-step is +2 along a K-major row
+        // and +128 (16 rows) down the MN-major A
+        const uint32_t a_lo = a_lo0 + (uint32_t)s * (C::STAGE_BYTES >> 4), b_lo = b_lo0 + (uint32_t)s * (C::STAGE_BYTES >> 4);
+        mma_ss_lohi(tmem + acc_col, a_lo, b_lo, hi, idesc, !first);
 #pragma unroll
-        for (int ks = 0; ks < 4; ++ks) {
-          const uint64_t ad = A_MN ? desc_sw128(sa + ks * 2048, 8192, 1024) : desc_sw128(sa + ks * 32, 16, 1024);
-          const uint64_t bd = desc_sw128(sb + ks * 32, 16, 1024);
-          mma_ss(tmem + acc_col, ad, bd, idesc, !(first && ks == 0));
-        }
+        for (int ks = 1; ks < 4; ++ks) mma_ss_lohi(tmem + acc_col, a_lo + (A_MN ? 128 : 2) * ks, b_lo + 2 * ks, hi, idesc, 1);
         mma_commit(smem_u32(empty + s));
         first = false;
         if (it == n_it - 1 || kbi == p.kb - 1) {

@@ -236,6 +236,7 @@ template <typename T>
 int gemm_sk(const Operand& A, bool a_mn, const Operand& B, int M, int N, int K, const SkPlan& g,
             const tc::EpiParams& epi, float* part, cudaStream_t st, int32_t& n) {
   if (N <= 0 || M <= 0) return MLA_OK;
+  if (g.stages < 2 || g.smem > kSkSmemMax) return MLA_ERR_CUDA;  // no shape of the library reaches this
   constexpr bool bf16 = tc::IsBf16<T>::value;
   CUtensorMap ma, mb;
   const bool ok_a = a_mn ? encode_2d(&ma, A.base, bf16, A.cols, A.rows, A.cols * 2, 64, 64)
