@@ -101,14 +101,14 @@ class ClockSampler:
             rows.append((ts, parts))
         inside = [r for r in rows if t0 <= r[0] <= t1]
         if not inside:
-            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "samples": 0,
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "samples": 0, "samples_under_load": 0,
                     "note": "no nvidia-smi sample fell inside the timed region"}
         sm = [float(p[0]) for _, p in inside if p[0].replace(".", "").isdigit()]
         mx = [float(p[1]) for _, p in inside if p[1].replace(".", "").isdigit()]
         names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
         reasons = sorted({names[i] for _, p in inside for i in range(4) if p[4 + i].lower() == "active"})
         return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": max(mx) if mx else None,
-                "reasons": reasons, "samples": len(inside)}
+                "reasons": reasons, "samples": len(inside), "samples_under_load": len(inside)}
 
 
 # ----------------------------------------------------------------------------------- CPU oracle
@@ -272,6 +272,11 @@ def run_mla(args):
     h = h0.clone()
     attn_call = M.CALL_PREFILL_ATTENTION if chunk > 1 else M.CALL_DECODE_ATTENTION
     calls = (M.CALL_APPEND_KV, M.CALL_ABSORB_QUERY, attn_call, M.CALL_OUT_PROJ)
+    fused = args.fused
+    if fused and (chunk > 1 or not M.layer_step_small_supported(d)):
+        raise SystemExit(f"--fused: workload {w.name} is not a decode step with small-head dims")
+    if fused:
+        calls = (M.CALL_LAYER_STEP_SMALL,)
     ws = torch.empty(max(M.workspace_size(d, c, T, ix.max_seq_len) for c in calls), dtype=torch.uint8, device=dev)
     # per-step index input besides the positions: the attended lengths (decode) or each new
     # token's sequence (prefill)
@@ -290,6 +295,20 @@ def run_mla(args):
     def one_step(record=False, inp=None, outs_=None):
         x, pos, aux = inp if inp is not None else (h, ix.pos, aux0)
         seq_idx = aux if chunk > 1 else ix.seq_idx
+        if fused:  # the whole layer step in one launch (mla_layer_step_small)
+            for L, o in zip(layers, outs if outs_ is None else outs_):
+                if record:
+                    ev = [EV() for _ in range(5)]
+                    ev[0].record(stream)
+                M.layer_step_small(L.state, x, aux, ix.max_seq_len, ws=ws, out=o, stream=stream)
+                if record:
+                    for k in range(1, 5):
+                        ev[k].record(stream)
+                    pending.append(ev)
+                launches[0] += M.last_launch_count(M.CALL_LAYER_STEP_SMALL)
+                if len(layers) > 1:
+                    x = x + o["u"]
+            return o["u"]
         for L, o in zip(layers, outs if outs_ is None else outs_):
             st, w_ = L.state, L.state.w
             if record:
@@ -409,6 +428,9 @@ def run_mla(args):
     n_layer_steps = args.steps * len(layers)
     call_ms /= n_layer_steps
     kernel_ms = sum(k0.elapsed_time(k1) for k0, k1 in kernel_events) / n_layer_steps
+    if fused:  # one launch per layer: the call is the kernel
+        kernel_ms = call_ms[0]
+        call_ms[2] = call_ms[0]
 
     # ---- e2e: host buffers through the public API (pinned h in, u out, inside the timed region)
     h_host = h0.cpu().pin_memory()
@@ -476,6 +498,8 @@ def run_mla(args):
         us_e2e_job = job_us_per_layer_step(ms_e2e, args.steps, len(layers), world)
         dbytes, dflops = harness.attention_work(d, cached, chunk)
         sbytes, sflops = harness.layer_work(d, cached, chunk)
+        if fused:  # the fused kernel does the whole layer: its roofline is the layer's
+            dbytes, dflops = sbytes, sflops
         dec_s = decode_ms * 1e-3    # the whole call: planner + attention kernel + merge
         ker_s = kernel_ms * 1e-3    # the attention kernel alone (events around its launch)
         t_mem = dbytes / (peaks["hbm_gbs"] * 1e9)
@@ -490,9 +514,10 @@ def run_mla(args):
         roof["frac"] = roof["achieved"] / roof["peak"]
         roof["frac_whole_call"] = call_frac  # counting the planner and merge launches too
         roof["traffic"] = measured_decode_traffic(w.name)
-        roof["kernel"] = ("attention kernel of mla_prefill_attention (k_decode_tc, one item per new token)" if chunk > 1
-                          else "attention kernel of mla_decode_attention (k_decode_tc; CUDA-core k_decode_simt at "
-                               "small n_h)")
+        roof["kernel"] = ("k_layer_small (mla_layer_step_small: the whole layer step in one launch)" if fused
+                          else "attention kernel of mla_prefill_attention (k_decode_tc, one item per new token)"
+                          if chunk > 1 else "attention kernel of mla_decode_attention (k_decode_tc; warp-MMA "
+                                            "k_decode_mma at small n_h)")
         roof["kernel_us"] = kernel_ms * 1e3
         roof["peak_source"] = peak_src + " (burst; MEASURED_PEAKS.json)" if peak_src == "measured" else peak_src
         roof["roofline_us"] = max(t_mem, t_flop) * 1e6
@@ -508,6 +533,8 @@ def run_mla(args):
                                                                          f"{int(cached.sum())}"),
                        "layers": len(layers), "dims": dims_desc(d), "paging": w.paging,
                        **({"chunk": chunk, "new_tokens": T} if chunk > 1 else {}),
+                       "path": ("one launch per layer (mla_layer_step_small)" if fused else
+                                "four C-ABI calls per layer"),
                        "l2": ("flushed before every step (256 MiB write, outside the step's events)" if args.flush_l2
                               else "inputs larger than L2" if sbytes > 126e6 else "L2 not flushed (inputs below L2)"),
                        "parallelism": f"replicas x{world} (sequence-independent, no collective)",
@@ -519,9 +546,10 @@ def run_mla(args):
             "cache_gbs": dbytes / dec_s / 1e9,
             "decode_us": decode_ms * 1e3,
             "decode_kernel_us": kernel_ms * 1e3,
-            "per_call_us": {"append_kv": call_ms[0] * 1e3, "absorb_query": call_ms[1] * 1e3,
-                            ("prefill_attention" if chunk > 1 else "decode_attention"): call_ms[2] * 1e3,
-                            "out_proj": call_ms[3] * 1e3},
+            "per_call_us": ({"layer_step_small": call_ms[0] * 1e3} if fused else
+                            {"append_kv": call_ms[0] * 1e3, "absorb_query": call_ms[1] * 1e3,
+                             ("prefill_attention" if chunk > 1 else "decode_attention"): call_ms[2] * 1e3,
+                             "out_proj": call_ms[3] * 1e3}),
             "layer_step_roofline_us": max(sbytes / (peaks["hbm_gbs"] * 1e9), sflops / (peaks["bf16_tflops"] * 1e12))
             * 1e6,
             "roofline": roof,
@@ -543,7 +571,7 @@ def run_mla(args):
 def main():
     ap = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawDescriptionHelpFormatter)
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--steps", type=int, default=200)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--workload", default=DEFAULT_WORKLOAD)
     ap.add_argument("--impl", choices=["mla", "reference"], default="mla")
@@ -552,6 +580,8 @@ def main():
                     help="repeat the K-step timed region until this many seconds are timed (at least 3 times)")
     ap.add_argument("--max-reps", type=int, default=1000)
     ap.add_argument("--flush-l2", action="store_true", help="write 256 MiB before every timed step (cold L2)")
+    ap.add_argument("--fused", action="store_true",
+                    help="small-head decode workloads: the whole layer step in one launch (mla_layer_step_small)")
     args = ap.parse_args()
     args.warmup = max(3, args.warmup)     # at least 3 untimed warm-up steps
     if args.impl == "reference":

@@ -91,7 +91,8 @@ enum mla_call {
   MLA_CALL_ABSORB_QUERY = 1,
   MLA_CALL_DECODE_ATTENTION = 2,
   MLA_CALL_OUT_PROJ = 3,
-  MLA_CALL_PREFILL_ATTENTION = 4
+  MLA_CALL_PREFILL_ATTENTION = 4,
+  MLA_CALL_LAYER_STEP_SMALL = 5
 };
 
 /* Returns MLA_OK if every call supports `dims`, else MLA_ERR_UNSUPPORTED_DIMS or
@@ -203,6 +204,34 @@ int mla_out_proj(const mla_dims* dims, const void* o_lat, const void* w_uv, cons
 
 /* Synchronises `stream`, returns the current device's status word in *status_out (MLA_OK or
  * the first device-side error recorded since the last read) and clears it. */
+/*
+ * mla_layer_step_small — one decode step of one layer (the four calls above for one new token per
+ * sequence: mla_append_kv, mla_absorb_query, mla_decode_attention, mla_out_proj) in a single
+ * cooperative launch, for small head counts such as the running model of the from-scratch page
+ * (§6: 8 heads, d_c = 128, d_h^R = 32). Where the four-call path is bound by its launches, the
+ * phases here meet at grid-wide barriers instead.
+ * Sequence b's new token sits at position seq_lens[b] - 1 (its row is computed, written to the
+ * cache, and attended by the token itself); h [B, d_model]; the weights as in the four calls
+ * (w_dkv_kr [d_c + d_rope, d_model], w_dq [d_cq, d_model], w_uq_qr [n_h*(d_h + d_rope), d_cq],
+ * w_uk and w_uv [n_h*d_h, d_c], w_o [d_model, n_h*d_h]); pool, block_table [B, max_pages] and
+ * seq_lens as in mla_decode_attention (sequence b of the block table is batch row b).
+ * Outputs: q_out [B, n_h, d_c + d_rope] (the absorbed query), o_lat [B, n_h, d_c], lse_out
+ * [B, n_h] (or NULL) and u [B, d_model], each as the corresponding call writes it; every
+ * product accumulates in fp32 and rounds where that call stores, so the two paths agree to
+ * rounding. ws at least mla_workspace_size(dims, MLA_CALL_LAYER_STEP_SMALL, B, max_seq_len)
+ * bytes. Supported dims: mla_layer_step_small_supported. 0 <= B <= 65535, B == 0 is a no-op.
+ * A bad sequence length or page id is recorded in the device status as in the four calls (the
+ * row is not written; the output is zero).
+ */
+int mla_layer_step_small_supported(const mla_dims* dims); /* MLA_OK or MLA_ERR_UNSUPPORTED_DIMS:
+  n_heads <= 16, d_c + d_rope <= 192 and a multiple of 16, d_c <= 128 and a multiple of 16,
+  page_size a multiple of 16, d_model, d_cq and n_heads*d_head multiples of 8. */
+int mla_layer_step_small(const mla_dims* dims, const void* h, const void* w_dkv_kr, const void* w_dq,
+                         const void* w_uq_qr, const void* w_uk, const void* w_uv, const void* w_o, void* pool,
+                         int32_t num_pages, const int32_t* block_table, int32_t max_pages, const int32_t* seq_lens,
+                         int32_t B, int32_t max_seq_len, void* q_out, void* o_lat, float* lse_out, void* u, void* ws,
+                         size_t ws_bytes, mla_stream_t stream);
+
 int mla_read_device_status(mla_stream_t stream, int32_t* status_out);
 
 /* Static string for a status code. */

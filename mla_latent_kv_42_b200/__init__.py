@@ -17,11 +17,14 @@ from dataclasses import dataclass
 __all__ = [
     "MLAError", "load_library", "library_path", "c_dims", "workspace_size", "cache_elems_per_token",
     "append_kv", "absorb_query", "decode_attention", "decode_attention_noalloc", "prefill_attention", "out_proj",
-    "read_device_status", "last_launch_count", "LayerState", "layer_step",
+    "read_device_status", "last_launch_count", "LayerState", "layer_step", "layer_step_small",
+    "layer_step_small_supported",
     "CALL_APPEND_KV", "CALL_ABSORB_QUERY", "CALL_DECODE_ATTENTION", "CALL_OUT_PROJ", "CALL_PREFILL_ATTENTION",
+    "CALL_LAYER_STEP_SMALL",
 ]
 
 CALL_APPEND_KV, CALL_ABSORB_QUERY, CALL_DECODE_ATTENTION, CALL_OUT_PROJ, CALL_PREFILL_ATTENTION = 0, 1, 2, 3, 4
+CALL_LAYER_STEP_SMALL = 5
 _PKG = os.path.dirname(os.path.abspath(__file__))
 
 
@@ -60,6 +63,9 @@ _SIGS = {
     "mla_decode_attention_noalloc": (ctypes.c_int, [_P, _P, _P, _I32, _P, _I32, _P, _I32, _I32, _P, _P, _P]),
     "mla_set_decode_timing_events": (ctypes.c_int, [_P, _P]),
     "mla_debug_inject_missing_load": (ctypes.c_int, [_I32]),
+    "mla_layer_step_small_supported": (ctypes.c_int, [_P]),
+    "mla_layer_step_small": (ctypes.c_int, [_P, _P, _P, _P, _P, _P, _P, _P, _P, _I32, _P, _I32, _P, _I32, _I32, _P, _P,
+                                            _P, _P, _P, _SZ, _P]),
 }
 
 
@@ -337,6 +343,44 @@ def layer_step(st: LayerState, h, pos, seq_idx, seq_lens, max_seq_len, ws=None, 
     o_lat, lse = decode_attention(d, q, st.pool, st.block_table, seq_lens, max_seq_len, o_lat=out.get("o_lat"),
                                   lse=out.get("lse"), want_lse=out.get("want_lse", True), ws=ws, stream=stream)
     u = out_proj(d, o_lat, w["w_uv"], w["w_o"], u=out.get("u"), ws=ws, stream=stream)
+    return u, q, o_lat, lse
+
+
+def layer_step_small_supported(dims) -> bool:
+    cd = c_dims(dims)
+    return _lib().mla_layer_step_small_supported(ctypes.byref(cd)) == 0
+
+
+def layer_step_small(st: LayerState, h, seq_lens, max_seq_len, ws=None, out=None, stream=None):
+    """mla_layer_step_small: the same decode step as ``layer_step`` (one new token per sequence,
+    sequence b = batch row b, new token at position seq_lens[b] - 1) in one launch, for small head
+    counts; returns (u, q, o_lat, lse)."""
+    import torch
+    d, w = st.dims, st.w
+    out = out or {}
+    e = _elem(d)
+    B = h.shape[0]
+    dev = h.device
+    q = out.get("q")
+    if q is None:
+        q = torch.empty((B, d.n_heads, d.d_c + d.d_rope), dtype=e, device=dev)
+    o_lat = out.get("o_lat")
+    if o_lat is None:
+        o_lat = torch.empty((B, d.n_heads, d.d_c), dtype=e, device=dev)
+    lse = out.get("lse")
+    if lse is None and out.get("want_lse", True):
+        lse = torch.empty((B, d.n_heads), dtype=torch.float32, device=dev)
+    u = out.get("u")
+    if u is None:
+        u = torch.empty((B, d.d_model), dtype=e, device=dev)
+    ws, nbytes = _ws(d, CALL_LAYER_STEP_SMALL, B, max_seq_len, ws, dev)
+    cd = c_dims(d)
+    pool, bt = st.pool, st.block_table
+    _check(_lib().mla_layer_step_small(ctypes.byref(cd), _ptr(h), _ptr(w["w_dkv_kr"]), _ptr(w["w_dq"]),
+                                       _ptr(w["w_uq_qr"]), _ptr(w["w_uk"]), _ptr(w["w_uv"]), _ptr(w["w_o"]),
+                                       _ptr(pool), pool.shape[0], _ptr(bt), bt.shape[1], _ptr(seq_lens), B,
+                                       max_seq_len, _ptr(q), _ptr(o_lat), _ptr(lse), _ptr(u), _ptr(ws), nbytes,
+                                       _stream(stream)), "mla_layer_step_small")
     return u, q, o_lat, lse
 
 

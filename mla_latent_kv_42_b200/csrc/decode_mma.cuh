@@ -127,7 +127,8 @@ __device__ void attn_mma_item(const MmaAttnArgs& a, int b, int split, uint8_t* s
       for (int e = 0; e < 4; ++e) {
         const int row = g + ((e & 1) ? 8 : 0), col = 16 * ks + 2 * tq + ((e & 2) ? 8 : 0);
         uint32_t v = 0;
-        if (ks < KD && row < n_h) v = *reinterpret_cast<const uint32_t*>(qb + (long)row * D + col);
+        // read at L2: the fused layer step writes q earlier in the same launch
+        if (ks < KD && row < n_h) v = __ldcg(reinterpret_cast<const unsigned*>(qb + (long)row * D + col));
         qa[ks][e] = v;
       }
     }

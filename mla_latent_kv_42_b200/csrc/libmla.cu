@@ -15,6 +15,7 @@
 #include "decode_mma.cuh"
 #include "decode_simt.cuh"
 #include "decode_tc.cuh"
+#include "layer_small.cuh"
 #include "prefill.cuh"
 #include "proj_host.cuh"
 
@@ -31,7 +32,7 @@ struct NvtxRange {
   NvtxRange& operator=(const NvtxRange&) = delete;
 };
 
-thread_local int32_t t_launches[5] = {0, 0, 0, 0, 0};
+thread_local int32_t t_launches[6] = {0, 0, 0, 0, 0, 0};
 // Profiling hook: events recorded around the attention kernel of this thread's decode calls.
 thread_local cudaEvent_t t_ev_before = nullptr, t_ev_after = nullptr;
 inline void mark_before(cudaStream_t st) {
@@ -431,6 +432,125 @@ int out_impl(const mla_dims* d, const void* o_lat, const void* w_uv, const void*
 
 }  // namespace
 
+// ------------------------------------------------------------------ fused small-head layer step
+bool layer_small_eligible(const mla_dims* d) {
+  return decode_mma_eligible(d) && d->d_model % 8 == 0 && d->d_cq % 8 == 0 && (d->n_heads * d->d_head) % 8 == 0;
+}
+
+struct SmallLayout {
+  DecodePlan p;
+  size_t cq, qc, o, o_part, lse_part, bytes;
+};
+// Attention split over `ctas` CTAs of the fused kernel: about one (sequence, split) item per CTA,
+// each a whole number of 64-token stages.
+DecodePlan plan_small(int B, int max_seq_len, long ctas) {
+  DecodePlan p;
+  p.head_groups = 1;
+  const long stages = ((long)max_seq_len + dmma::kStageTokens - 1) / dmma::kStageTokens;
+  long s = std::max(1L, ctas / B);
+  if (s > stages) s = stages;
+  const long per = (stages + s - 1) / s;
+  p.split_len = (int)(per * dmma::kStageTokens);
+  p.n_splits = (int)(((long)max_seq_len + p.split_len - 1) / p.split_len);
+  return p;
+}
+// ctas: the grid the call launches (the workspace query assumes the largest, 3 per SM)
+SmallLayout small_layout(const mla_dims* d, int B, int max_seq_len, long ctas) {
+  SmallLayout L;
+  L.p = plan_small(B, max_seq_len, ctas);
+  const size_t e = 2, nq = (size_t)d->n_heads * d->d_head, bh = (size_t)B * d->n_heads;
+  L.cq = 0;
+  L.qc = L.cq + align256((size_t)B * d->d_cq * e);
+  L.o = L.qc + align256((size_t)B * nq * e);
+  L.o_part = L.o + align256((size_t)B * nq * e);
+  L.lse_part = L.o_part + (L.p.n_splits > 1 ? align256(bh * L.p.n_splits * d->d_c * 4) : 0);
+  L.bytes = L.lse_part + (L.p.n_splits > 1 ? align256(bh * L.p.n_splits * 4) : 0);
+  return L;
+}
+size_t ws_layer_small(const mla_dims* d, int B, int max_seq_len) {
+  if (B <= 0 || max_seq_len < 1 || max_seq_len > kMaxSeqLen || !layer_small_eligible(d)) return 0;
+  // the most splits any grid of the call gives: the smallest grid (one CTA per SM)
+  size_t most = 0;
+  for (int per_sm = 1; per_sm <= 3; ++per_sm)
+    most = std::max(most, small_layout(d, B, max_seq_len, (long)per_sm * device_sm_count()).bytes);
+  return most;
+}
+
+template <typename T>
+int layer_small_impl(const mla_dims* d, const void* h, const void* w_dkv_kr, const void* w_dq, const void* w_uq_qr,
+                     const void* w_uk, const void* w_uv, const void* w_o, void* pool, int32_t num_pages,
+                     const int32_t* bt, int32_t max_pages, const int32_t* seq_lens, int32_t B, int32_t max_seq_len,
+                     void* q_out, void* o_lat, float* lse_out, void* u, void* ws, cudaStream_t st) {
+  const int D = d->d_c + d->d_rope;
+  const size_t smem = dmma::smem_bytes(D);
+  // resident CTAs per SM for this row width (the cooperative grid must fit at once), cached per
+  // device and width (D / 16 <= kMaxKD)
+  static std::atomic<int> blocks_per_sm[kMaxDevices][dmma::kMaxKD + 1];
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return MLA_ERR_CUDA;
+  int bps = blocks_per_sm[dev][D / 16].load(std::memory_order_acquire);
+  if (bps == 0) {
+    // the largest row the kernel takes, so that one setting serves every eligible shape
+    if (cudaFuncSetAttribute(k_layer_small<T>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             (int)dmma::smem_bytes(16 * dmma::kMaxKD)) != cudaSuccess)
+      return MLA_ERR_CUDA;
+    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&bps, k_layer_small<T>, 128, smem) != cudaSuccess || bps < 1)
+      return MLA_ERR_CUDA;
+    blocks_per_sm[dev][D / 16].store(bps, std::memory_order_release);
+  }
+  // As many CTAs as the largest phase has warp items for (two rows per warp, four warps per CTA),
+  // at least one per SM and at most what fits at once: with little work (one sequence) fewer CTAs
+  // make each grid-wide barrier cheaper.
+  const long nq = (long)d->n_heads * d->d_head, half = d->d_rope / 2;
+  const long warps = std::max({(long)B * (d->d_c + d->d_cq) / 2 + (long)B * half, (long)B * nq / 2 + (long)B * d->n_heads * half,
+                               (long)B * d->d_model / 2});
+  const int grid = (int)std::max<long>(device_sm_count(),
+                                       std::min<long>((long)std::min(bps, 3) * device_sm_count(), (warps + 3) / 4));
+  // attention items (sequence, split) for one round over the grid
+  SmallLayout L = small_layout(d, B, max_seq_len, grid);
+  char* w = static_cast<char*>(ws);
+  SmallStepArgs a;
+  a.B = B;
+  a.h = h;
+  a.w_dkv_kr = w_dkv_kr;
+  a.w_dq = w_dq;
+  a.w_uq_qr = w_uq_qr;
+  a.w_uk = w_uk;
+  a.w_uv = w_uv;
+  a.w_o = w_o;
+  a.d_model = d->d_model;
+  a.n_h = d->n_heads;
+  a.d_h = d->d_head;
+  a.d_c = d->d_c;
+  a.d_cq = d->d_cq;
+  a.d_rope = d->d_rope;
+  a.rope_base = d->rope_base;
+  a.rope_table = d->rope_inv_freq;
+  a.pool = pool;
+  a.cq = w + L.cq;
+  a.qc = w + L.qc;
+  a.q = q_out;
+  a.o = w + L.o;
+  a.u = u;
+  const float scale_log2 = (float)(1.0 / std::sqrt((double)(d->d_head + d->d_rope)) * 1.4426950408889634);
+  a.attn = MmaAttnArgs{q_out, pool, bt, (int)max_pages, seq_lens, (int)max_seq_len, (int)num_pages, (int)d->n_heads,
+                       (int)d->d_c, D, (int)d->page_size, scale_log2, L.p.split_len, L.p.n_splits, o_lat, lse_out,
+                       L.p.n_splits > 1 ? reinterpret_cast<float*>(w + L.o_part) : nullptr,
+                       L.p.n_splits > 1 ? reinterpret_cast<float*>(w + L.lse_part) : nullptr};
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(grid);
+  cfg.blockDim = dim3(128);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeCooperative;
+  attr[0].val.cooperative = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  if (cudaLaunchKernelEx(&cfg, k_layer_small<T>, a) != cudaSuccess) return MLA_ERR_CUDA;
+  return finish_launches(MLA_CALL_LAYER_STEP_SMALL, 1);
+}
+
 extern "C" {
 
 int mla_check_dims(const mla_dims* dims) { return check_dims_impl(dims); }
@@ -449,6 +569,7 @@ size_t mla_workspace_size(const mla_dims* dims, int32_t call, int32_t B, int32_t
     case MLA_CALL_DECODE_ATTENTION: return ws_decode(dims, B, max_seq_len);
     case MLA_CALL_OUT_PROJ: return ws_out(dims, B);
     case MLA_CALL_PREFILL_ATTENTION: return ws_prefill(dims, B, max_seq_len);
+    case MLA_CALL_LAYER_STEP_SMALL: return ws_layer_small(dims, B, max_seq_len);
     default: return 0;
   }
 }
@@ -574,6 +695,44 @@ int mla_out_proj(const mla_dims* dims, const void* o_lat, const void* w_uv, cons
   return out_impl<__half>(dims, o_lat, w_uv, w_o, u, B, ws, st);
 }
 
+int mla_layer_step_small_supported(const mla_dims* dims) {
+  const int r = check_dims_impl(dims);
+  if (r != MLA_OK) return r;
+  return layer_small_eligible(dims) ? MLA_OK : MLA_ERR_UNSUPPORTED_DIMS;
+}
+
+int mla_layer_step_small(const mla_dims* dims, const void* h, const void* w_dkv_kr, const void* w_dq,
+                         const void* w_uq_qr, const void* w_uk, const void* w_uv, const void* w_o, void* pool,
+                         int32_t num_pages, const int32_t* block_table, int32_t max_pages, const int32_t* seq_lens,
+                         int32_t B, int32_t max_seq_len, void* q_out, void* o_lat, float* lse_out, void* u, void* ws,
+                         size_t ws_bytes, mla_stream_t stream) {
+  NvtxRange nvtx_range("mla_layer_step_small");
+  int r = mla_layer_step_small_supported(dims);
+  if (r != MLA_OK) return r;
+  if (B < 0 || B > 65535 || num_pages < 0 || max_pages < 1 || max_seq_len < 1 || max_seq_len > kMaxSeqLen)
+    return MLA_ERR_INVALID_ARG;
+  if (B == 0) {
+    t_launches[MLA_CALL_LAYER_STEP_SMALL] = 0;
+    return MLA_OK;
+  }
+  if (!page_total_fits(dims, B, max_seq_len)) return MLA_ERR_INVALID_ARG;
+  if (!h || !w_dkv_kr || !w_dq || !w_uq_qr || !w_uk || !w_uv || !w_o || !pool || !block_table || !seq_lens ||
+      !q_out || !o_lat || !u || !ws)
+    return MLA_ERR_INVALID_ARG;
+  if (!aligned16(h) || !aligned16(w_dkv_kr) || !aligned16(w_dq) || !aligned16(w_uq_qr) || !aligned16(w_uk) ||
+      !aligned16(w_uv) || !aligned16(w_o) || !aligned16(pool) || !aligned16(q_out) || !aligned16(o_lat) ||
+      !aligned16(u) || !aligned16(ws))
+    return MLA_ERR_ALIGNMENT;
+  if (ws_bytes < ws_layer_small(dims, B, max_seq_len)) return MLA_ERR_WORKSPACE_TOO_SMALL;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  if (dims->dtype == MLA_BF16)
+    return layer_small_impl<__nv_bfloat16>(dims, h, w_dkv_kr, w_dq, w_uq_qr, w_uk, w_uv, w_o, pool, num_pages,
+                                           block_table, max_pages, seq_lens, B, max_seq_len, q_out, o_lat, lse_out, u,
+                                           ws, st);
+  return layer_small_impl<__half>(dims, h, w_dkv_kr, w_dq, w_uq_qr, w_uk, w_uv, w_o, pool, num_pages, block_table,
+                                  max_pages, seq_lens, B, max_seq_len, q_out, o_lat, lse_out, u, ws, st);
+}
+
 int mla_read_device_status(mla_stream_t stream, int32_t* status_out) {
   if (!status_out) return MLA_ERR_INVALID_ARG;
   if (cudaStreamSynchronize(reinterpret_cast<cudaStream_t>(stream)) != cudaSuccess) return MLA_ERR_CUDA;
@@ -600,7 +759,7 @@ const char* mla_error_string(int code) {
   }
 }
 
-int32_t mla_last_launch_count(int32_t call) { return (call >= 0 && call < 5) ? t_launches[call] : -1; }
+int32_t mla_last_launch_count(int32_t call) { return (call >= 0 && call < 6) ? t_launches[call] : -1; }
 
 int mla_debug_gemm_plan(int32_t M, int32_t N, int32_t K, int32_t batch, int32_t fused_rope, int32_t d_rope,
                         int64_t* out) {

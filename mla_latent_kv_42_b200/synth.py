@@ -87,6 +87,8 @@ WORKLOADS = {
         Workload("production_b128_ragged_paged_bf16", PRODUCTION, 128, (512, 32768), 1, 0.006, "shuffled"),
         Workload("production_b4_n131072_bf16", PRODUCTION, 4, 131072, 1, 0.006, "contiguous"),
         Workload("production_b8_n4096_chunk128_bf16", PRODUCTION, 8, 4096, 1, 0.006, "contiguous", chunk=128),
+        # chunked prefill over a prefix larger than L2 (64 x 4096 cached rows = 302 MB)
+        Workload("production_b64_n4096_chunk32_bf16", PRODUCTION, 64, 4096, 1, 0.006, "contiguous", chunk=32),
     ]
 }
 
