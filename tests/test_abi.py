@@ -178,7 +178,41 @@ def test_prefill_argument_errors_queue_nothing(lib):
     assert call(a14=16) == -3                             # too-small workspace
     assert call(a9=0, a1=None, a13=None) == 0             # T == 0 is a no-op
     assert lib.mla_last_launch_count(M.CALL_PREFILL_ATTENTION) == 0
-    assert lib.mla_last_launch_count(5) == -1
+    assert lib.mla_last_launch_count(6) == -1
+
+
+def test_layer_step_small_argument_errors_queue_nothing(lib):
+    """The fused single-launch layer step: argument checks return before anything is queued."""
+    assert lib.mla_layer_step_small_supported(ctypes.byref(dims(synth.RUNNING))) == 0
+    assert lib.mla_layer_step_small_supported(ctypes.byref(dims(synth.PRODUCTION))) == -2
+    cd = dims(synth.RUNNING)
+    ws_need = lib.mla_workspace_size(ctypes.byref(cd), M.CALL_LAYER_STEP_SMALL, 4, 300)
+    assert ws_need > 0
+    assert lib.mla_workspace_size(ctypes.byref(cd), M.CALL_LAYER_STEP_SMALL, 4, (1 << 30) + 1) == 0
+    assert lib.mla_workspace_size(ctypes.byref(dims(synth.PRODUCTION)), M.CALL_LAYER_STEP_SMALL, 4, 300) == 0
+    f = lib.mla_layer_step_small
+    # dims, h, w_dkv_kr, w_dq, w_uq_qr, w_uk, w_uv, w_o, pool, num_pages, block_table, max_pages,
+    # seq_lens, B, max_seq_len, q_out, o_lat, lse_out, u, ws, ws_bytes, stream
+    args = [ctypes.byref(cd), FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, 100, FAKE, 8, FAKE, 4, 300, FAKE,
+            FAKE, None, FAKE, FAKE, ws_need, None]
+
+    def call(**kw):
+        a = list(args)
+        for k, v in kw.items():
+            a[int(k[1:])] = v
+        return f(*a)
+
+    assert call(a0=ctypes.byref(dims(synth.PRODUCTION))) == -2  # dims outside the fused kernel
+    assert call(a1=None) == -1                            # null h
+    assert call(a8=None) == -1                            # null pool
+    assert call(a19=None) == -1                           # null workspace
+    assert call(a16=MISALIGNED) == -4                     # misaligned o_lat
+    assert call(a13=-1) == -1                             # negative batch
+    assert call(a14=0) == -1                              # max_seq_len < 1
+    assert call(a14=(1 << 30) + 1) == -1                  # max_seq_len beyond 2^30
+    assert call(a20=ws_need - 1) == -3                    # too-small workspace
+    assert call(a13=0, a1=None) == 0                      # B == 0 is a no-op
+    assert lib.mla_last_launch_count(M.CALL_LAYER_STEP_SMALL) == 0
 
 
 def test_prefill_workspace_covers_decode_and_stops_growing():
