@@ -95,9 +95,9 @@ __global__ void __launch_bounds__(256) k_decode_simt(
 }
 
 // Merge of split-KV partials: o = sum_s w_s o_s / sum_s w_s with w_s = e^{lse_s - max lse},
-// summed in split order. One warp per (b, head), lanes over the latent columns (d_c <= 512, a
-// multiple of 8), every split's loads in flight together; grid ceil(B n_h / 8), 256 threads.
-// o_part [BH][S][d_c], lse_part [BH][S].
+// summed in split order. One warp per (b, head), grid ceil(B n_h / 8), 256 threads; lane l takes
+// columns 4l + 128q (d_c a multiple of 4, <= 512). Lane s holds w_s (splits past 32 recompute it);
+// each lane keeps eight partial rows' loads in flight. o_part [BH][S][d_c], lse_part [BH][S].
 template <typename T>
 __global__ void __launch_bounds__(256) k_lse_merge_warp(const float* __restrict__ o_part,
                                                          const float* __restrict__ lse_part, int n_splits, int d_c,
@@ -108,32 +108,42 @@ __global__ void __launch_bounds__(256) k_lse_merge_warp(const float* __restrict_
   const int lane = threadIdx.x & 31;
   if (bh >= BH) return;
   const float* lp = lse_part + bh * n_splits;
-  float mx = -INFINITY;
-  for (int s = lane; s < n_splits; s += 32) mx = fmaxf(mx, lp[s]);
+  const float l_lane = lane < n_splits ? lp[lane] : -INFINITY;
+  float mx = l_lane;
+  for (int s = lane + 32; s < n_splits; s += 32) mx = fmaxf(mx, lp[s]);
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
-  float acc[16];
+  auto weight = [&](float l) { return l > -INFINITY ? exp2f((l - mx) * kLog2e) : 0.f; };  // -inf: no tokens
+  const float w_lane = weight(l_lane);
+  float z = w_lane;
+  for (int s = lane + 32; s < n_splits; s += 32) z += weight(lp[s]);
 #pragma unroll
-  for (int j = 0; j < 16; ++j) acc[j] = 0.f;
-  float z = 0.f;
-  if (mx != -INFINITY) {
-#pragma unroll 4
-    for (int s = 0; s < n_splits; ++s) {
-      const float w = exp2f((lp[s] - mx) * kLog2e);  // -inf partials (no tokens) weigh 0
-      z += w;
-      const float* src = o_part + (bh * n_splits + s) * d_c;
+  for (int o = 16; o > 0; o >>= 1) z += __shfl_xor_sync(0xffffffffu, z, o);
+  const float inv = z > 0.f ? 1.f / z : 0.f;
+  const float* src0 = o_part + bh * n_splits * d_c;
+  for (int c = 4 * lane; c < d_c; c += 128) {
+    float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+    for (int s0 = 0; s0 < n_splits; s0 += 8) {
+      float4 v[8];
 #pragma unroll
-      for (int j = 0; j < 16; ++j) {
-        const int e = lane + 32 * j;
-        if (e < d_c) acc[j] = fmaf(w, src[e], acc[j]);
+      for (int u = 0; u < 8; ++u)
+        v[u] = s0 + u < n_splits ? *reinterpret_cast<const float4*>(src0 + (long)(s0 + u) * d_c + c)
+                                 : make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+      for (int u = 0; u < 8; ++u) {
+        const int s = s0 + u;
+        const float w = s < 32 ? __shfl_sync(0xffffffffu, w_lane, s & 31) : (s < n_splits ? weight(lp[s]) : 0.f);
+        acc.x = fmaf(w, v[u].x, acc.x);
+        acc.y = fmaf(w, v[u].y, acc.y);
+        acc.z = fmaf(w, v[u].z, acc.z);
+        acc.w = fmaf(w, v[u].w, acc.w);
       }
     }
-  }
-  const float inv = z > 0.f ? 1.f / z : 0.f;
-#pragma unroll
-  for (int j = 0; j < 16; ++j) {
-    const int e = lane + 32 * j;
-    if (e < d_c) Out<T>::put(o_lat + bh * d_c + e, acc[j] * inv);
+    T* out = o_lat + bh * d_c + c;
+    Out<T>::put(out, acc.x * inv);
+    Out<T>::put(out + 1, acc.y * inv);
+    Out<T>::put(out + 2, acc.z * inv);
+    Out<T>::put(out + 3, acc.w * inv);
   }
   if (lse_out != nullptr && lane == 0) lse_out[bh] = z > 0.f ? mx + logf(z) : -INFINITY;
 }
