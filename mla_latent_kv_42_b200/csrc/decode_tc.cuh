@@ -602,18 +602,26 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(dec::kThreads, 1)
           const bool whole = it.t0 == 0 && it.t1 == it.n_b;
           const long slot = (long)it.b + cluster;
           const int col0 = 256 * ch + 128 * g;  // latent columns [col0, col0 + 128)
-          // The warp writes its 32 heads x 128 columns in rounds of 64 bytes per head through its
-          // own 2 KB of the P buffer (free: the last O MMAs are done): each lane puts its head's
-          // segment in row `lane` in the 64-byte swizzle (16-byte chunk c of row r at c ^ (r/2 % 4),
-          // conflict-free), and lane 0 stores the 32 x 64-byte box with one TMA store, which heads
-          // past n_h fall outside of. The warp goes on while the copy engine reads the box.
-          uint8_t* const stage = data + kPOff + warp * 2048;
-          const uint32_t stage_u32 = data_u32 + kPOff + warp * 2048;
+          // The warp writes its 32 heads x 128 columns in rounds of 64 bytes per head through
+          // shared memory: each lane puts its head's segment in row `lane` of a 2 KB box in the
+          // 64-byte swizzle (16-byte chunk c of row r at c ^ (r/2 % 4), conflict-free), and lane 0
+          // stores the 32 x 64-byte box with one TMA store, which heads past n_h fall outside of.
+          // Mid-range the box is the warp's 2 KB of the P buffer (free: the last O MMAs are done),
+          // reused once the copy engine has read it; at the pair's last item every round gets a
+          // box of its own in the latent sets, which no tile needs any more, so nothing waits.
+          const bool last_item = c.it.g >= c.it.g_end;
           const uint32_t wsw = (lane >> 1) & 3;
           const int head0 = 64 * (int)rank + 32 * (qd & 1);
+          int round = 0;
           auto stage_store = [&](const uint32_t (&w)[16], int col) {
-            if (lane == 0) bulk_wait_read<0>();  // the previous round's box has been read
-            __syncwarp();
+            const uint32_t stage_u32 =
+                last_item ? set_u32 + warp * 16384 + round * 2048 : data_u32 + kPOff + warp * 2048;
+            uint8_t* const stage = data + (stage_u32 - data_u32);
+            ++round;
+            if (!last_item) {
+              if (lane == 0) bulk_wait_read<0>();  // the previous round's box has been read
+              __syncwarp();
+            }
 #pragma unroll
             for (int i2 = 0; i2 < 4; ++i2)
               *reinterpret_cast<uint4*>(stage + lane * 64 + ((i2 ^ wsw) << 4)) =
@@ -656,12 +664,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(dec::kThreads, 1)
               p.lse_part[slot * p.n_h + head] = lse;
             }
           }
-          // the boxes have left the P buffer before the next tile's softmax writes it; at the
-          // pair's last item they are also complete in global memory before the CTA exits
-          if (lane == 0) {
-            if (c.it.g >= c.it.g_end) bulk_wait<0>();
-            else bulk_wait_read<0>();
-          }
+          // the boxes have left shared memory before the next tile's softmax writes P, or before
+          // the CTA exits
+          if (lane == 0) bulk_wait_read<0>();
           __syncwarp();
           tc_fence_before();
           __syncwarp();
