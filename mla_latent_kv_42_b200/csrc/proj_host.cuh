@@ -151,21 +151,25 @@ inline SkPlan plan_sk(int M, int N, int K, int batch, bool fused_epi, int d_rope
   g.tiles = g.m_tiles * g.n_tiles * batch;
   g.iters = (long)g.tiles * g.kb;
   const int sms = sm_count();
-  if (g.kb >= kSkLongTile) {
+  const size_t stage = (size_t)(128 + g.bn) * 64 * 2;
+  const size_t table = fused_epi ? (size_t)g.bn * (d_rope / 2) * 8 + (size_t)g.bn * 8 : 0;
+  const size_t fixed = 1024 + table + 256;
+  // Long tiles, at least one per SM: whole tiles per CTA, two CTAs per SM (half-size rings), so
+  // no tile is split and no reduction launch follows ([W^UQ; W^QR] at decode sizes: 192 tiles of
+  // 24 k blocks).
+  const bool long_many = g.kb >= kSkLongTile && g.tiles >= sms && fixed + 2 * stage <= kSkSmemHalf;
+  if (g.kb >= kSkLongTile && !long_many) {
     g.aligned = false;
     g.G = (int)std::max(1L, std::min((long)sms, g.iters / kSkMinIters));
   } else {
     g.aligned = true;
-    const int per = (g.tiles + sms - 1) / sms;
+    const int per = (g.tiles + (long_many ? 2 : 1) * sms - 1) / ((long_many ? 2 : 1) * sms);
     g.G = (g.tiles + per - 1) / per;
   }
   g.split = false;
   if (!g.aligned)
     for (int c = 1; c < g.G && !g.split; ++c) g.split = (g.iters * c / g.G) % g.kb != 0;
-  const size_t stage = (size_t)(128 + g.bn) * 64 * 2;
-  const size_t table = fused_epi ? (size_t)g.bn * (d_rope / 2) * 8 + (size_t)g.bn * 8 : 0;
-  const size_t fixed = 1024 + table + 256;
-  g.stages = (int)std::min<size_t>(12, (kSkSmemMax - fixed) / stage);
+  g.stages = (int)std::min<size_t>(12, ((long_many ? kSkSmemHalf : kSkSmemMax) - fixed) / stage);
   // Many short tiles (the per-head products): when a CTA's whole range fits a half-size ring,
   // run two CTAs per SM, so that two sets of epilogue warps drain tiles side by side.
   if (g.aligned && g.tiles > sms) {

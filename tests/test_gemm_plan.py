@@ -70,7 +70,9 @@ def check_plan(p, Mr, N, K, batch, fused, d_rope):
     assert p["smem"] <= SMEM_MAX
     if G > SMS:
         assert p["aligned"] and p["smem"] <= SMEM_HALF
-        assert p["stages"] >= start[1] - start[0], "two CTAs per SM only with the whole range resident"
+        # short tiles: the whole range resident; long tiles (>= 16 k blocks, at least one per SM):
+        # whole tiles per CTA through a half-size ring
+        assert p["stages"] >= start[1] - start[0] or kb >= 16, "two CTAs per SM only with the whole range resident"
 
 
 def products(d):
