@@ -92,7 +92,9 @@ enum mla_call {
   MLA_CALL_DECODE_ATTENTION = 2,
   MLA_CALL_OUT_PROJ = 3,
   MLA_CALL_PREFILL_ATTENTION = 4,
-  MLA_CALL_LAYER_STEP_SMALL = 5
+  MLA_CALL_LAYER_STEP_SMALL = 5,
+  MLA_CALL_APPEND_KV_FP8 = 6,
+  MLA_CALL_DECODE_ATTENTION_FP8 = 7
 };
 
 /* Returns MLA_OK if every call supports `dims`, else MLA_ERR_UNSUPPORTED_DIMS or
@@ -231,6 +233,49 @@ int mla_layer_step_small(const mla_dims* dims, const void* h, const void* w_dkv_
                          int32_t num_pages, const int32_t* block_table, int32_t max_pages, const int32_t* seq_lens,
                          int32_t B, int32_t max_seq_len, void* q_out, void* o_lat, float* lse_out, void* u, void* ws,
                          size_t ws_bytes, mla_stream_t stream);
+
+/*
+ * FP8 latent cache (DeepSeek-V2 paper review (velog) §4.2 and the DeepSeek-V2 summary page:
+ * the deployed model quantises its KV cache to about 6 bits per element; the pages give no
+ * format, so this cache takes e4m3 with two float32 scales per token). A page of page_size
+ * tokens is page_size rows of d_c + d_rope e4m3 bytes (token order), then page_size pairs of
+ * float32 scales (s_c, s_r): mla_fp8_page_bytes(dims) = page_size * (d_c + d_rope + 8) bytes.
+ * Row j of a token stands for
+ *   c_j = s_c * e4m3(row[0 .. d_c)),   k^R_j = s_r * e4m3(row[d_c .. d_c + d_rope)),
+ * with s = max|part| / 448 in float32 (1 for an all-zero part) and each byte the nearest e4m3
+ * value (ties to even) of the element-type value divided by s in float32, saturated to +-448.
+ */
+int64_t mla_fp8_page_bytes(const mla_dims* dims); /* negative on invalid dims */
+
+/* MLA_OK if the FP8 calls support `dims`: the DeepSeek-V2 cache shape of the tensor-core decode
+ * (d_c = 512, d_rope = 64, page_size = 64, 65 <= n_heads <= 128), else MLA_ERR_UNSUPPORTED_DIMS. */
+int mla_fp8_supported(const mla_dims* dims);
+
+/*
+ * mla_append_kv_fp8 — mla_append_kv into an FP8 cache: the rows [c ‖ k^R] are computed and
+ * rounded to the element type exactly as mla_append_kv computes them, then quantised as above
+ * and written, with their scales, to the token's slot of `pool` (FP8 pages, num_pages of
+ * mla_fp8_page_bytes each, 16-byte aligned). Arguments, checks and error behaviour as
+ * mla_append_kv; ws at least mla_workspace_size(dims, MLA_CALL_APPEND_KV_FP8, T, 0) bytes.
+ */
+int mla_append_kv_fp8(const mla_dims* dims, const void* h, const void* w_dkv_kr,
+                      const int32_t* seq_idx, const int32_t* pos,
+                      const int32_t* block_table, int32_t num_seqs, int32_t max_pages,
+                      void* pool, int32_t num_pages, int32_t T,
+                      void* ws, size_t ws_bytes, mla_stream_t stream);
+
+/*
+ * mla_decode_attention_fp8 — mla_decode_attention over an FP8 cache: the attention of every
+ * sequence and head over the rows the cache stands for. The bytes are converted to the element
+ * type in shared memory (each value times its token's scale, in float32, rounded once) before
+ * the tensor-core products, which are those of mla_decode_attention. Arguments, outputs,
+ * checks and error behaviour as mla_decode_attention, with pool the FP8 pages; ws at least
+ * mla_workspace_size(dims, MLA_CALL_DECODE_ATTENTION_FP8, B, max_seq_len) bytes.
+ */
+int mla_decode_attention_fp8(const mla_dims* dims, const void* q, const void* pool, int32_t num_pages,
+                             const int32_t* block_table, int32_t max_pages, const int32_t* seq_lens,
+                             int32_t B, int32_t max_seq_len, void* o_lat, float* lse_out,
+                             void* ws, size_t ws_bytes, mla_stream_t stream);
 
 int mla_read_device_status(mla_stream_t stream, int32_t* status_out);
 

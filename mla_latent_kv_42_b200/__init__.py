@@ -18,13 +18,14 @@ __all__ = [
     "MLAError", "load_library", "library_path", "c_dims", "workspace_size", "cache_elems_per_token",
     "append_kv", "absorb_query", "decode_attention", "decode_attention_noalloc", "prefill_attention", "out_proj",
     "read_device_status", "last_launch_count", "LayerState", "layer_step", "layer_step_small",
-    "layer_step_small_supported",
+    "layer_step_small_supported", "fp8_page_bytes", "fp8_supported", "append_kv_fp8", "decode_attention_fp8",
     "CALL_APPEND_KV", "CALL_ABSORB_QUERY", "CALL_DECODE_ATTENTION", "CALL_OUT_PROJ", "CALL_PREFILL_ATTENTION",
-    "CALL_LAYER_STEP_SMALL",
+    "CALL_LAYER_STEP_SMALL", "CALL_APPEND_KV_FP8", "CALL_DECODE_ATTENTION_FP8",
 ]
 
 CALL_APPEND_KV, CALL_ABSORB_QUERY, CALL_DECODE_ATTENTION, CALL_OUT_PROJ, CALL_PREFILL_ATTENTION = 0, 1, 2, 3, 4
 CALL_LAYER_STEP_SMALL = 5
+CALL_APPEND_KV_FP8, CALL_DECODE_ATTENTION_FP8 = 6, 7
 _PKG = os.path.dirname(os.path.abspath(__file__))
 
 
@@ -64,6 +65,10 @@ _SIGS = {
     "mla_set_decode_timing_events": (ctypes.c_int, [_P, _P]),
     "mla_debug_inject_missing_load": (ctypes.c_int, [_I32]),
     "mla_layer_step_small_supported": (ctypes.c_int, [_P]),
+    "mla_fp8_page_bytes": (ctypes.c_int64, [_P]),
+    "mla_fp8_supported": (ctypes.c_int, [_P]),
+    "mla_append_kv_fp8": (ctypes.c_int, [_P, _P, _P, _P, _P, _P, _I32, _I32, _P, _I32, _I32, _P, _SZ, _P]),
+    "mla_decode_attention_fp8": (ctypes.c_int, [_P, _P, _P, _I32, _P, _I32, _P, _I32, _I32, _P, _P, _P, _SZ, _P]),
     "mla_layer_step_small": (ctypes.c_int, [_P, _P, _P, _P, _P, _P, _P, _P, _P, _I32, _P, _I32, _P, _I32, _I32, _P, _P,
                                             _P, _P, _P, _SZ, _P]),
 }
@@ -219,6 +224,64 @@ def decode_attention(dims, q, pool, block_table, seq_lens, max_seq_len, o_lat=No
     _check(_lib().mla_decode_attention(ctypes.byref(cd), _ptr(q), _ptr(pool), pool.shape[0], _ptr(block_table),
                                        block_table.shape[1], _ptr(seq_lens), B, int(max_seq_len), _ptr(o_lat),
                                        _ptr(lse), _ptr(ws), nbytes, _stream(stream)), "mla_decode_attention")
+    return o_lat, lse
+
+
+def fp8_page_bytes(dims) -> int:
+    """Bytes of one FP8 cache page: page_size rows of d_c + d_rope e4m3 bytes, then page_size
+    float32 pairs (s_c, s_r)."""
+    cd = c_dims(dims)
+    return int(_lib().mla_fp8_page_bytes(ctypes.byref(cd)))
+
+
+def fp8_supported(dims) -> bool:
+    cd = c_dims(dims)
+    return _lib().mla_fp8_supported(ctypes.byref(cd)) == 0
+
+
+def append_kv_fp8(dims, h, w_dkv_kr, seq_idx, pos, block_table, pool, ws=None, stream=None):
+    """mla_append_kv_fp8: the rows of mla_append_kv, quantised to e4m3 with two scales per token,
+    into ``pool`` (uint8 [num_pages, fp8_page_bytes(dims)])."""
+    import torch
+    e = _elem(dims)
+    for t, n, dt in ((h, "h", e), (w_dkv_kr, "w_dkv_kr", e), (seq_idx, "seq_idx", torch.int32),
+                     (pos, "pos", torch.int32), (block_table, "block_table", torch.int32), (pool, "pool", torch.uint8)):
+        _need(t, dt, n)
+    if pool.dim() != 2 or pool.shape[1] != fp8_page_bytes(dims):
+        raise ValueError("pool must be uint8 [num_pages, fp8_page_bytes(dims)]")
+    T = h.shape[0]
+    ws, nbytes = _ws(dims, CALL_APPEND_KV_FP8, T, 0, ws, h.device)
+    cd = c_dims(dims)
+    _check(_lib().mla_append_kv_fp8(ctypes.byref(cd), _ptr(h), _ptr(w_dkv_kr), _ptr(seq_idx), _ptr(pos),
+                                    _ptr(block_table), block_table.shape[0], block_table.shape[1], _ptr(pool),
+                                    pool.shape[0], T, _ptr(ws), nbytes, _stream(stream)), "mla_append_kv_fp8")
+    return pool
+
+
+def decode_attention_fp8(dims, q, pool, block_table, seq_lens, max_seq_len, o_lat=None, lse=None, want_lse=True,
+                         ws=None, stream=None):
+    """mla_decode_attention_fp8: mla_decode_attention over an FP8 cache (uint8 [num_pages,
+    fp8_page_bytes(dims)])."""
+    import torch
+    e = _elem(dims)
+    for t, n, dt in ((q, "q", e), (pool, "pool", torch.uint8), (block_table, "block_table", torch.int32),
+                     (seq_lens, "seq_lens", torch.int32)):
+        _need(t, dt, n)
+    if pool.dim() != 2 or pool.shape[1] != fp8_page_bytes(dims):
+        raise ValueError("pool must be uint8 [num_pages, fp8_page_bytes(dims)]")
+    B = q.shape[0]
+    if o_lat is None:
+        o_lat = torch.empty((B, dims.n_heads, dims.d_c), dtype=e, device=q.device)
+    if lse is None and want_lse:
+        lse = torch.empty((B, dims.n_heads), dtype=torch.float32, device=q.device)
+    _need(o_lat, e, "o_lat")
+    if lse is not None:
+        _need(lse, torch.float32, "lse")
+    ws, nbytes = _ws(dims, CALL_DECODE_ATTENTION_FP8, B, max_seq_len, ws, q.device)
+    cd = c_dims(dims)
+    _check(_lib().mla_decode_attention_fp8(ctypes.byref(cd), _ptr(q), _ptr(pool), pool.shape[0], _ptr(block_table),
+                                           block_table.shape[1], _ptr(seq_lens), B, int(max_seq_len), _ptr(o_lat),
+                                           _ptr(lse), _ptr(ws), nbytes, _stream(stream)), "mla_decode_attention_fp8")
     return o_lat, lse
 
 

@@ -27,6 +27,7 @@
 // spans pairs is merged afterwards by log-sum-exp in a fixed order.
 #pragma once
 
+#include "fp8.cuh"
 #include "tc_common.cuh"
 
 namespace mla {
@@ -59,6 +60,11 @@ constexpr int kMmaWarp = 9;        // TMEM allocation; rank 0: S MMA issue
 constexpr int kPairWarp = 10;      // the other page's latent half
 constexpr int kOWarp = 11;        // rank 0: O MMA issue
 constexpr int kThreads = 12 * 32;
+// FP8 cache (see fp8.cuh): warps 12-15 turn the e4m3 boxes the two loaders bring into the chunks
+// above, so that the MMAs are those of the 16-bit cache.
+constexpr int kConvWarp0 = 12;
+constexpr int kThreadsF8 = 16 * 32;
+constexpr int kF8Page = kPage * (kD + 8);  // 64 rows of 576 bytes, then 64 (s_c, s_r) pairs
 // TMEM columns
 constexpr uint32_t kOCol = 0;      // O: n-half j in columns [128j, 128j + 128)
 constexpr uint32_t kSCol = 256;    // S buffer b in columns [256 + 64b, 320 + 64b)
@@ -79,6 +85,7 @@ struct Ctrl {
   uint64_t s_full[2], p_free;
   // Local barriers.
   uint64_t xm_full, xm_free;  // exchange of per-thread partial maxima / sums among the softmax warps
+  uint64_t f8_qk[2][2], f8_pv[2][2], f8_rope;  // FP8: an e4m3 box has landed in this CTA
   uint64_t drain;
   float xm[2][128];          // [column half][TMEM lane]
   uint32_t tmem_slot;
@@ -99,6 +106,7 @@ struct DecodeTcParams {
   float* lse_out;         // [B, n_h] or null
   float* o_part;          // [B + C][n_h][512]
   float* lse_part;        // [B + C][n_h]
+  const uint8_t* f8_pool;  // FP8 pages (their scales are read directly), or null
 };
 
 // Tensor maps of the attention kernel: the paged pool viewed as (64 columns, 64 rows of a page,
@@ -110,8 +118,12 @@ struct DecodeTcParams {
 // its tokens land in slot rows [64 - nv, 64) and the rows before are the tensor map's zero fill,
 // so whatever the pool holds past the end of a sequence never reaches shared memory, and a page
 // wholly past the end (nv = 0) loads as zeros. Softmax masks slot rows r < 64 - nv.
+//
+// FP8 pages are viewed as (576 byte columns, 64 rows, pages) with boxes of 256, 128 and 64 bytes
+// x 64 rows, unswizzled, loaded the same way into the upper half of the chunks they become.
 struct DecodeTcMaps {
   CUtensorMap page1, page2, page4, q9;
+  CUtensorMap f8_256, f8_128, f8_64;
   CUtensorMap o_lat, o_part;  // outputs as (512 columns, n_h heads, rows), 64-byte x 32-head boxes
 };
 
@@ -213,8 +225,27 @@ __device__ __forceinline__ void tma_load_page_pair(uint32_t dst, const CUtensorM
       : "memory");
 }
 
-template <typename T>
-__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(dec::kThreads, 1)
+__device__ __forceinline__ uint4 lds128(uint32_t a) {
+  uint4 v;
+  asm volatile("ld.shared.v4.u32 {%0, %1, %2, %3}, [%4];" : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w) : "r"(a));
+  return v;
+}
+__device__ __forceinline__ void sts128(uint32_t a, const uint4& v) {
+  asm volatile("st.shared.v4.u32 [%0], {%1, %2, %3, %4};" ::"r"(a), "r"(v.x), "r"(v.y), "r"(v.z), "r"(v.w) : "memory");
+}
+// Named barrier with a vote: true on every thread iff `v` was true on all `count` threads.
+__device__ __forceinline__ bool named_bar_and(uint32_t id, uint32_t count, bool v) {
+  uint32_t r;
+  asm volatile(
+      "{\n .reg .pred p, q;\n setp.ne.u32 p, %1, 0;\n bar.red.and.pred q, %2, %3, p;\n selp.u32 %0, 1, 0, q;\n}"
+      : "=r"(r)
+      : "r"((uint32_t)v), "r"(id), "r"(count)
+      : "memory");
+  return r != 0;
+}
+
+template <typename T, bool F8 = false>
+__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(F8 ? dec::kThreadsF8 : dec::kThreads, 1)
     k_decode_tc(const __grid_constant__ DecodeTcMaps maps, const DecodeTcParams p) {
   using namespace dec;
   extern __shared__ uint8_t smem_raw[];
@@ -251,6 +282,12 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(dec::kThreads, 1)
     mbar_init(bar(ctl->xm_full), kSoftWarps);
     mbar_init(bar(ctl->xm_free), kSoftWarps);
     mbar_init(bar(ctl->drain), 2);
+    for (int s = 0; s < 2; ++s)
+      for (int h = 0; h < 2; ++h) {
+        mbar_init(bar(ctl->f8_qk[s][h]), 1);
+        mbar_init(bar(ctl->f8_pv[s][h]), 1);
+      }
+    mbar_init(bar(ctl->f8_rope), 1);
     ctl->abort_flag = 0;
     fence_mbar_init();
   }
@@ -291,9 +328,15 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(dec::kThreads, 1)
     if (warp == kLoadWarp) {
       // ---------------------------------------------------------------- Q, rope and own-page loads
       if (lane == 0) {
-        tma_prefetch_map(&maps.page1);
-        tma_prefetch_map(&maps.page2);
-        tma_prefetch_map(&maps.page4);
+        if constexpr (F8) {  // the maps of the other cache type are left zero
+          tma_prefetch_map(&maps.f8_256);
+          tma_prefetch_map(&maps.f8_128);
+          tma_prefetch_map(&maps.f8_64);
+        } else {
+          tma_prefetch_map(&maps.page1);
+          tma_prefetch_map(&maps.page2);
+          tma_prefetch_map(&maps.page4);
+        }
         tma_prefetch_map(&maps.q9);
         Cursor c;
         c.start(prefix, p.B, cluster, nclusters);
@@ -312,14 +355,25 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(dec::kThreads, 1)
             tma_load_3d_pair(data_u32 + kQOff, &maps.q9, lead(ctl->q_full), 0, b * p.n_h + 64 * (int)rank, 0);
           }
           if (!wait(ctl->rope_done, (c.ti & 1) ^ 1)) break;
-          mbar_arrive_expect_tx_cl(lead(ctl->rope_full), kChunk);
-          tma_load_page_pair(data_u32 + kRopeOff, &maps.page1, lead(ctl->rope_full), nv - kPage, page, 8);
+          if constexpr (F8) {
+            mbar_arrive_expect_tx(bar(ctl->f8_rope), kPage * 64);
+            tma_load_3d(data_u32 + kRopeOff + kChunk / 2, &maps.f8_64, bar(ctl->f8_rope), kDc, nv - kPage, page);
+          } else {
+            mbar_arrive_expect_tx_cl(lead(ctl->rope_full), kChunk);
+            tma_load_page_pair(data_u32 + kRopeOff, &maps.page1, lead(ctl->rope_full), nv - kPage, page, 8);
+          }
           bool ok = true;
           for (int h = 0; h < 2; ++h) {
             // the O MMAs of tile ti - 2 are done with chunks [4h, 4h + 4) of set s
             if (!wait(ctl->set_free[s][h], ((c.ti >> 1) & 1) ^ 1)) {
               ok = false;
               break;
+            }
+            if constexpr (F8) {
+              mbar_arrive_expect_tx(bar(ctl->f8_qk[s][h]), kPage * 256);
+              tma_load_3d(set_u32 + s * kSetBytes + 4 * h * kChunk + 2 * kChunk, &maps.f8_256, bar(ctl->f8_qk[s][h]),
+                          256 * h, nv - kPage, page);
+              continue;
             }
 #ifdef MLA_FAULT_INJECT
             if (h == 0 && rank == 0 && prefix[b] + t == g_inject_missing_tile) {
@@ -363,9 +417,15 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(dec::kThreads, 1)
               ok = false;
               break;
             }
-            mbar_arrive_expect_tx_cl(lead(ctl->pv_full[s][pr]), 2 * kChunk);
-            tma_load_page_pair(set_u32 + s * kSetBytes + 2 * pr * kChunk, &maps.page2, lead(ctl->pv_full[s][pr]),
-                               nv - kPage, page, 4 * j + 2 * (int)rank);
+            if constexpr (F8) {
+              mbar_arrive_expect_tx(bar(ctl->f8_pv[s][j]), kPage * 128);
+              tma_load_3d(set_u32 + s * kSetBytes + 2 * pr * kChunk + kChunk, &maps.f8_128, bar(ctl->f8_pv[s][j]),
+                          256 * j + 128 * (int)rank, nv - kPage, page);
+            } else {
+              mbar_arrive_expect_tx_cl(lead(ctl->pv_full[s][pr]), 2 * kChunk);
+              tma_load_page_pair(set_u32 + s * kSetBytes + 2 * pr * kChunk, &maps.page2, lead(ctl->pv_full[s][pr]),
+                                 nv - kPage, page, 4 * j + 2 * (int)rank);
+            }
           }
           if (!ok) break;
           c.advance(prefix);
@@ -474,6 +534,138 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(dec::kThreads, 1)
         mma_commit2(bar(ctl->drain), 1);  // once all of this thread's MMAs are complete
       }
       __syncwarp();
+    } else if (F8 && warp >= kConvWarp0) {
+      // ---------------------------------------------------------------- FP8: e4m3 boxes -> chunks
+      // Each box (64 slot rows, unswizzled, rows of 256, 128 or 64 bytes) lies in the upper half
+      // of the chunks it becomes: a latent group (4 chunks), a pair (2 chunks), the rope chunk.
+      // The four warps convert it in place, each value times its token's scale in float32: first
+      // the units whose output lies below the box, then, once every thread holds its share of the
+      // rest in registers (a named barrier), the units whose output overwrites it. Thread ct takes
+      // slot row ct / 2 and half ct % 2 of its units, in an order rotated by the row so that a
+      // warp's 16-byte reads spread over the banks. Tile i + 1's rope and latent groups go before
+      // tile i's pairs, the order in which their loads are issued.
+      const int ct = (int)threadIdx.x - 32 * kConvWarp0;
+      const int row = ct >> 1, half = ct & 1;
+      const uint32_t sw = (uint32_t)(row & 7);
+      const float2* const scale_base =
+          reinterpret_cast<const float2*>(p.f8_pool + (size_t)kPage * kD);  // page 0's scales
+      // (s_c, s_r) of slot row `row` of a page with nv tokens (rows before 64 - nv are zero fill)
+      auto scales = [&](int page, int nv) {
+        const int pr = row - (kPage - nv);
+        if (pr < 0) return make_float2(0.f, 0.f);
+        return __ldg(reinterpret_cast<const float2*>(reinterpret_cast<const uint8_t*>(scale_base) +
+                                                     (size_t)page * kF8Page) + pr);
+      };
+      auto put16 = [&](uint32_t dst, int v, const uint4& in, float sc) {
+        uint4 o0, o1;
+        dequant16<T>(in, sc, o0, o1);
+        const uint32_t rb = dst + (v >> 2) * kChunk + row * 128;
+        const uint32_t u = 2u * (v & 3);
+        sts128(rb + ((u ^ sw) << 4), o0);
+        sts128(rb + (((u + 1) ^ sw) << 4), o1);
+      };
+      auto cwait = [&](uint64_t& b, uint32_t parity) {
+        const bool all = named_bar_and(1, 128, mbar_wait(bar(b), parity, abort_flag));
+        if (!all && ct == 0) st_cluster_u32(peer_abort, 1u);
+        return all;
+      };
+      auto publish = [&](uint64_t& full) {  // the chunks are written: both CTAs' MMAs may read them
+        fence_proxy_async_cta();
+        named_bar_sync(1, 128);
+        if (ct == 0) mbar_arrive_cl(lead(full));
+      };
+      // latent group: 4 chunks from dst, box of 256-byte rows at dst + 2 chunks
+      auto conv_group = [&](uint32_t dst, float sc) {
+        const uint32_t box = dst + 2 * kChunk + row * 256;
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+          const int v = 4 * half + ((j + row) & 3);
+          put16(dst, v, lds128(box + 16 * v), sc);
+        }
+        uint4 keep[4];
+#pragma unroll
+        for (int j = 0; j < 4; ++j) keep[j] = lds128(box + 16 * (8 + 4 * half + ((j + row) & 3)));
+        named_bar_sync(1, 128);
+#pragma unroll
+        for (int j = 0; j < 4; ++j) put16(dst, 8 + 4 * half + ((j + row) & 3), keep[j], sc);
+      };
+      // pair: 2 chunks from dst, box of 128-byte rows at dst + 1 chunk
+      auto conv_pair = [&](uint32_t dst, float sc) {
+        const uint32_t box = dst + kChunk + row * 128;
+#pragma unroll
+        for (int j = 0; j < 2; ++j) {
+          const int v = 2 * half + ((j + row) & 1);
+          put16(dst, v, lds128(box + 16 * v), sc);
+        }
+        uint4 keep[2];
+#pragma unroll
+        for (int j = 0; j < 2; ++j) keep[j] = lds128(box + 16 * (4 + 2 * half + ((j + row) & 1)));
+        named_bar_sync(1, 128);
+#pragma unroll
+        for (int j = 0; j < 2; ++j) put16(dst, 4 + 2 * half + ((j + row) & 1), keep[j], sc);
+      };
+      // rope chunk, box of 64-byte rows in its upper half: output rows 32-63 overwrite the box
+      auto conv_rope = [&](uint32_t dst, float sr) {
+        const uint32_t box = dst + kChunk / 2 + row * 64;
+        uint4 keep[2];
+#pragma unroll
+        for (int j = 0; j < 2; ++j) keep[j] = lds128(box + 16 * (2 * half + j));
+        named_bar_sync(1, 128);
+#pragma unroll
+        for (int j = 0; j < 2; ++j) put16(dst, 2 * half + j, keep[j], sr);
+      };
+      // the own page of a tile: rope, then latent groups 0 and 1
+      auto conv_own = [&](const Cursor& c, int L) {
+        const int s = c.ti & 1, page_idx = 2 * c.t + (int)rank;
+        const int nv = min(kPage, max(0, L - kPage * page_idx));
+        const int page = nv > 0 ? p.bt[(long)c.item.b * p.max_pages + page_idx] : 0;
+        const float2 sc = scales(page, nv);
+        if (!cwait(ctl->f8_rope, c.ti & 1)) return false;
+        conv_rope(data_u32 + kRopeOff, sc.y);
+        publish(ctl->rope_full);
+        for (int h = 0; h < 2; ++h) {
+          if (!cwait(ctl->f8_qk[s][h], (c.ti >> 1) & 1)) return false;
+          conv_group(set_u32 + s * kSetBytes + 4 * h * kChunk, sc.x);
+          publish(ctl->qk_full[s][h]);
+        }
+        return true;
+      };
+      // the other page's latent half of a tile: pairs 2j + g, j = 0, 1
+      auto conv_pairs = [&](const Cursor& c, int L) {
+        const int s = c.ti & 1, g = 1 - (int)rank;
+        const int nv = min(kPage, max(0, L - kTile * c.t - kPage * g));
+        const int page = nv > 0 ? p.bt[(long)c.item.b * p.max_pages + 2 * c.t + g] : 0;
+        const float sc = scales(page, nv).x;
+        for (int j = 0; j < 2; ++j) {
+          const int pr = 2 * j + g;
+          if (!cwait(ctl->f8_pv[s][j], (c.ti >> 1) & 1)) return false;
+          conv_pair(set_u32 + s * kSetBytes + 2 * pr * kChunk, sc);
+          publish(ctl->pv_full[s][pr]);
+        }
+        return true;
+      };
+      if constexpr (F8) {
+        Cursor ca, cb;
+        ca.start(prefix, p.B, cluster, nclusters);
+        cb.start(prefix, p.B, cluster, nclusters);
+        int La = 0, Lb = 0;
+        bool ok = true;
+        if (ca.valid) {
+          La = p.seq_lens[ca.item.b];
+          ok = conv_own(ca, La);
+          ca.advance(prefix);
+        }
+        while (ok && cb.valid) {
+          if (ca.valid) {
+            if (ca.first()) La = p.seq_lens[ca.item.b];
+            if (!conv_own(ca, La)) break;
+            ca.advance(prefix);
+          }
+          if (cb.first()) Lb = p.seq_lens[cb.item.b];
+          if (!conv_pairs(cb, Lb)) break;
+          cb.advance(prefix);
+        }
+      }
     } else if (warp < kSoftWarps) {
       // ---------------------------------------------------------------- softmax, rescale, epilogue
       // Thread: TMEM lane lt = 32 (warp % 4) + lane, head h = lt % 64 of this CTA, page g = lt / 64,
@@ -552,14 +744,16 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(dec::kThreads, 1)
         if (!wwait(ctl->p_free, (ti & 1) ^ 1)) break;
         if (!c.first() && __any_sync(0xffffffffu, alpha != 1.f)) {
           tc_fence_after();
+          // two TMEM loads in flight per wait (one with the FP8 cache's smaller register budget)
+          constexpr int kRl = F8 ? 1 : 2;
 #pragma unroll 1
-          for (int c0 = 0; c0 < 128; c0 += 64) {  // two TMEM loads in flight per wait
-            uint32_t r[2][32];
+          for (int c0 = 0; c0 < 128; c0 += 32 * kRl) {
+            uint32_t r[kRl][32];
 #pragma unroll
-            for (int q2 = 0; q2 < 2; ++q2) tmem_ld32(tmem + lane_base + kOCol + 128 * ch + c0 + 32 * q2, r[q2]);
+            for (int q2 = 0; q2 < kRl; ++q2) tmem_ld32(tmem + lane_base + kOCol + 128 * ch + c0 + 32 * q2, r[q2]);
             tmem_wait_ld();
 #pragma unroll
-            for (int q2 = 0; q2 < 2; ++q2) {
+            for (int q2 = 0; q2 < kRl; ++q2) {
 #pragma unroll
               for (int k = 0; k < 32; ++k) r[q2][k] = __float_as_uint(u2f(r[q2][k]) * alpha);
               tmem_st32(tmem + lane_base + kOCol + 128 * ch + c0 + 32 * q2, r[q2]);

@@ -53,6 +53,7 @@ struct EpiParams {
   const int* seq_idx;   // [N]
   const int* bt;
   int num_seqs, max_pages, num_pages, page_size;
+  int stage_rows;       // 1: token n's row goes to row n of `out` ([N][rope_lo + d_rope]), not to the cache
   // query
   void* qc;             // [N][rope_lo] element type
   int n_h, d_c;
@@ -149,6 +150,7 @@ __device__ __noinline__ float2 rope_cs_out_of_line(const float2* tab, const int*
 
 // Cache row offset (elements) of token n for the append step, or -1 (error recorded).
 __device__ __forceinline__ long append_row_base(const EpiParams& e, int n) {
+  if (e.stage_rows) return (long)n * (e.rope_lo + e.d_rope);
   const int s = e.seq_idx[n], p = e.pos[n];
   const int lp = p >= 0 ? p / e.page_size : -1;
   int page = -1;

@@ -32,7 +32,7 @@ struct NvtxRange {
   NvtxRange& operator=(const NvtxRange&) = delete;
 };
 
-thread_local int32_t t_launches[6] = {0, 0, 0, 0, 0, 0};
+thread_local int32_t t_launches[8] = {0, 0, 0, 0, 0, 0, 0, 0};
 // Profiling hook: events recorded around the attention kernel of this thread's decode calls.
 thread_local cudaEvent_t t_ev_before = nullptr, t_ev_after = nullptr;
 inline void mark_before(cudaStream_t st) {
@@ -136,6 +136,7 @@ DecodePlan plan_decode(const mla_dims* d, int B, int max_seq_len) {
 }
 
 size_t ws_append(const mla_dims* d, int T) { return T > 0 ? host::append_layout(d, T, nullptr).bytes : 0; }
+size_t ws_append_fp8(const mla_dims* d, int T) { return T > 0 ? host::append_fp8_bytes(d, T) : 0; }
 size_t ws_absorb(const mla_dims* d, int B) { return B > 0 ? host::absorb_layout(d, B, nullptr).bytes : 0; }
 size_t ws_out(const mla_dims* d, int B) { return B > 0 ? host::out_layout(d, B, nullptr).bytes : 0; }
 
@@ -174,13 +175,20 @@ bool decode_tc_eligible(const mla_dims* d) {
          d->d_c + d->d_rope == tc::dec::kD && d->page_size == tc::dec::kPage;
 }
 
-template <typename T>
+// The FP8 cache serves the tensor-core decode's shape only.
+int fp8_dims(const mla_dims* d) {
+  const int r = check_dims_impl(d);
+  if (r != MLA_OK) return r;
+  return decode_tc_eligible(d) ? MLA_OK : MLA_ERR_UNSUPPORTED_DIMS;
+}
+
+template <typename T, bool F8 = false>
 bool decode_tc_set_smem() {
   static std::atomic<bool> done[kMaxDevices];
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return false;
   if (!done[dev].load(std::memory_order_acquire)) {
-    if (cudaFuncSetAttribute(tc::k_decode_tc<T>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)tc::dec::kSmem) !=
+    if (cudaFuncSetAttribute(tc::k_decode_tc<T, F8>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)tc::dec::kSmem) !=
         cudaSuccess)
       return false;
     done[dev].store(true, std::memory_order_release);
@@ -234,12 +242,12 @@ size_t ws_decode(const mla_dims* d, int B, int max_seq_len) {
   return align256(bh * p.n_splits * d->d_c * 4) + align256(bh * p.n_splits * 4);
 }
 
-template <typename T>
+template <typename T, bool F8 = false>
 int decode_tc_impl(const mla_dims* d, const void* q, const void* pool, int32_t num_pages, const int32_t* bt,
                    int32_t max_pages, const int32_t* seq_lens, int32_t B, int32_t max_seq_len, void* o_lat,
                    float* lse_out, void* ws, cudaStream_t st, int32_t& launches) {
   const int C = decode_clusters();
-  if (!decode_tc_set_smem<T>()) return MLA_ERR_CUDA;
+  if (!decode_tc_set_smem<T, F8>()) return MLA_ERR_CUDA;
   Carve c{static_cast<char*>(ws)};
   int* prefix = c.take<int>((size_t)B + 1);
   int* seq_pairs = c.take<int>((size_t)B);
@@ -248,9 +256,15 @@ int decode_tc_impl(const mla_dims* d, const void* q, const void* pool, int32_t n
   float* lse_part = c.take<float>(((size_t)B + C) * d->n_heads);
   constexpr bool bf16 = tc::IsBf16<T>::value;
   tc::DecodeTcMaps maps;
-  if (!host::encode_pages(&maps.page1, pool, bf16, (uint64_t)num_pages, tc::dec::kD * 2, 1) ||
-      !host::encode_pages(&maps.page2, pool, bf16, (uint64_t)num_pages, tc::dec::kD * 2, 2) ||
-      !host::encode_pages(&maps.page4, pool, bf16, (uint64_t)num_pages, tc::dec::kD * 2, 4) ||
+  std::memset(&maps, 0, sizeof(maps));
+  const bool pages_ok =
+      F8 ? host::encode_pages_fp8(&maps.f8_256, pool, (uint64_t)num_pages, 256) &&
+               host::encode_pages_fp8(&maps.f8_128, pool, (uint64_t)num_pages, 128) &&
+               host::encode_pages_fp8(&maps.f8_64, pool, (uint64_t)num_pages, 64)
+         : host::encode_pages(&maps.page1, pool, bf16, (uint64_t)num_pages, tc::dec::kD * 2, 1) &&
+               host::encode_pages(&maps.page2, pool, bf16, (uint64_t)num_pages, tc::dec::kD * 2, 2) &&
+               host::encode_pages(&maps.page4, pool, bf16, (uint64_t)num_pages, tc::dec::kD * 2, 4);
+  if (!pages_ok ||
       !host::encode_chunks(&maps.q9, q, bf16, (uint64_t)B * d->n_heads, tc::dec::kD * 2, 9) ||
       !host::encode_heads_out(&maps.o_lat, o_lat, bf16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT16,
                               2, (uint64_t)d->n_heads, (uint64_t)B) ||
@@ -272,8 +286,10 @@ int decode_tc_impl(const mla_dims* d, const void* q, const void* pool, int32_t n
   p.lse_out = lse_out;
   p.o_part = o_part;
   p.lse_part = lse_part;
+  p.f8_pool = F8 ? static_cast<const uint8_t*>(pool) : nullptr;
   mark_before(st);
-  if (launch_pdl(tc::k_decode_tc<T>, dim3(2 * C), dim3(tc::dec::kThreads), tc::dec::kSmem, st, maps, p) != cudaSuccess)
+  if (launch_pdl(tc::k_decode_tc<T, F8>, dim3(2 * C), dim3(F8 ? tc::dec::kThreadsF8 : tc::dec::kThreads),
+                 tc::dec::kSmem, st, maps, p) != cudaSuccess)
     return MLA_ERR_CUDA;
   mark_after(st);
   if (launch_pdl(tc::k_decode_tc_merge<T>, dim3(B, (d->n_heads + 31) / 32), dim3(512), 0, st,
@@ -570,6 +586,11 @@ size_t mla_workspace_size(const mla_dims* dims, int32_t call, int32_t B, int32_t
     case MLA_CALL_OUT_PROJ: return ws_out(dims, B);
     case MLA_CALL_PREFILL_ATTENTION: return ws_prefill(dims, B, max_seq_len);
     case MLA_CALL_LAYER_STEP_SMALL: return ws_layer_small(dims, B, max_seq_len);
+    case MLA_CALL_APPEND_KV_FP8: return fp8_dims(dims) == MLA_OK ? ws_append_fp8(dims, B) : 0;
+    case MLA_CALL_DECODE_ATTENTION_FP8:
+      return fp8_dims(dims) == MLA_OK && B > 0 && max_seq_len >= 1 && max_seq_len <= kMaxSeqLen
+                 ? ws_decode_tc(dims, B)
+                 : 0;
     default: return 0;
   }
 }
@@ -648,6 +669,72 @@ int mla_decode_attention(const mla_dims* dims, const void* q, const void* pool, 
                                 lse_out, ws, st, n);
   if (r != MLA_OK) return r;
   return finish_launches(MLA_CALL_DECODE_ATTENTION, n);
+}
+
+int64_t mla_fp8_page_bytes(const mla_dims* dims) {
+  const int r = check_dims_impl(dims);
+  if (r != MLA_OK) return r;
+  return fp8::page_bytes(dims->page_size, dims->d_c + dims->d_rope);
+}
+
+int mla_fp8_supported(const mla_dims* dims) {
+  if (dims == nullptr) return MLA_ERR_INVALID_ARG;
+  const int r = fp8_dims(dims);
+  return r == MLA_ERR_INVALID_ARG ? r : (r == MLA_OK ? MLA_OK : MLA_ERR_UNSUPPORTED_DIMS);
+}
+
+int mla_append_kv_fp8(const mla_dims* dims, const void* h, const void* w_dkv_kr, const int32_t* seq_idx,
+                      const int32_t* pos, const int32_t* block_table, int32_t num_seqs, int32_t max_pages, void* pool,
+                      int32_t num_pages, int32_t T, void* ws, size_t ws_bytes, mla_stream_t stream) {
+  NvtxRange nvtx_range("mla_append_kv_fp8");
+  int r = fp8_dims(dims);
+  if (r != MLA_OK) return r;
+  if (T < 0 || num_seqs <= 0 || max_pages <= 0 || num_pages <= 0) return MLA_ERR_INVALID_ARG;
+  if (T == 0) {
+    t_launches[MLA_CALL_APPEND_KV_FP8] = 0;
+    return MLA_OK;
+  }
+  if (!h || !w_dkv_kr || !seq_idx || !pos || !block_table || !pool || !ws) return MLA_ERR_INVALID_ARG;
+  if (!aligned16(h) || !aligned16(w_dkv_kr) || !aligned16(pool) || !aligned16(ws)) return MLA_ERR_ALIGNMENT;
+  if (ws_bytes < ws_append_fp8(dims, T)) return MLA_ERR_WORKSPACE_TOO_SMALL;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  int32_t n = 0;
+  r = dims->dtype == MLA_BF16 ? host::append_fp8_run<__nv_bfloat16>(dims, h, w_dkv_kr, seq_idx, pos, block_table,
+                                                                      num_seqs, max_pages, pool, num_pages, T, ws, st, n)
+                              : host::append_fp8_run<__half>(dims, h, w_dkv_kr, seq_idx, pos, block_table, num_seqs,
+                                                             max_pages, pool, num_pages, T, ws, st, n);
+  if (r != MLA_OK) return r;
+  return finish_launches(MLA_CALL_APPEND_KV_FP8, n);
+}
+
+int mla_decode_attention_fp8(const mla_dims* dims, const void* q, const void* pool, int32_t num_pages,
+                             const int32_t* block_table, int32_t max_pages, const int32_t* seq_lens, int32_t B,
+                             int32_t max_seq_len, void* o_lat, float* lse_out, void* ws, size_t ws_bytes,
+                             mla_stream_t stream) {
+  NvtxRange nvtx_range("mla_decode_attention_fp8");
+  int r = fp8_dims(dims);
+  if (r != MLA_OK) return r;
+  if (B < 0 || B > 65535 || max_seq_len < 1 || max_seq_len > kMaxSeqLen || max_pages <= 0 || num_pages <= 0)
+    return MLA_ERR_INVALID_ARG;
+  if ((long)max_pages * dims->page_size < (long)max_seq_len) return MLA_ERR_INVALID_ARG;
+  if (!page_total_fits(dims, B, max_seq_len)) return MLA_ERR_INVALID_ARG;
+  if (B == 0) {
+    t_launches[MLA_CALL_DECODE_ATTENTION_FP8] = 0;
+    return MLA_OK;
+  }
+  if (!q || !pool || !block_table || !seq_lens || !o_lat || !ws) return MLA_ERR_INVALID_ARG;
+  if (!aligned16(q) || !aligned16(pool) || !aligned16(o_lat) || !aligned16(ws) || !aligned16(lse_out))
+    return MLA_ERR_ALIGNMENT;
+  if (ws_bytes < ws_decode_tc(dims, B)) return MLA_ERR_WORKSPACE_TOO_SMALL;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  int32_t n = 0;
+  r = dims->dtype == MLA_BF16
+          ? decode_tc_impl<__nv_bfloat16, true>(dims, q, pool, num_pages, block_table, max_pages, seq_lens, B,
+                                                max_seq_len, o_lat, lse_out, ws, st, n)
+          : decode_tc_impl<__half, true>(dims, q, pool, num_pages, block_table, max_pages, seq_lens, B, max_seq_len,
+                                         o_lat, lse_out, ws, st, n);
+  if (r != MLA_OK) return r;
+  return finish_launches(MLA_CALL_DECODE_ATTENTION_FP8, n);
 }
 
 int mla_prefill_attention(const mla_dims* dims, const void* q, const void* pool, int32_t num_pages,
@@ -759,7 +846,7 @@ const char* mla_error_string(int code) {
   }
 }
 
-int32_t mla_last_launch_count(int32_t call) { return (call >= 0 && call < 6) ? t_launches[call] : -1; }
+int32_t mla_last_launch_count(int32_t call) { return (call >= 0 && call < 8) ? t_launches[call] : -1; }
 
 int mla_debug_gemm_plan(int32_t M, int32_t N, int32_t K, int32_t batch, int32_t fused_rope, int32_t d_rope,
                         int64_t* out) {

@@ -14,6 +14,7 @@
 #include <cstring>
 #include <mutex>
 
+#include "fp8.cuh"
 #include "gemm_sk.cuh"
 #include "proj_simt.cuh"
 
@@ -109,6 +110,21 @@ inline bool encode_pages(CUtensorMap* map, const void* base, bool bf16, uint64_t
   return fn(map, bf16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 4, const_cast<void*>(base),
             dims, strides, box, es, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+// FP8 pages (see fp8.cuh) viewed as (576 byte columns, 64 rows, pages): rows of 576 bytes, pages
+// of 64 rows plus their 512 bytes of scales; boxes of `width` bytes x 64 rows x 1 page, no
+// swizzle. Rows outside the page read as zeros.
+inline bool encode_pages_fp8(CUtensorMap* map, const void* base, uint64_t pages, uint32_t width) {
+  auto fn = tensor_map_encoder();
+  if (fn == nullptr) return false;
+  cuuint64_t dims[3] = {576, 64, pages};
+  cuuint64_t strides[2] = {576, 64 * (576 + 8)};
+  cuuint32_t box[3] = {width, 64, 1};
+  cuuint32_t es[3] = {1, 1, 1};
+  return fn(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 3, const_cast<void*>(base), dims, strides, box, es,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
 // 3-D view of an output [rows][n_h][512] (fp32, bf16 or fp16) as (512 columns, n_h heads, rows)
@@ -337,6 +353,47 @@ int append_run(const mla_dims* d, const void* h, const void* w, const int32_t* s
   e.d_c = d->d_c;
   e.cs_glob = L.cs;
   return gemm_sk<T>({w, D, d->d_model, 0}, false, {h, T_, d->d_model, 0}, D, T_, d->d_model, L.g, e, L.part, st, n);
+}
+
+// ------------------------------------------------------------------ mla_append_kv_fp8
+// The append GEMM writes the rows (element type, RoPE applied) to a staging area after its own
+// workspace; k_quant_fp8 then quantises each into its FP8 cache slot.
+inline size_t append_fp8_bytes(const mla_dims* d, int T_) {
+  return ((append_layout(d, T_, nullptr).bytes + 255) & ~size_t(255)) + (size_t)T_ * (d->d_c + d->d_rope) * 2;
+}
+
+template <typename T>
+int append_fp8_run(const mla_dims* d, const void* h, const void* w, const int32_t* seq_idx, const int32_t* pos,
+                   const int32_t* bt, int32_t num_seqs, int32_t max_pages, void* pool, int32_t num_pages, int32_t T_,
+                   void* ws, cudaStream_t st, int32_t& n) {
+  const int D = d->d_c + d->d_rope;
+  const AppendLayout L = append_layout(d, T_, ws);
+  T* rows = reinterpret_cast<T*>(static_cast<char*>(ws) + ((L.bytes + 255) & ~size_t(255)));
+  tc::EpiParams e{};
+  e.mode = tc::kEpiAppend;
+  e.out = rows;
+  e.stage_rows = 1;
+  e.rope_lo = d->d_c;
+  e.d_rope = d->d_rope;
+  e.rope_base = d->rope_base;
+  e.rope_table = d->rope_inv_freq;
+  e.pos = pos;
+  e.seq_idx = seq_idx;
+  e.bt = bt;
+  e.num_seqs = num_seqs;
+  e.max_pages = max_pages;
+  e.num_pages = num_pages;
+  e.page_size = d->page_size;
+  e.d_c = d->d_c;
+  e.cs_glob = L.cs;
+  const int r = gemm_sk<T>({w, D, d->d_model, 0}, false, {h, T_, d->d_model, 0}, D, T_, d->d_model, L.g, e, L.part, st, n);
+  if (r != MLA_OK) return r;
+  if (launch_pdl(k_quant_fp8<T>, dim3((unsigned)((T_ + 7) / 8)), dim3(256), 0, st, static_cast<const T*>(rows),
+                 seq_idx, pos, bt, (int)num_seqs, (int)max_pages, (int)num_pages, (int)d->page_size, (int)d->d_c, D,
+                 (int)T_, static_cast<uint8_t*>(pool)) != cudaSuccess)
+    return MLA_ERR_CUDA;
+  ++n;
+  return MLA_OK;
 }
 
 // ------------------------------------------------------------------ mla_absorb_query

@@ -178,7 +178,7 @@ def test_prefill_argument_errors_queue_nothing(lib):
     assert call(a14=16) == -3                             # too-small workspace
     assert call(a9=0, a1=None, a13=None) == 0             # T == 0 is a no-op
     assert lib.mla_last_launch_count(M.CALL_PREFILL_ATTENTION) == 0
-    assert lib.mla_last_launch_count(6) == -1
+    assert lib.mla_last_launch_count(8) == -1
 
 
 def test_layer_step_small_argument_errors_queue_nothing(lib):
@@ -278,3 +278,41 @@ def test_prefill_groups_shrink_to_keep_page_totals_in_int32():
     assert a == M.workspace_size(P, M.CALL_PREFILL_ATTENTION, 128, big) == M.workspace_size(
         P, M.CALL_PREFILL_ATTENTION, 4096, big)
     assert a >= 127 * (1 << 24) * 4
+
+
+def test_fp8_calls_argument_errors_queue_nothing(lib):
+    """The FP8 cache calls: page size, shape support and argument checks, before anything is
+    queued (no GPU)."""
+    P, R = dims(synth.PRODUCTION), dims(synth.RUNNING)
+    assert lib.mla_fp8_page_bytes(ctypes.byref(P)) == 64 * 584
+    assert lib.mla_fp8_supported(ctypes.byref(P)) == 0
+    assert lib.mla_fp8_supported(ctypes.byref(R)) == -2
+    assert lib.mla_workspace_size(ctypes.byref(R), M.CALL_DECODE_ATTENTION_FP8, 4, 256) == 0
+    need = lib.mla_workspace_size(ctypes.byref(P), M.CALL_APPEND_KV_FP8, 64, 0)
+    assert need >= 64 * 576 * 2 and need % 256 == 0
+    args = [ctypes.byref(P), FAKE, FAKE, FAKE, FAKE, FAKE, 2, 4, FAKE, 8, 64, FAKE, need, None]
+
+    def append(**kw):
+        a = list(args)
+        for k, v in kw.items():
+            a[int(k[1:])] = v
+        return lib.mla_append_kv_fp8(*a)
+    assert append(a0=ctypes.byref(R)) == -2
+    assert append(a12=need - 16) == -3
+    assert append(a8=MISALIGNED) == -4
+    assert append(a10=0, a1=None) == 0
+    assert lib.mla_last_launch_count(M.CALL_APPEND_KV_FP8) == 0
+    dneed = lib.mla_workspace_size(ctypes.byref(P), M.CALL_DECODE_ATTENTION_FP8, 2, 256)
+    assert dneed > 0
+    dargs = [ctypes.byref(P), FAKE, FAKE, 10, FAKE, 4, FAKE, 2, 256, FAKE, None, FAKE, dneed, None]
+
+    def decode(**kw):
+        a = list(dargs)
+        for k, v in kw.items():
+            a[int(k[1:])] = v
+        return lib.mla_decode_attention_fp8(*a)
+    assert decode(a0=ctypes.byref(R)) == -2
+    assert decode(a12=dneed - 16) == -3
+    assert decode(a8=257 * 64) == -1                      # max_pages * page_size < max_seq_len
+    assert decode(a7=0) == 0
+    assert lib.mla_last_launch_count(M.CALL_DECODE_ATTENTION_FP8) == 0
