@@ -270,10 +270,15 @@ def run_mla(args):
     T = B * chunk                    # new tokens per step
     h0 = synth.hidden(w, batch=T).to(dev)
     h = h0.clone()
-    attn_call = M.CALL_PREFILL_ATTENTION if chunk > 1 else M.CALL_DECODE_ATTENTION
-    calls = (M.CALL_APPEND_KV, M.CALL_ABSORB_QUERY, attn_call, M.CALL_OUT_PROJ)
+    fp8 = w.cache == "fp8"           # FP8 latent cache: mla_append_kv_fp8 and mla_decode_attention_fp8
+    if fp8 and chunk > 1:
+        raise SystemExit(f"workload {w.name}: the FP8 cache serves decode steps")
+    attn_call = (M.CALL_PREFILL_ATTENTION if chunk > 1 else M.CALL_DECODE_ATTENTION_FP8 if fp8
+                 else M.CALL_DECODE_ATTENTION)
+    append_call = M.CALL_APPEND_KV_FP8 if fp8 else M.CALL_APPEND_KV
+    calls = (append_call, M.CALL_ABSORB_QUERY, attn_call, M.CALL_OUT_PROJ)
     fused = args.fused
-    if fused and (chunk > 1 or not M.layer_step_small_supported(d)):
+    if fused and (chunk > 1 or fp8 or not M.layer_step_small_supported(d)):
         raise SystemExit(f"--fused: workload {w.name} is not a decode step with small-head dims")
     if fused:
         calls = (M.CALL_LAYER_STEP_SMALL,)
@@ -314,8 +319,9 @@ def run_mla(args):
             if record:
                 ev = [EV() for _ in range(5)]
                 ev[0].record(stream)
-            M.append_kv(d, x, w_["w_dkv_kr"], seq_idx, pos, st.block_table, st.pool, ws=ws, stream=stream)
-            n = M.last_launch_count(0)
+            (M.append_kv_fp8 if fp8 else M.append_kv)(d, x, w_["w_dkv_kr"], seq_idx, pos, st.block_table, st.pool,
+                                                      ws=ws, stream=stream)
+            n = M.last_launch_count(append_call)
             if record:
                 ev[1].record(stream)
             M.absorb_query(d, x, w_["w_dq"], w_["w_uq_qr"], w_["w_uk"], pos, q_out=o["q"], ws=ws, stream=stream)
@@ -331,8 +337,9 @@ def run_mla(args):
                 M.prefill_attention(d, o["q"], st.pool, st.block_table, seq_idx, pos, ix.max_seq_len,
                                     o_lat=o["o_lat"], lse=o["lse"], ws=ws, stream=stream)
             else:
-                M.decode_attention(d, o["q"], st.pool, st.block_table, aux, ix.max_seq_len, o_lat=o["o_lat"],
-                                   lse=o["lse"], ws=ws, stream=stream)
+                (M.decode_attention_fp8 if fp8 else M.decode_attention)(
+                    d, o["q"], st.pool, st.block_table, aux, ix.max_seq_len, o_lat=o["o_lat"], lse=o["lse"], ws=ws,
+                    stream=stream)
             if record:
                 M.set_decode_timing_events(None, None)
                 kernel_events.append(kev)
@@ -496,8 +503,8 @@ def run_mla(args):
         ms_step = ms_total / args.steps
         us_layer_job = job_us_per_layer_step(ms_total, args.steps, len(layers), world)
         us_e2e_job = job_us_per_layer_step(ms_e2e, args.steps, len(layers), world)
-        dbytes, dflops = harness.attention_work(d, cached, chunk)
-        sbytes, sflops = harness.layer_work(d, cached, chunk)
+        dbytes, dflops = harness.attention_work(d, cached, chunk, w.cache)
+        sbytes, sflops = harness.layer_work(d, cached, chunk, w.cache)
         if fused:  # the fused kernel does the whole layer: its roofline is the layer's
             dbytes, dflops = sbytes, sflops
         dec_s = decode_ms * 1e-3    # the whole call: planner + attention kernel + merge
@@ -515,6 +522,8 @@ def run_mla(args):
         roof["frac_whole_call"] = call_frac  # counting the planner and merge launches too
         roof["traffic"] = measured_decode_traffic(w.name)
         roof["kernel"] = ("k_layer_small (mla_layer_step_small: the whole layer step in one launch)" if fused
+                          else "attention kernel of mla_decode_attention_fp8 (k_decode_tc with the FP8 converting "
+                               "warps)" if fp8
                           else "attention kernel of mla_prefill_attention (k_decode_tc, one item per new token)"
                           if chunk > 1 else "attention kernel of mla_decode_attention (k_decode_tc; warp-MMA "
                                             "k_decode_mma at small n_h)")
@@ -532,6 +541,7 @@ def run_mla(args):
                                                                          f"U[{w.cached[0]},{w.cached[1]}], sum "
                                                                          f"{int(cached.sum())}"),
                        "layers": len(layers), "dims": dims_desc(d), "paging": w.paging,
+                       **({"cache": "fp8 e4m3 rows + (s_c, s_r) float32 per token, 584 B"} if fp8 else {}),
                        **({"chunk": chunk, "new_tokens": T} if chunk > 1 else {}),
                        "path": ("one launch per layer (mla_layer_step_small)" if fused else
                                 "four C-ABI calls per layer"),

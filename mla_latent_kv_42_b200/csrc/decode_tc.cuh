@@ -542,8 +542,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(F8 ? dec::kThreadsF8
       // the units whose output lies below the box, then, once every thread holds its share of the
       // rest in registers (a named barrier), the units whose output overwrites it. Thread ct takes
       // slot row ct / 2 and half ct % 2 of its units, in an order rotated by the row so that a
-      // warp's 16-byte reads spread over the banks. Tile i + 1's rope and latent groups go before
-      // tile i's pairs, the order in which their loads are issued.
+      // warp's 16-byte reads spread over the banks. Tiles go in order, each tile's own page (rope,
+      // latent groups) and then its pairs: the next tile's own page was loaded while this tile's S
+      // ran, so it is ready by the time the pairs are done.
       const int ct = (int)threadIdx.x - 32 * kConvWarp0;
       const int row = ct >> 1, half = ct & 1;
       const uint32_t sw = (uint32_t)(row & 7);
@@ -615,11 +616,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(F8 ? dec::kThreadsF8
         for (int j = 0; j < 2; ++j) put16(dst, 2 * half + j, keep[j], sr);
       };
       // the own page of a tile: rope, then latent groups 0 and 1
-      auto conv_own = [&](const Cursor& c, int L) {
-        const int s = c.ti & 1, page_idx = 2 * c.t + (int)rank;
-        const int nv = min(kPage, max(0, L - kPage * page_idx));
-        const int page = nv > 0 ? p.bt[(long)c.item.b * p.max_pages + page_idx] : 0;
-        const float2 sc = scales(page, nv);
+      auto conv_own = [&](const Cursor& c, float2 sc) {
+        const int s = c.ti & 1;
         if (!cwait(ctl->f8_rope, c.ti & 1)) return false;
         conv_rope(data_u32 + kRopeOff, sc.y);
         publish(ctl->rope_full);
@@ -631,11 +629,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(F8 ? dec::kThreadsF8
         return true;
       };
       // the other page's latent half of a tile: pairs 2j + g, j = 0, 1
-      auto conv_pairs = [&](const Cursor& c, int L) {
+      auto conv_pairs = [&](const Cursor& c, float sc) {
         const int s = c.ti & 1, g = 1 - (int)rank;
-        const int nv = min(kPage, max(0, L - kTile * c.t - kPage * g));
-        const int page = nv > 0 ? p.bt[(long)c.item.b * p.max_pages + 2 * c.t + g] : 0;
-        const float sc = scales(page, nv).x;
         for (int j = 0; j < 2; ++j) {
           const int pr = 2 * j + g;
           if (!cwait(ctl->f8_pv[s][j], (c.ti >> 1) & 1)) return false;
@@ -644,26 +639,39 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(F8 ? dec::kThreadsF8
         }
         return true;
       };
+      // this thread's scales for a tile: the own page's (s_c, s_r) and the other page's s_c (their
+      // page ids and values are read a tile ahead, so that their latency hides behind a tile)
+      struct TileScales {
+        float2 own;
+        float pair;
+      };
+      auto tile_scales = [&](const Cursor& c, int L) {
+        const int pi = 2 * c.t + (int)rank, g = 1 - (int)rank;
+        const int nv_o = min(kPage, max(0, L - kPage * pi));
+        const int nv_p = min(kPage, max(0, L - kTile * c.t - kPage * g));
+        const long bt0 = (long)c.item.b * p.max_pages;
+        const int pg_o = nv_o > 0 ? p.bt[bt0 + pi] : 0;
+        const int pg_p = nv_p > 0 ? p.bt[bt0 + 2 * c.t + g] : 0;
+        return TileScales{scales(pg_o, nv_o), scales(pg_p, nv_p).x};
+      };
       if constexpr (F8) {
-        Cursor ca, cb;
-        ca.start(prefix, p.B, cluster, nclusters);
-        cb.start(prefix, p.B, cluster, nclusters);
-        int La = 0, Lb = 0;
-        bool ok = true;
-        if (ca.valid) {
-          La = p.seq_lens[ca.item.b];
-          ok = conv_own(ca, La);
-          ca.advance(prefix);
-        }
-        while (ok && cb.valid) {
-          if (ca.valid) {
-            if (ca.first()) La = p.seq_lens[ca.item.b];
-            if (!conv_own(ca, La)) break;
-            ca.advance(prefix);
+        Cursor c;
+        c.start(prefix, p.B, cluster, nclusters);
+        int L = c.valid ? p.seq_lens[c.item.b] : 0;
+        TileScales cur = c.valid ? tile_scales(c, L) : TileScales{};
+        while (c.valid) {
+          Cursor nx = c;
+          nx.advance(prefix);
+          int Ln = L;
+          TileScales nxt{};
+          if (nx.valid) {
+            if (nx.first()) Ln = p.seq_lens[nx.item.b];
+            nxt = tile_scales(nx, Ln);
           }
-          if (cb.first()) Lb = p.seq_lens[cb.item.b];
-          if (!conv_pairs(cb, Lb)) break;
-          cb.advance(prefix);
+          if (!conv_own(c, cur.own) || !conv_pairs(c, cur.pair)) break;
+          c = nx;
+          L = Ln;
+          cur = nxt;
         }
       }
     } else if (warp < kSoftWarps) {

@@ -52,7 +52,10 @@ def make_layer(w: synth.Workload, cached: np.ndarray, layer: int = 0, device="cu
     if block_table is None:
         block_table, num_pages = synth.page_table(cached, d.page_size, w.paging, w.seed, spare_tokens=spare_tokens)
     rows = synth.prefix_rows(w, cached, layer=layer, device=device)
-    pool = synth.paged_pool(rows, cached, block_table, num_pages, d.page_size, fill=fill)
+    if w.cache == "fp8":  # random bytes in the FP8 page format (the rows above are not in it)
+        pool = synth.fp8_pages(w, num_pages, layer=layer, device=device)
+    else:
+        pool = synth.paged_pool(rows, cached, block_table, num_pages, d.page_size, fill=fill)
     st = LayerState(dims=d, w={k: v.to(device) for k, v in W.items()}, pool=pool,
                     block_table=torch.from_numpy(block_table).to(device))
     return Layer(state=st, W_host=W, rows=rows, offsets=np.concatenate([[0], np.cumsum(cached)]))
@@ -90,7 +93,13 @@ def step_work(d: synth.Dims, seq_lens: np.ndarray) -> tuple[int, int]:
     return db + weight_bytes(d) + act_bytes, df + proj_flops
 
 
-def attention_work(d: synth.Dims, cached: np.ndarray, chunk: int = 1) -> tuple[int, int]:
+def cache_row_bytes(d: synth.Dims, cache: str = "elem") -> int:
+    """Bytes of one cached token: D element-type values, or D e4m3 bytes and two float32 scales."""
+    D = d.d_c + d.d_rope
+    return D + 8 if cache == "fp8" else 2 * D
+
+
+def attention_work(d: synth.Dims, cached: np.ndarray, chunk: int = 1, cache: str = "elem") -> tuple[int, int]:
     """Algorithmic bytes and flops of the attention call of a step bringing ``chunk`` new tokens
     to every sequence (chunk = 1: decode; equals ``decode_work(d, cached + 1)``).
 
@@ -103,19 +112,19 @@ def attention_work(d: synth.Dims, cached: np.ndarray, chunk: int = 1) -> tuple[i
     T = len(cached) * chunk
     rows = int(np.sum(cached + chunk))
     attended = int(np.sum(chunk * (cached + 1) + chunk * (chunk - 1) // 2))
-    byts = 2 * (rows * D + T * d.n_heads * D + T * d.n_heads * d.d_c)
+    byts = rows * cache_row_bytes(d, cache) + 2 * (T * d.n_heads * D + T * d.n_heads * d.d_c)
     flops = 2 * attended * d.n_heads * (D + d.d_c)
     return byts, flops
 
 
-def layer_work(d: synth.Dims, cached: np.ndarray, chunk: int = 1) -> tuple[int, int]:
+def layer_work(d: synth.Dims, cached: np.ndarray, chunk: int = 1, cache: str = "elem") -> tuple[int, int]:
     """Algorithmic bytes and flops of a whole layer step bringing ``chunk`` new tokens to every
     sequence: weights read once, the projections of every new token, and the attention call
     (chunk = 1: equals ``step_work(d, cached + 1)``)."""
     T = len(cached) * chunk
-    ab, af = attention_work(d, cached, chunk)
+    ab, af = attention_work(d, cached, chunk, cache)
     n_h = d.n_heads
     proj_flops = 2 * T * ((d.d_c + d.d_rope) * d.d_model + d.d_cq * d.d_model + n_h * (d.d_head + d.d_rope) * d.d_cq
                           + 2 * n_h * d.d_head * d.d_c + d.d_model * n_h * d.d_head)
-    act_bytes = 2 * T * (2 * d.d_model + (d.d_c + d.d_rope))
+    act_bytes = 2 * T * 2 * d.d_model + T * cache_row_bytes(d, cache)  # h in, u out, the appended rows
     return ab + weight_bytes(d) + act_bytes, af + proj_flops

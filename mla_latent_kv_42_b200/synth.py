@@ -29,7 +29,7 @@ import torch
 __all__ = [
     "Dims", "RUNNING", "PRODUCTION", "Workload", "WORKLOADS", "workload",
     "WEIGHT_ORDER", "weights", "hidden", "cached_lengths", "page_table", "prefix_rows",
-    "paged_pool", "synthetic_query", "to_storage", "storage_dtype", "yarn_inv_freq",
+    "paged_pool", "synthetic_query", "to_storage", "storage_dtype", "yarn_inv_freq", "fp8_pages",
 ]
 
 
@@ -72,6 +72,7 @@ class Workload:
     paging: str                     # "contiguous" or "shuffled"
     seed: int = 0
     chunk: int = 1                  # new tokens per sequence per step (1 = decode; more = chunked prefill)
+    cache: str = "elem"             # "elem": element-type rows; "fp8": e4m3 pages with two scales per token
 
     @property
     def ragged(self) -> bool:
@@ -89,6 +90,8 @@ WORKLOADS = {
         Workload("production_b8_n4096_chunk128_bf16", PRODUCTION, 8, 4096, 1, 0.006, "contiguous", chunk=128),
         # chunked prefill over a prefix larger than L2 (64 x 4096 cached rows = 302 MB)
         Workload("production_b64_n4096_chunk32_bf16", PRODUCTION, 64, 4096, 1, 0.006, "contiguous", chunk=32),
+        # the decode shape above over an FP8 latent cache (584 bytes per token instead of 1152)
+        Workload("production_b64_n4096_fp8", PRODUCTION, 64, 4096, 1, 0.006, "contiguous", cache="fp8"),
     ]
 }
 
@@ -206,6 +209,21 @@ def paged_pool(rows: torch.Tensor, cached: np.ndarray, block_table: np.ndarray, 
     idx = torch.from_numpy(np.concatenate(slots) if slots else np.zeros(0, np.int64)).to(rows.device)
     pool.view(-1, D).index_copy_(0, idx, rows)
     return pool
+
+
+def fp8_pages(w: Workload, num_pages: int, layer: int = 0, device: str = "cpu") -> torch.Tensor:
+    """An FP8 cache of ``num_pages`` pages (uint8 [num_pages, page_size * (D + 8)]) filled with
+    random bytes in the cache format: every row byte a uniformly drawn non-NaN e4m3 code, every
+    scale pair uniform in [0.5, 1.5] / 448 (decoded magnitudes up to about 1.5, as the 16-bit
+    prefix rows have). Drawn, not computed from rows: a timing input for the FP8 decode."""
+    d = w.dims
+    g = torch.Generator().manual_seed(w.seed * 1000003 + layer * 7919 + 17)
+    P, D = d.page_size, d.D
+    codes = torch.randint(0, 0x7F, (num_pages, P * D), generator=g, dtype=torch.int32)  # 0x00 .. 0x7E
+    codes |= torch.randint(0, 2, (num_pages, P * D), generator=g, dtype=torch.int32) << 7
+    scales = (0.5 + torch.rand((num_pages, P * 2), generator=g)) / 448.0
+    pages = torch.cat([codes.to(torch.uint8), scales.contiguous().view(torch.uint8).view(num_pages, -1)], dim=1)
+    return pages.to(device)
 
 
 def synthetic_query(w: Workload, batch: int, scale: float = 1.0, seed_tag: int = 0) -> torch.Tensor:
