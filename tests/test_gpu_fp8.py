@@ -15,6 +15,8 @@ summary page ("The Model"): e4m3 bytes with two float32 scales per token, max|pa
   float32) to the element type before the tensor-core products, as the 16-bit cache holds
   element-type rows.
 """
+import dataclasses
+
 import numpy as np
 import pytest
 import torch
@@ -27,6 +29,7 @@ from parity import CacheCase, assert_parity, to64
 pytestmark = pytest.mark.gpu
 
 W_PROD = synth.workload("production_b64_n4096_bf16")
+W_PROD16 = dataclasses.replace(W_PROD, name="production_b64_n4096_fp16", dims=W_PROD.dims.with_(dtype="fp16"))
 POS_VALS = O.e4m3_values()[:0x7F]  # codes 0x00 .. 0x7E, increasing
 
 
@@ -87,11 +90,11 @@ def append_fp8(d, h, w, seq_idx, pos, bt, num_pages):
     return pool.cpu().numpy()
 
 
-def test_append_fp8_bytes_exact_on_exact_rows():
+@pytest.mark.parametrize("w", [W_PROD, W_PROD16], ids=["bf16", "fp16"])
+def test_append_fp8_bytes_exact_on_exact_rows(w):
     """Scaled one-hot hidden states: the rows are weight columns times a power of two, exact on
     both sides, so bytes and scales must agree bit for bit (RoPE at position 0 for all parts,
     and the latent part at any position)."""
-    w = W_PROD
     d = w.dims
     W = synth.weights(w)
     T = 12
@@ -169,9 +172,9 @@ def test_append_fp8_bad_page_is_reported_and_skipped():
     assert changed == [(0, 3)]
 
 
+@pytest.mark.parametrize("w", [W_PROD, W_PROD16], ids=["bf16", "fp16"])
 @pytest.mark.parametrize("scale", [1.0, 300.0], ids=["pages_law", "peaked"])
-def test_decode_fp8_ragged_paged(scale):
-    w = W_PROD
+def test_decode_fp8_ragged_paged(w, scale):
     d = w.dims
     lens = np.array([1, 2, 63, 64, 65, 129, 1000, 4097])
     case = CacheCase(w, cached=lens, paging="shuffled", spare_tokens=0, device="cpu")
