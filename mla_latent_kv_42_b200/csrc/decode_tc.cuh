@@ -84,10 +84,11 @@ struct Ctrl {
   uint64_t rope_done, q_free;
   uint64_t s_full[2], p_free;
   // Local barriers.
-  uint64_t xm_full, xm_free;  // exchange of per-thread partial maxima / sums among the softmax warps
+  uint64_t mx_full[2][2];  // exchanges among the softmax warps: [head group][buffer xm, xh]
   uint64_t f8_qk[2][2], f8_pv[2][2], f8_rope;  // FP8: an e4m3 box has landed in this CTA
   uint64_t drain;
-  float xm[2][128];          // [column half][TMEM lane]
+  float xm[2][128];          // [column half][TMEM lane]: partial maxima or sums
+  __nv_bfloat16 xh[2][128];  // the same, for maxima only (the second buffer)
   uint32_t tmem_slot;
   int abort_flag;
 };
@@ -279,8 +280,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(F8 ? dec::kThreadsF8
     mbar_init(bar(ctl->rope_done), 1);
     mbar_init(bar(ctl->q_free), 1);
     mbar_init(bar(ctl->p_free), 1);
-    mbar_init(bar(ctl->xm_full), kSoftWarps);
-    mbar_init(bar(ctl->xm_free), kSoftWarps);
+    for (int g2 = 0; g2 < 2; ++g2)
+      for (int b2 = 0; b2 < 2; ++b2) mbar_init(bar(ctl->mx_full[g2][b2]), kSoftWarps / 2);
     mbar_init(bar(ctl->drain), 2);
     for (int s = 0; s < 2; ++s)
       for (int h = 0; h < 2; ++h) {
@@ -685,23 +686,38 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(F8 ? dec::kThreadsF8
       const uint32_t lane_base = (uint32_t)(qd * 32) << 16;
       const uint32_t p_row = data_u32 + kPOff + g * kChunk + (h >> 3) * 1024 + (h & 7) * 128;
       uint8_t* const p_row_ptr = data + (p_row - data_u32);
-      uint32_t xc = 0;  // exchanges so far (phase of xm_full / xm_free)
       // Exchange one value among the four threads of a head; returns the four in a fixed order
-      // (page 0 half 0, page 0 half 1, page 1 half 0, page 1 half 1).
-      auto exchange = [&](float v, float (&out)[4]) {
-        if (xc > 0 && !wwait(ctl->xm_free, (xc - 1) & 1)) return false;
-        ctl->xm[ch][lt] = v;
-        __syncwarp();
-        if (lane == 0) mbar_arrive(bar(ctl->xm_full));
-        if (!wwait(ctl->xm_full, xc & 1)) return false;
+      // (page 0 half 0, page 0 half 1, page 1 half 0, page 1 half 1). A head's four threads sit
+      // in the four warps of one parity, so each group of four warps exchanges on barriers of its
+      // own: one barrier round per exchange. Successive maxima alternate between two buffers, the
+      // fp32 xm and the bf16 xh (a reference maximum need not be exact, only the same for the
+      // four threads), so that a writer never waits for the readers of the exchange before: they
+      // have arrived at the one in between. The denominator exchange at an item's end is fp32
+      // (xm); the tile before it is complete (its O MMAs have read every thread's P, which each
+      // thread writes after reading that tile's maxima), and the next maximum goes to xh.
+      const int xg = warp & 1;
+      uint32_t xuse0 = 0, xuse1 = 0;  // completed exchanges on xm / xh (their barriers' phases)
+      int xnext = 0;                  // buffer of the next maximum: 0 = xm, 1 = xh
+      auto exchange = [&](float v, int buf, float (&out)[4]) {
         const int l0 = lt & 63;
-        out[0] = ctl->xm[0][l0];
-        out[1] = ctl->xm[1][l0];
-        out[2] = ctl->xm[0][l0 + 64];
-        out[3] = ctl->xm[1][l0 + 64];
+        if (buf == 0) ctl->xm[ch][lt] = v;
+        else ctl->xh[ch][lt] = __float2bfloat16_rn(v);
         __syncwarp();
-        if (lane == 0) mbar_arrive(bar(ctl->xm_free));
-        ++xc;
+        if (lane == 0) mbar_arrive(bar(ctl->mx_full[xg][buf]));
+        if (!wwait(ctl->mx_full[xg][buf], (buf == 0 ? xuse0 : xuse1) & 1)) return false;
+        if (buf == 0) {
+          ++xuse0;
+          out[0] = ctl->xm[0][l0];
+          out[1] = ctl->xm[1][l0];
+          out[2] = ctl->xm[0][l0 + 64];
+          out[3] = ctl->xm[1][l0 + 64];
+        } else {
+          ++xuse1;
+          out[0] = __bfloat162float(ctl->xh[0][l0]);
+          out[1] = __bfloat162float(ctl->xh[1][l0]);
+          out[2] = __bfloat162float(ctl->xh[0][l0 + 64]);
+          out[3] = __bfloat162float(ctl->xh[1][l0 + 64]);
+        }
         return true;
       };
       Cursor c;
@@ -739,8 +755,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(F8 ? dec::kThreadsF8
         float four[4];
         if (!exchange(fmaxf(fmaxf(fmaxf(mxs[0], mxs[1]), fmaxf(mxs[2], mxs[3])),
                             fmaxf(fmaxf(mxs[4], mxs[5]), fmaxf(mxs[6], mxs[7]))),
-                      four))
+                      xnext, four))
           break;
+        xnext ^= 1;
         const float mx = fmaxf(fmaxf(four[0], four[1]), fmaxf(four[2], four[3])) * p.scale_log2;
         float alpha = 1.f;
         if (mx > m_ref + kLazy) {
@@ -796,7 +813,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(F8 ? dec::kThreadsF8
         if (c.last()) {  // ---- epilogue of the item: O / l for this thread's head and columns
           if (!wwait(ctl->p_free, ti & 1)) break;  // the last O MMAs are done
           tc_fence_after();
-          if (!exchange(lsum, four)) break;
+          if (!exchange(lsum, 0, four)) break;
+          xnext = 1;
           const float l = (four[0] + four[1]) + (four[2] + four[3]);
           const float inv = l > 0.f ? 1.f / l : 0.f;
           const float lse = l > 0.f ? (m_ref + log2f(l)) * kLn2 : -INFINITY;
