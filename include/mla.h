@@ -266,9 +266,12 @@ int mla_append_kv_fp8(const mla_dims* dims, const void* h, const void* w_dkv_kr,
 
 /*
  * mla_decode_attention_fp8 — mla_decode_attention over an FP8 cache: the attention of every
- * sequence and head over the rows the cache stands for. The bytes are converted to the element
- * type in shared memory (each value times its token's scale, in float32, rounded once) before
- * the tensor-core products, which are those of mla_decode_attention. Arguments, outputs,
+ * sequence and head over the rows the cache stands for. Its tensor-core products run in fp16
+ * with fp32 accumulation: each cached value is converted in shared memory as its e4m3 value
+ * (exact in fp16) times its token's scale rounded to fp16, the product rounded once to fp16; the
+ * queries are rounded to fp16 and the softmax weights are fp16. So the queries and the values the
+ * cache stands for must lie within fp16's range (|x| < 65504), and scales below 2^-14 (parts
+ * whose largest magnitude is below about 0.027) lose relative precision. Arguments, outputs,
  * checks and error behaviour as mla_decode_attention, with pool the FP8 pages; ws at least
  * mla_workspace_size(dims, MLA_CALL_DECODE_ATTENTION_FP8, B, max_seq_len) bytes.
  */

@@ -27,6 +27,8 @@
 // spans pairs is merged afterwards by log-sum-exp in a fixed order.
 #pragma once
 
+#include <type_traits>
+
 #include "fp8.cuh"
 #include "tc_common.cuh"
 
@@ -86,6 +88,7 @@ struct Ctrl {
   // Local barriers.
   uint64_t mx_full[2][2];  // exchanges among the softmax warps: [head group][buffer xm, xh]
   uint64_t f8_qk[2][2], f8_pv[2][2], f8_rope;  // FP8: an e4m3 box has landed in this CTA
+  uint64_t f8_q;                               // FP8: this CTA's queries have landed
   uint64_t drain;
   float xm[2][128];          // [column half][TMEM lane]: partial maxima or sums
   __nv_bfloat16 xh[2][128];  // the same, for maxima only (the second buffer)
@@ -260,6 +263,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(F8 ? dec::kThreadsF8
   auto bar = [&](uint64_t& b) { return smem_u32(&b); };
   auto lead = [&](uint64_t& b) { return mapa(smem_u32(&b), 0u); };  // the barrier in rank 0
   constexpr bool kBf16 = IsBf16<T>::value;
+  // With the FP8 cache the products run in fp16: a cached value is then one hardware conversion
+  // and one fp16 multiply by its scale; the queries are converted once per sequence and P is fp16.
+  constexpr bool kMmaBf16 = kBf16 && !F8;
+  using PT = std::conditional_t<F8, __half, T>;
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < 2; ++s) {
@@ -289,6 +296,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(F8 ? dec::kThreadsF8
         mbar_init(bar(ctl->f8_pv[s][h]), 1);
       }
     mbar_init(bar(ctl->f8_rope), 1);
+    mbar_init(bar(ctl->f8_q), 1);
     ctl->abort_flag = 0;
     fence_mbar_init();
   }
@@ -352,8 +360,13 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(F8 ? dec::kThreadsF8
           const int page = nv > 0 ? btb[page_idx] : 0;
           if (c.first()) {  // this CTA's 64 heads of the sequence's queries, after the last S MMA of the item before
             if (!wait(ctl->q_free, (c.ii & 1) ^ 1)) break;
-            mbar_arrive_expect_tx_cl(lead(ctl->q_full), 9 * kChunk);
-            tma_load_3d_pair(data_u32 + kQOff, &maps.q9, lead(ctl->q_full), 0, b * p.n_h + 64 * (int)rank, 0);
+            if constexpr (F8) {  // the converting warps turn them into fp16 and publish them
+              mbar_arrive_expect_tx(bar(ctl->f8_q), 9 * kChunk);
+              tma_load_3d(data_u32 + kQOff, &maps.q9, bar(ctl->f8_q), 0, b * p.n_h + 64 * (int)rank, 0);
+            } else {
+              mbar_arrive_expect_tx_cl(lead(ctl->q_full), 9 * kChunk);
+              tma_load_3d_pair(data_u32 + kQOff, &maps.q9, lead(ctl->q_full), 0, b * p.n_h + 64 * (int)rank, 0);
+            }
           }
           if (!wait(ctl->rope_done, (c.ti & 1) ^ 1)) break;
           if constexpr (F8) {
@@ -446,8 +459,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(F8 ? dec::kThreadsF8
       // (16-byte units: a K-step of 16 elements is +2 along a K-major row and +128, i.e. 16 rows,
       // down an MN-major operand).
       if (rank == 0 && lane == 0) {
-        constexpr uint32_t idesc_qk = idesc_f16(128, kTile, kBf16, false, false);
-        constexpr uint32_t idesc_pv = idesc_f16(128, 256, kBf16, false, true);
+        constexpr uint32_t idesc_qk = idesc_f16(128, kTile, kMmaBf16, false, false);
+        constexpr uint32_t idesc_pv = idesc_f16(128, 256, kMmaBf16, false, true);
         constexpr uint32_t hi = desc_sw128_hi(1024);
         constexpr uint32_t kChunkD = kChunk >> 4, kSetD = kSetBytes >> 4;
         const uint32_t b_qk_full = bar(ctl->qk_full[0][0]), b_pv_full = bar(ctl->pv_full[0][0]);
@@ -536,7 +549,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(F8 ? dec::kThreadsF8
       }
       __syncwarp();
     } else if (F8 && warp >= kConvWarp0) {
-      // ---------------------------------------------------------------- FP8: e4m3 boxes -> chunks
+      // ---------------------------------------------------------------- FP8: e4m3 boxes -> fp16 chunks
       // Each box (64 slot rows, unswizzled, rows of 256, 128 or 64 bytes) lies in the upper half
       // of the chunks it becomes: a latent group (4 chunks), a pair (2 chunks), the rope chunk.
       // The four warps convert it in place, each value times its token's scale in float32: first
@@ -558,9 +571,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(F8 ? dec::kThreadsF8
         return __ldg(reinterpret_cast<const float2*>(reinterpret_cast<const uint8_t*>(scale_base) +
                                                      (size_t)page * kF8Page) + pr);
       };
-      auto put16 = [&](uint32_t dst, int v, const uint4& in, float sc) {
+      auto put16 = [&](uint32_t dst, int v, const uint4& in, __half2 sc) {
         uint4 o0, o1;
-        dequant16<T>(in, sc, o0, o1);
+        dequant16_f16(in, sc, o0, o1);
         const uint32_t rb = dst + (v >> 2) * kChunk + row * 128;
         const uint32_t u = 2u * (v & 3);
         sts128(rb + ((u ^ sw) << 4), o0);
@@ -577,7 +590,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(F8 ? dec::kThreadsF8
         if (ct == 0) mbar_arrive_cl(lead(full));
       };
       // latent group: 4 chunks from dst, box of 256-byte rows at dst + 2 chunks
-      auto conv_group = [&](uint32_t dst, float sc) {
+      auto conv_group = [&](uint32_t dst, __half2 sc) {
         const uint32_t box = dst + 2 * kChunk + row * 256;
 #pragma unroll
         for (int j = 0; j < 4; ++j) {
@@ -592,7 +605,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(F8 ? dec::kThreadsF8
         for (int j = 0; j < 4; ++j) put16(dst, 8 + 4 * half + ((j + row) & 3), keep[j], sc);
       };
       // pair: 2 chunks from dst, box of 128-byte rows at dst + 1 chunk
-      auto conv_pair = [&](uint32_t dst, float sc) {
+      auto conv_pair = [&](uint32_t dst, __half2 sc) {
         const uint32_t box = dst + kChunk + row * 128;
 #pragma unroll
         for (int j = 0; j < 2; ++j) {
@@ -607,7 +620,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(F8 ? dec::kThreadsF8
         for (int j = 0; j < 2; ++j) put16(dst, 4 + 2 * half + ((j + row) & 1), keep[j], sc);
       };
       // rope chunk, box of 64-byte rows in its upper half: output rows 32-63 overwrite the box
-      auto conv_rope = [&](uint32_t dst, float sr) {
+      auto conv_rope = [&](uint32_t dst, __half2 sr) {
         const uint32_t box = dst + kChunk / 2 + row * 64;
         uint4 keep[2];
 #pragma unroll
@@ -616,15 +629,36 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(F8 ? dec::kThreadsF8
 #pragma unroll
         for (int j = 0; j < 2; ++j) put16(dst, 2 * half + j, keep[j], sr);
       };
+      // an item's queries: bf16 -> fp16 in place, each thread its own 16-byte units
+      auto conv_q = [&](const Cursor& c) {
+        if (!cwait(ctl->f8_q, c.ii & 1)) return false;
+        if constexpr (kBf16) {
+          for (int u = ct; u < 9 * kChunk / 16; u += 128) {
+            const uint32_t a = data_u32 + kQOff + 16 * u;
+            const uint4 v = lds128(a);
+            uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+              const float2 f = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&w[e]));
+              const __half2 hv = __floats2half2_rn(f.x, f.y);
+              w[e] = *reinterpret_cast<const uint32_t*>(&hv);
+            }
+            sts128(a, make_uint4(w[0], w[1], w[2], w[3]));
+          }
+        }
+        publish(ctl->q_full);
+        return true;
+      };
       // the own page of a tile: rope, then latent groups 0 and 1
       auto conv_own = [&](const Cursor& c, float2 sc) {
         const int s = c.ti & 1;
+        const __half2 hc = __float2half2_rn(sc.x), hr = __float2half2_rn(sc.y);
         if (!cwait(ctl->f8_rope, c.ti & 1)) return false;
-        conv_rope(data_u32 + kRopeOff, sc.y);
+        conv_rope(data_u32 + kRopeOff, hr);
         publish(ctl->rope_full);
         for (int h = 0; h < 2; ++h) {
           if (!cwait(ctl->f8_qk[s][h], (c.ti >> 1) & 1)) return false;
-          conv_group(set_u32 + s * kSetBytes + 4 * h * kChunk, sc.x);
+          conv_group(set_u32 + s * kSetBytes + 4 * h * kChunk, hc);
           publish(ctl->qk_full[s][h]);
         }
         return true;
@@ -635,7 +669,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(F8 ? dec::kThreadsF8
         for (int j = 0; j < 2; ++j) {
           const int pr = 2 * j + g;
           if (!cwait(ctl->f8_pv[s][j], (c.ti >> 1) & 1)) return false;
-          conv_pair(set_u32 + s * kSetBytes + 2 * pr * kChunk, sc);
+          conv_pair(set_u32 + s * kSetBytes + 2 * pr * kChunk, __float2half2_rn(sc));
           publish(ctl->pv_full[s][pr]);
         }
         return true;
@@ -669,7 +703,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(F8 ? dec::kThreadsF8
             if (nx.first()) Ln = p.seq_lens[nx.item.b];
             nxt = tile_scales(nx, Ln);
           }
-          if (!conv_own(c, cur.own) || !conv_pairs(c, cur.pair)) break;
+          if ((c.first() && !conv_q(c)) || !conv_own(c, cur.own) || !conv_pairs(c, cur.pair)) break;
           c = nx;
           L = Ln;
           cur = nxt;
@@ -796,9 +830,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(F8 ? dec::kThreadsF8
 #pragma unroll
           for (int e = 0; e < 4; ++e) {
             const int k = 8 * u4 + 2 * e;
-            const typename Pack<T>::T2 pr2 = Pack<T>::make(ex2_approx(fmaf(u2f(sr[k]), p.scale_log2, -m_ref)),
+            const typename Pack<PT>::T2 pr2 = Pack<PT>::make(ex2_approx(fmaf(u2f(sr[k]), p.scale_log2, -m_ref)),
                                                            ex2_approx(fmaf(u2f(sr[k + 1]), p.scale_log2, -m_ref)));
-            const float2 back = Pack<T>::f2(pr2);
+            const float2 back = Pack<PT>::f2(pr2);
             sums[e] += back.x + back.y;
             w[e] = *reinterpret_cast<const uint32_t*>(&pr2);
           }

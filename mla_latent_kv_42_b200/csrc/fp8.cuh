@@ -88,18 +88,16 @@ __global__ void __launch_bounds__(256) k_quant_fp8(const T* __restrict__ rows, c
   if (lane == 0) *reinterpret_cast<float2*>(pg + (long)page_size * D + 8 * row) = make_float2(sc, sr);
 }
 
-// 16 e4m3 values (16 bytes, element order) times `s` in float32, rounded once to bf16 / fp16:
-// two 16-byte groups of eight elements.
-template <typename T>
-__device__ __forceinline__ void dequant16(const uint4& in, float s, uint4& out0, uint4& out1) {
+// 16 e4m3 values (16 bytes, element order) as fp16 times the fp16 scale `s` (the e4m3 value is
+// exact in fp16; the product is rounded once): two 16-byte groups of eight elements.
+__device__ __forceinline__ void dequant16_f16(const uint4& in, __half2 s, uint4& out0, uint4& out1) {
   const uint32_t w[4] = {in.x, in.y, in.z, in.w};
   uint32_t o[8];
 #pragma unroll
   for (int e = 0; e < 8; ++e) {
     const __nv_fp8x2_storage_t two = (__nv_fp8x2_storage_t)(w[e >> 1] >> (16 * (e & 1)));
     const __half2_raw hr = __nv_cvt_fp8x2_to_halfraw2(two, __NV_E4M3);
-    const float2 f = __half22float2(*reinterpret_cast<const __half2*>(&hr));
-    const typename Pack<T>::T2 v = Pack<T>::make(f.x * s, f.y * s);
+    const __half2 v = __hmul2(*reinterpret_cast<const __half2*>(&hr), s);
     o[e] = *reinterpret_cast<const uint32_t*>(&v);
   }
   out0 = make_uint4(o[0], o[1], o[2], o[3]);

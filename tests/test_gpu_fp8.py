@@ -10,10 +10,9 @@ summary page ("The Model"): e4m3 bytes with two float32 scales per token, max|pa
 - With general hidden states, the rows the FP8 cache stands for are compared with the oracle's
   rows at the parity tolerance, and every nonzero part reaches code 448 exactly.
 - The decode runs over caches whose bytes the oracle wrote (on the host), shuffled pages, ragged
-  lengths and tail pages, against the oracle's attention over the rows the cache stands for,
-  each rounded once to the element type: the decode converts every value (times its scale, in
-  float32) to the element type before the tensor-core products, as the 16-bit cache holds
-  element-type rows.
+  lengths and tail pages, against the oracle's attention over the rows the cache stands for as
+  the decode forms them: its tensor-core products run in fp16, each e4m3 value (exact in fp16)
+  times its token's scale rounded to fp16, the product rounded once to fp16.
 """
 import dataclasses
 
@@ -58,8 +57,8 @@ def page_views(pool: np.ndarray, d):
 
 def fp8_pool_from_rows(rows64: np.ndarray, cached, bt, num_pages, d):
     """FP8 pages holding each sequence's rows (quantised by the oracle), and the rows they stand
-    for rounded to the element type; bytes of unused slots are the e4m3 NaN code and their scales
-    NaN, so that a read past a sequence shows."""
+    for as the decode forms them (fp16 value times fp16 scale, rounded to fp16); bytes of unused
+    slots are the e4m3 NaN code and their scales NaN, so that a read past a sequence shows."""
     vals, sc = O.quantize_rows_fp8(rows64, d.d_c)
     codes = codes_of(vals)
     pool = np.full((num_pages, M.fp8_page_bytes(d)), 0x7F, dtype=np.uint8)
@@ -73,7 +72,8 @@ def fp8_pool_from_rows(rows64: np.ndarray, cached, bt, num_pages, d):
             scales[pg, r] = sc[off + j]
         off += int(n)
     pool[:, d.page_size * d.D:] = scales.view(np.uint8).reshape(num_pages, -1)
-    return pool, O.as64(synth.to_storage(O.dequantize_rows_fp8(vals, sc, d.d_c), d))
+    sc16 = sc.astype(np.float16).astype(np.float64)  # the scale rounded to fp16
+    return pool, O.dequantize_rows_fp8(vals, sc16, d.d_c).astype(np.float16).astype(np.float64)
 
 
 def test_page_bytes_and_support():
@@ -215,8 +215,9 @@ def test_decode_fp8_full_load_sampled():
 
 
 def test_decode_fp8_matches_bf16_path_on_dequantised_rows():
-    """The FP8 decode equals the 16-bit decode run over the rows the FP8 cache stands for
-    (rounded to bf16 as the converter rounds them) up to the order of summation."""
+    """The FP8 decode agrees with the 16-bit decode run over the rows the FP8 cache stands for:
+    the one forms them in fp16, the other reads them rounded to bf16, so they differ by that
+    rounding (half a bf16 step, 2^-9 relative, per value) and the order of summation."""
     w = W_PROD
     d = w.dims
     lens = np.array([5, 300, 2000])
@@ -230,8 +231,8 @@ def test_decode_fp8_matches_bf16_path_on_dequantised_rows():
     pool16 = synth.paged_pool(rows16.cuda(), lens, case.bt_np, case.num_pages, d.page_size, fill=0.0)
     o16, l16 = M.decode_attention(d, q, pool16, bt, sl, int(lens.max()))
     assert M.read_device_status() == 0
-    assert_parity(to64(o8), to64(o16), "fp8 vs bf16 over the same rows", max_tol=1e-2, mean_tol=5e-4)
-    torch.testing.assert_close(l8, l16, rtol=0, atol=1e-3)
+    assert_parity(to64(o8), to64(o16), "fp8 vs bf16 over the same rows", max_tol=1e-2, mean_tol=1e-3)
+    torch.testing.assert_close(l8, l16, rtol=0, atol=1e-2)
 
 
 def test_decode_fp8_bad_seq_len():
