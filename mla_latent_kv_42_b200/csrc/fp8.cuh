@@ -6,6 +6,10 @@
 // page_size float2 scales (s_c, s_r). A byte is the nearest e4m3 value (ties to even, saturated
 // to +-448) of the element-type value divided by its part's scale max|part| / 448 in float32
 // (1 for an all-zero part), so the largest magnitude of each part lands on 448.
+//
+// Writer: k_quant_fp8 below, after the append GEMM has staged the element-type rows. Reader: the
+// decode kernel of decode_tc.cuh instantiated with F8 = true, where four more warps convert each
+// landed e4m3 box in place to fp16 (dequant16_f16) and the products run as fp16 MMAs.
 #pragma once
 
 #include <cuda_fp8.h>
