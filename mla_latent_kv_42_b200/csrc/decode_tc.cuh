@@ -961,10 +961,19 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(F8 ? dec::kThreadsF8
 // keeps the total (B x tiles of max_seq_len) within int32.
 __global__ void __launch_bounds__(1024) k_decode_plan(const int* __restrict__ seq_lens, const int* __restrict__ bt,
                                                       int B, int max_pages, int num_pages, int max_seq_len, int C,
-                                                      int* __restrict__ tile_prefix, int* __restrict__ seq_pairs,
+                                                      int caller_inputs, int* __restrict__ tile_prefix,
+                                                      int* __restrict__ seq_pairs,
                                                       int* __restrict__ pair_start) {
-  griddep_wait();
+  // When the lengths and block tables come from the caller (caller_inputs: no kernel of this
+  // call wrote them), up to kPlanEarlySeqs sequences are checked, their tile counts kept in shared
+  // memory, before the wait for the kernel before, which may still be using the workspace this
+  // kernel writes. (Prefill's per-token tables are written by the kernel before: it waits first.)
+  constexpr int kPlanEarlySeqs = 4096;
+  __shared__ int s_count[kPlanEarlySeqs];
+  const bool early = caller_inputs != 0 && B <= kPlanEarlySeqs;
+  if (!early) griddep_wait();
   if (threadIdx.x == 0) griddep_launch();
+  int* const count = early ? s_count : tile_prefix;
   __shared__ int warp_total[32];
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   // Tiles of each sequence (0 for a rejected one), a half-warp per sequence, 64 sequences per
@@ -992,15 +1001,16 @@ __global__ void __launch_bounds__(1024) k_decode_plan(const int* __restrict__ se
       ok = false;
       if (sub == 0) record_error(MLA_ERR_BAD_PAGE);
     }
-    if (b < B && sub == 0) tile_prefix[b] = ok ? (int)(((long)L + dec::kTile - 1) / dec::kTile) : 0;
+    if (b < B && sub == 0) count[b] = ok ? (int)(((long)L + dec::kTile - 1) / dec::kTile) : 0;
   }
   __syncthreads();
+  if (early) griddep_wait();
   // exclusive scan: thread tid sums the counts of sequences [tid * per, tid * per + per), then a
   // two-level warp-shuffle scan over the 1024 thread sums
   const int per = (B + 1023) / 1024;
   const int b0 = min(B, tid * per), b1 = min(B, b0 + per);
   int sum = 0;
-  for (int b = b0; b < b1; ++b) sum += tile_prefix[b];
+  for (int b = b0; b < b1; ++b) sum += count[b];
   int incl = sum;
 #pragma unroll
   for (int o = 1; o < 32; o <<= 1) {
@@ -1024,7 +1034,7 @@ __global__ void __launch_bounds__(1024) k_decode_plan(const int* __restrict__ se
   const long T_ = warp_total[31];
   int run = incl - sum + (warp > 0 ? warp_total[warp - 1] : 0);
   for (int b = b0; b < b1; ++b) {
-    const int n = tile_prefix[b];
+    const int n = count[b];
     tile_prefix[b] = run;
     if (n > 0) {
       const int c0 = cluster_of(run, T_, C), c1 = cluster_of(run + n - 1, T_, C);

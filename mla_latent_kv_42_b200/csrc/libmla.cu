@@ -242,10 +242,12 @@ size_t ws_decode(const mla_dims* d, int B, int max_seq_len) {
   return align256(bh * p.n_splits * d->d_c * 4) + align256(bh * p.n_splits * 4);
 }
 
+// caller_inputs: seq_lens and bt come from the caller (no kernel of this call wrote them), so the
+// planner may read them before waiting for the kernel before it.
 template <typename T, bool F8 = false>
 int decode_tc_impl(const mla_dims* d, const void* q, const void* pool, int32_t num_pages, const int32_t* bt,
                    int32_t max_pages, const int32_t* seq_lens, int32_t B, int32_t max_seq_len, void* o_lat,
-                   float* lse_out, void* ws, cudaStream_t st, int32_t& launches) {
+                   float* lse_out, void* ws, cudaStream_t st, int32_t& launches, bool caller_inputs) {
   const int C = decode_clusters();
   if (!decode_tc_set_smem<T, F8>()) return MLA_ERR_CUDA;
   Carve c{static_cast<char*>(ws)};
@@ -272,7 +274,7 @@ int decode_tc_impl(const mla_dims* d, const void* q, const void* pool, int32_t n
                               (uint64_t)B + C))
     return MLA_ERR_CUDA;
   if (launch_pdl(tc::k_decode_plan, dim3(1), dim3(1024), 0, st, seq_lens, bt, (int)B, (int)max_pages, (int)num_pages,
-                 (int)max_seq_len, C, prefix, seq_pairs, pair_start) != cudaSuccess)
+                 (int)max_seq_len, C, (int)caller_inputs, prefix, seq_pairs, pair_start) != cudaSuccess)
     return MLA_ERR_CUDA;
   tc::DecodeTcParams p;
   p.bt = bt;
@@ -333,10 +335,10 @@ void launch_decode_simt(const mla_dims* d, const DecodePlan& p, const void* q, c
 template <typename T>
 int decode_impl(const mla_dims* d, const void* q, const void* pool, int32_t num_pages, const int32_t* bt,
                 int32_t max_pages, const int32_t* seq_lens, int32_t B, int32_t max_seq_len, void* o_lat,
-                float* lse_out, void* ws, cudaStream_t st, int32_t& launches) {
+                float* lse_out, void* ws, cudaStream_t st, int32_t& launches, bool caller_inputs) {
   if (decode_tc_eligible(d))
     return decode_tc_impl<T>(d, q, pool, num_pages, bt, max_pages, seq_lens, B, max_seq_len, o_lat, lse_out, ws, st,
-                             launches);
+                             launches, caller_inputs);
   const DecodePlan p = plan_decode(d, B, max_seq_len);
   const size_t bh = (size_t)B * d->n_heads;
   float* o_part = nullptr;
@@ -431,7 +433,8 @@ int prefill_impl(const mla_dims* d, const void* q, const void* pool, int32_t num
     ++n;
     const int r = decode_impl<T>(d, static_cast<const char*>(q) + g0 * q_row, pool, num_pages, item_bt, item_pages,
                                  item_len, g, max_seq_len, static_cast<char*>(o_lat) + g0 * o_row,
-                                 lse_out != nullptr ? lse_out + (size_t)g0 * d->n_heads : nullptr, dec_ws, st, n);
+                                 lse_out != nullptr ? lse_out + (size_t)g0 * d->n_heads : nullptr, dec_ws, st, n,
+                                 false);
     if (r != MLA_OK) return r;
   }
   return finish_launches(MLA_CALL_PREFILL_ATTENTION, n);
@@ -664,9 +667,9 @@ int mla_decode_attention(const mla_dims* dims, const void* q, const void* pool, 
   int32_t n = 0;
   r = dims->dtype == MLA_BF16
           ? decode_impl<__nv_bfloat16>(dims, q, pool, num_pages, block_table, max_pages, seq_lens, B, max_seq_len,
-                                       o_lat, lse_out, ws, st, n)
+                                       o_lat, lse_out, ws, st, n, true)
           : decode_impl<__half>(dims, q, pool, num_pages, block_table, max_pages, seq_lens, B, max_seq_len, o_lat,
-                                lse_out, ws, st, n);
+                                lse_out, ws, st, n, true);
   if (r != MLA_OK) return r;
   return finish_launches(MLA_CALL_DECODE_ATTENTION, n);
 }
@@ -730,9 +733,9 @@ int mla_decode_attention_fp8(const mla_dims* dims, const void* q, const void* po
   int32_t n = 0;
   r = dims->dtype == MLA_BF16
           ? decode_tc_impl<__nv_bfloat16, true>(dims, q, pool, num_pages, block_table, max_pages, seq_lens, B,
-                                                max_seq_len, o_lat, lse_out, ws, st, n)
+                                                max_seq_len, o_lat, lse_out, ws, st, n, true)
           : decode_tc_impl<__half, true>(dims, q, pool, num_pages, block_table, max_pages, seq_lens, B, max_seq_len,
-                                         o_lat, lse_out, ws, st, n);
+                                         o_lat, lse_out, ws, st, n, true);
   if (r != MLA_OK) return r;
   return finish_launches(MLA_CALL_DECODE_ATTENTION_FP8, n);
 }
