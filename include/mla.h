@@ -244,6 +244,8 @@ int mla_layer_step_small(const mla_dims* dims, const void* h, const void* w_dkv_
  *   c_j = s_c * e4m3(row[0 .. d_c)),   k^R_j = s_r * e4m3(row[d_c .. d_c + d_rope)),
  * with s = max|part| / 448 in float32 (1 for an all-zero part) and each byte the nearest e4m3
  * value (ties to even) of the element-type value divided by s in float32, saturated to +-448.
+ * The FP8 cache serves decode steps (mla_append_kv_fp8, mla_decode_attention_fp8);
+ * mla_prefill_attention and mla_layer_step_small read the element-type cache only.
  */
 int64_t mla_fp8_page_bytes(const mla_dims* dims); /* negative on invalid dims */
 
