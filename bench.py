@@ -370,7 +370,7 @@ def run_mla(args):
     time.sleep(0.3)
 
     # ---- timed region: K steps, device time, barrier + synchronize on both sides. The K-step
-    # region is repeated (at least 3 times, until about half a second has been timed, so that the
+    # region is repeated (at least 3 times, until about a second has been timed, so that the
     # clock sampler sees it) and the median repetition is reported; every rank runs the same number
     # of repetitions (the count is agreed from rank 0's first one).
     # With --flush-l2 every step runs cold: a 256 MiB write (twice L2) precedes it, outside its
@@ -586,7 +586,7 @@ def main():
     ap.add_argument("--workload", default=DEFAULT_WORKLOAD)
     ap.add_argument("--impl", choices=["mla", "reference"], default="mla")
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--min-timed-s", type=float, default=0.5,
+    ap.add_argument("--min-timed-s", type=float, default=1.0,
                     help="repeat the K-step timed region until this many seconds are timed (at least 3 times)")
     ap.add_argument("--max-reps", type=int, default=1000)
     ap.add_argument("--flush-l2", action="store_true", help="write 256 MiB before every timed step (cold L2)")
