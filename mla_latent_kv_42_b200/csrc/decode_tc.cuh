@@ -129,6 +129,7 @@ struct DecodeTcMaps {
   CUtensorMap page1, page2, page4, q9;
   CUtensorMap f8_256, f8_128, f8_64;
   CUtensorMap o_lat, o_part;  // outputs as (512 columns, n_h heads, rows), 64-byte x 32-head boxes
+  CUtensorMap o_lat_h, o_part_h;  // the same with 32-byte x 32-head boxes, unswizzled
 };
 
 // Tiles [t0, t1) of sequence b handled by this pair (n_b = tiles of the sequence).
@@ -860,22 +861,42 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(F8 ? dec::kThreadsF8
           // shared memory: each lane puts its head's segment in row `lane` of a 2 KB box in the
           // 64-byte swizzle (16-byte chunk c of row r at c ^ (r/2 % 4), conflict-free), and lane 0
           // stores the 32 x 64-byte box with one TMA store, which heads past n_h fall outside of.
-          // Mid-range the box is the warp's 2 KB of the P buffer (free: the last O MMAs are done),
-          // reused once the copy engine has read it; at the pair's last item every round gets a
-          // box of its own in the latent sets, which no tile needs any more, so nothing waits.
+          // Mid-range the warp's 2 KB of the P buffer (free: the last O MMAs are done) holds two
+          // 1 KB boxes of 32 bytes per head, used in turn by half rounds, so a box waits only for
+          // the store two half rounds back; at the pair's last item every round gets a 2 KB box
+          // of its own in the latent sets, which no tile needs any more, so nothing waits.
           const bool last_item = c.it.g >= c.it.g_end;
           const uint32_t wsw = (lane >> 1) & 3;
           const int head0 = 64 * (int)rank + 32 * (qd & 1);
           int round = 0;
           auto stage_store = [&](const uint32_t (&w)[16], int col) {
-            const uint32_t stage_u32 =
-                last_item ? set_u32 + warp * 16384 + round * 2048 : data_u32 + kPOff + warp * 2048;
+            if (!last_item) {
+              // mid-range: two half rounds of 32 bytes per head through the warp's two 1 KB boxes
+              // of P (unswizzled), each box reused once the store two half rounds back has read it
+#pragma unroll
+              for (int hf = 0; hf < 2; ++hf) {
+                const uint32_t box_u32 = data_u32 + kPOff + warp * 2048 + (round & 1) * 1024;
+                uint8_t* const box = data + (box_u32 - data_u32);
+                ++round;
+                if (lane == 0) bulk_wait_read<1>();
+                __syncwarp();
+                *reinterpret_cast<uint4*>(box + lane * 32) = make_uint4(w[8 * hf], w[8 * hf + 1], w[8 * hf + 2], w[8 * hf + 3]);
+                *reinterpret_cast<uint4*>(box + lane * 32 + 16) =
+                    make_uint4(w[8 * hf + 4], w[8 * hf + 5], w[8 * hf + 6], w[8 * hf + 7]);
+                fence_proxy_async_cta();
+                __syncwarp();
+                if (lane == 0) {
+                  const int c = col + hf * (whole ? 16 : 8);  // 32 bytes of columns
+                  if (whole) tma_store_3d(&maps.o_lat_h, box_u32, c, head0, it.b);
+                  else tma_store_3d(&maps.o_part_h, box_u32, c, head0, (int)slot);
+                  bulk_commit_group();
+                }
+              }
+              return;
+            }
+            const uint32_t stage_u32 = set_u32 + warp * 16384 + round * 2048;
             uint8_t* const stage = data + (stage_u32 - data_u32);
             ++round;
-            if (!last_item) {
-              if (lane == 0) bulk_wait_read<0>();  // the previous round's box has been read
-              __syncwarp();
-            }
 #pragma unroll
             for (int i2 = 0; i2 < 4; ++i2)
               *reinterpret_cast<uint4*>(stage + lane * 64 + ((i2 ^ wsw) << 4)) =

@@ -271,7 +271,12 @@ int decode_tc_impl(const mla_dims* d, const void* q, const void* pool, int32_t n
       !host::encode_heads_out(&maps.o_lat, o_lat, bf16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT16,
                               2, (uint64_t)d->n_heads, (uint64_t)B) ||
       !host::encode_heads_out(&maps.o_part, o_part, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, (uint64_t)d->n_heads,
-                              (uint64_t)B + C))
+                              (uint64_t)B + C) ||
+      !host::encode_heads_out32(&maps.o_lat_h, o_lat,
+                                bf16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2,
+                                (uint64_t)d->n_heads, (uint64_t)B) ||
+      !host::encode_heads_out32(&maps.o_part_h, o_part, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, (uint64_t)d->n_heads,
+                                (uint64_t)B + C))
     return MLA_ERR_CUDA;
   if (launch_pdl(tc::k_decode_plan, dim3(1), dim3(1024), 0, st, seq_lens, bt, (int)B, (int)max_pages, (int)num_pages,
                  (int)max_seq_len, C, (int)caller_inputs, prefix, seq_pairs, pair_start) != cudaSuccess)

@@ -127,6 +127,19 @@ inline bool encode_pages_fp8(CUtensorMap* map, const void* base, uint64_t pages,
             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+// The same view with 32-byte x 32-head boxes, unswizzled: the attention epilogue's half rounds.
+inline bool encode_heads_out32(CUtensorMap* map, void* base, CUtensorMapDataType dtype, uint32_t elem_bytes,
+                               uint64_t n_h, uint64_t rows) {
+  auto fn = tensor_map_encoder();
+  if (fn == nullptr) return false;
+  cuuint64_t dims[3] = {512, n_h, rows};
+  cuuint64_t strides[2] = {512 * elem_bytes, 512 * elem_bytes * n_h};
+  cuuint32_t box[3] = {32 / elem_bytes, 32, 1};
+  cuuint32_t es[3] = {1, 1, 1};
+  return fn(map, dtype, 3, base, dims, strides, box, es, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
+            CU_TENSOR_MAP_L2_PROMOTION_NONE, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 // 3-D view of an output [rows][n_h][512] (fp32, bf16 or fp16) as (512 columns, n_h heads, rows)
 // with boxes of 64 bytes x 32 heads x 1 row in the 64-byte swizzle: the attention epilogue's
 // staging layout. Heads past n_h fall outside the tensor and are not written by a store.
