@@ -3,6 +3,7 @@ tokens per sequence, and the algorithmic byte and flop counts the roofline divid
 against brute-force enumeration."""
 import numpy as np
 import pytest
+import torch
 
 from mla_latent_kv_42_b200 import harness, synth
 
@@ -59,3 +60,25 @@ def test_layer_work_adds_weights_once_and_projections_per_token():
     T = 8 * 128
     assert lb - ab == harness.weight_bytes(d) + 2 * T * (2 * d.d_model + d.d_c + d.d_rope)
     assert lf - af == 2 * T * (harness.weight_bytes(d) // 2)   # 2 flops per weight element per token
+
+
+def test_fp8_cache_bytes_per_token():
+    """The FP8 cache's roofline bytes: D e4m3 bytes and two float32 scales per cached token (584 B at
+    production dims, against 1152 for the 16-bit cache); queries, outputs and flops are unchanged."""
+    d = synth.PRODUCTION
+    cached = np.array([4096] * 64)
+    assert harness.cache_row_bytes(d, "fp8") == 584 and harness.cache_row_bytes(d) == 1152
+    b16, f16 = harness.attention_work(d, cached, 1)
+    b8, f8 = harness.attention_work(d, cached, 1, "fp8")
+    rows = int((cached + 1).sum())
+    assert f8 == f16 and b16 - b8 == rows * (1152 - 584)
+    lb16, _ = harness.layer_work(d, cached, 1)
+    lb8, _ = harness.layer_work(d, cached, 1, "fp8")
+    assert lb16 - lb8 == (rows + len(cached)) * (1152 - 584)  # the appended rows too
+    w = synth.workload("production_b64_n4096_fp8")
+    pages = synth.fp8_pages(w, 3)
+    assert pages.shape == (3, 64 * 584) and pages.dtype == torch.uint8
+    codes = pages[:, :64 * 576]
+    assert not ((codes & 0x7F) == 0x7F).any()  # no NaN code
+    scales = pages[:, 64 * 576:].contiguous().view(torch.float32)
+    assert (scales >= 0.5 / 448).all() and (scales <= 1.5 / 448).all()
